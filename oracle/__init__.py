@@ -1,0 +1,223 @@
+"""Python handle on the oracle (``oracle.cpp``): TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The product
+library never imports it, and it imports nothing from the product: the two
+share only the seeded input generators in ``workloads.py``.
+
+Every function is a thin ctypes marshaller around the C++ oracle, which is the
+plain fp64 restatement of the pages (see the header comment of oracle.cpp).
+"""
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+OK, INVALID, OOM, NOT_FOUND = 0, 1, 2, 3
+DTYPE_CODE = {"f32": 0, "f16": 1, "bf16": 2}
+ELEM_BYTES = {"f32": 4, "f16": 2, "bf16": 2}
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        P = C.c_void_p
+        L.orc_f16_to_f64.restype = C.c_double
+        L.orc_f16_to_f64.argtypes = [C.c_uint16]
+        L.orc_bf16_to_f64.restype = C.c_double
+        L.orc_bf16_to_f64.argtypes = [C.c_uint16]
+        L.orc_f64_to_f16.restype = C.c_uint16
+        L.orc_f64_to_f16.argtypes = [C.c_double]
+        L.orc_f64_to_bf16.restype = C.c_uint16
+        L.orc_f64_to_bf16.argtypes = [C.c_double]
+        L.orc_round_array.restype = None
+        L.orc_round_array.argtypes = [P, C.c_int64, C.c_int, P]
+        L.orc_kv_bytes.restype = C.c_uint64
+        L.orc_kv_bytes.argtypes = [C.c_int32, C.c_int64, C.c_int32, C.c_int32, C.c_int32]
+        L.orc_pool_new.restype = P
+        L.orc_pool_new.argtypes = [C.c_int32, C.c_int32]
+        L.orc_pool_delete.restype = None
+        L.orc_pool_delete.argtypes = [P]
+        L.orc_num_free.restype = C.c_int32
+        L.orc_num_free.argtypes = [P]
+        L.orc_holders.restype = C.c_int32
+        L.orc_holders.argtypes = [P, C.c_int32]
+        L.orc_alloc.restype = C.c_int
+        L.orc_alloc.argtypes = [P, C.c_int64, C.c_int32, P, P, P]
+        L.orc_free.restype = C.c_int
+        L.orc_free.argtypes = [P, C.c_int64]
+        L.orc_fork.restype = C.c_int
+        L.orc_fork.argtypes = [P, C.c_int64, C.c_int64]
+        L.orc_seq_len.restype = C.c_int64
+        L.orc_seq_len.argtypes = [P, C.c_int64]
+        L.orc_block_table.restype = C.c_int
+        L.orc_block_table.argtypes = [P, P, C.c_int32, C.c_int32, P, P]
+        L.orc_reshape_and_cache.restype = C.c_int
+        L.orc_reshape_and_cache.argtypes = [P, P, P, P, P, C.c_int64, C.c_int32, C.c_int32,
+                                            C.c_int32, C.c_int32, C.c_int32]
+        L.orc_copy_blocks.restype = C.c_int
+        L.orc_copy_blocks.argtypes = [P, P, C.c_int32, P, C.c_int32, C.c_int64]
+        L.orc_paged_decode_attention.restype = C.c_int
+        L.orc_paged_decode_attention.argtypes = [P, P, P, P, P, C.c_int32, C.c_int32, C.c_int32,
+                                                 C.c_int32, C.c_int32, C.c_int32, C.c_double,
+                                                 C.c_int, P, P, C.c_int64, C.c_int32]
+        L.orc_contiguous_attention.restype = C.c_int
+        L.orc_contiguous_attention.argtypes = [P, P, P, C.c_int64, C.c_int32, C.c_int32,
+                                               C.c_int32, C.c_double, C.c_int, P, P, C.c_int32]
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------------ numbers
+def f16_to_f64(bits):
+    return lib().orc_f16_to_f64(int(bits))
+
+
+def bf16_to_f64(bits):
+    return lib().orc_bf16_to_f64(int(bits))
+
+
+def f64_to_f16(x):
+    return lib().orc_f64_to_f16(float(x))
+
+
+def f64_to_bf16(x):
+    return lib().orc_f64_to_bf16(float(x))
+
+
+def round_to(x, dtype):
+    """Round fp64 values to the storage dtype; returns raw storage (uint16 or float32)."""
+    x = _c(x, np.float64)
+    out = np.empty(x.shape, dtype=np.float32 if dtype == "f32" else np.uint16)
+    lib().orc_round_array(_ptr(x), x.size, DTYPE_CODE[dtype], _ptr(out))
+    return out
+
+
+def kv_bytes(num_layers, seq_length, num_kv_heads, head_dim, precision_bytes):
+    return int(lib().orc_kv_bytes(num_layers, seq_length, num_kv_heads, head_dim,
+                                  precision_bytes))
+
+
+# --------------------------------------------------------------- pool model
+class Pool:
+    """The allocator restated: free stack, holder counts, per-sequence block lists."""
+
+    def __init__(self, num_blocks, block_size):
+        self.h = lib().orc_pool_new(num_blocks, block_size)
+        if not self.h:
+            raise ValueError("bad pool geometry")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def __del__(self):
+        if getattr(self, "h", None):
+            lib().orc_pool_delete(self.h)
+            self.h = None
+
+    def alloc(self, seq, n):
+        """Returns (status, slots int64[n], cow pairs int32[k, 2])."""
+        slots = np.zeros(max(n, 1), dtype=np.int64)
+        pair = np.zeros(2, dtype=np.int32)
+        ncow = np.zeros(1, dtype=np.int32)
+        st = lib().orc_alloc(self.h, seq, n, _ptr(slots), _ptr(pair), _ptr(ncow))
+        if st != OK:
+            return st, None, None
+        return st, slots[:n].copy(), pair.reshape(1, 2)[: int(ncow[0])].copy()
+
+    def free(self, seq):
+        return lib().orc_free(self.h, seq)
+
+    def fork(self, parent, child):
+        return lib().orc_fork(self.h, parent, child)
+
+    def num_free(self):
+        return lib().orc_num_free(self.h)
+
+    def holders(self, block):
+        return lib().orc_holders(self.h, block)
+
+    def seq_len(self, seq):
+        return lib().orc_seq_len(self.h, seq)
+
+    def block_table(self, seqs, max_blocks):
+        seqs = _c(seqs, np.int64)
+        table = np.empty((len(seqs), max_blocks), dtype=np.int32)
+        ctx = np.empty(len(seqs), dtype=np.int32)
+        st = lib().orc_block_table(self.h, _ptr(seqs), len(seqs), max_blocks, _ptr(table),
+                                   _ptr(ctx))
+        return st, table, ctx
+
+
+# ---------------------------------------------------------- data movement
+def reshape_and_cache(key, value, k_cache, v_cache, slots, block_size, elem_bytes):
+    """In place on numpy caches [NB, Hkv, bs, D] (raw storage dtype)."""
+    T, Hkv, D = key.shape
+    key = np.ascontiguousarray(key)
+    value = np.ascontiguousarray(value)
+    slots = _c(slots, np.int64)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    return lib().orc_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(slots), T, Hkv, D, block_size, k_cache.shape[0],
+                                       elem_bytes)
+
+
+def copy_blocks(k_caches, v_caches, pairs):
+    pairs = _c(pairs, np.int32).reshape(-1, 2)
+    L = len(k_caches)
+    kp = (C.c_void_p * L)(*[c.ctypes.data for c in k_caches])
+    vp = (C.c_void_p * L)(*[c.ctypes.data for c in v_caches])
+    block_bytes = k_caches[0][0].nbytes
+    return lib().orc_copy_blocks(kp, vp, L, _ptr(pairs), pairs.shape[0], block_bytes)
+
+
+# --------------------------------------------------------------- attention
+def paged_decode_attention(q, k_cache, v_cache, tables, ctx, scale, dtype, rows=None,
+                           n_threads=None):
+    """fp64 output [B, Hq, D]; rows (flat b*Hq+h) limits the work (others left NaN)."""
+    q = np.ascontiguousarray(q)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    tables = _c(tables, np.int32)
+    ctx = _c(ctx, np.int32)
+    out = np.full((B, Hq, D), np.nan, dtype=np.float64)
+    r = None if rows is None else _c(rows, np.int64)
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    st = lib().orc_paged_decode_attention(
+        _ptr(q), _ptr(np.ascontiguousarray(k_cache)), _ptr(np.ascontiguousarray(v_cache)),
+        _ptr(tables), _ptr(ctx), B, Hq, Hkv, D, bs, tables.shape[1], float(scale),
+        DTYPE_CODE[dtype], _ptr(out), _ptr(r), 0 if r is None else len(r), n_threads)
+    if st != OK:
+        raise ValueError(f"oracle attention rejected its arguments ({st})")
+    return out
+
+
+def contiguous_attention(q, k, v, scale, dtype, heads=None):
+    """q [Hq, D], k/v [n, Hkv, D] in logical order -> fp64 [Hq, D] (unlisted heads NaN)."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    Hq, D = q.shape
+    n, Hkv, _ = k.shape
+    out = np.full((Hq, D), np.nan, dtype=np.float64)
+    hs = None if heads is None else _c(heads, np.int32)
+    st = lib().orc_contiguous_attention(_ptr(q), _ptr(k), _ptr(v), n, Hq, Hkv, D, float(scale),
+                                        DTYPE_CODE[dtype], _ptr(out), _ptr(hs),
+                                        0 if hs is None else len(hs))
+    if st != OK:
+        raise ValueError(f"oracle attention rejected its arguments ({st})")
+    return out

@@ -1,0 +1,78 @@
+"""Runs a workload's op script through the oracle (test infrastructure)."""
+import numpy as np
+import torch
+
+import oracle
+
+STORAGE = {"f32": np.float32, "f16": np.uint16, "bf16": np.uint16}
+
+
+def raw(t: torch.Tensor) -> np.ndarray:
+    """Host numpy view of a tensor's storage bits (float32 stays float32)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def run_script(wl, with_cache=True, write_tokens=True):
+    """Execute every op of ``wl`` on an oracle pool.
+
+    Returns dict(pool, table, ctx, k_cache, v_cache, records) where records[i] is
+    (slots, cow_pairs) for alloc op i (None for other ops)."""
+    pool = oracle.Pool(wl.num_blocks, wl.bs)
+    shape = (wl.num_blocks, wl.Hkv, wl.bs, wl.D)
+    kc = np.zeros(shape, dtype=STORAGE[wl.dtype]) if with_cache else None
+    vc = np.zeros(shape, dtype=STORAGE[wl.dtype]) if with_cache else None
+    records = []
+    for op in wl.ops:
+        if op[0] == "alloc":
+            _, seq, n, pos0, write = op
+            st, slots, cow = pool.alloc(seq, n)
+            assert st == oracle.OK, (op, st)
+            records.append((slots, cow))
+            if with_cache:
+                if len(cow):
+                    oracle.copy_blocks([kc], [vc], cow)
+                if write and write_tokens and n > 0:
+                    k = raw(wl.tokens(seq, pos0, n, 0))
+                    v = raw(wl.tokens(seq, pos0, n, 1))
+                    assert oracle.reshape_and_cache(k, v, kc, vc, slots, wl.bs,
+                                                    wl.elem_bytes) == oracle.OK
+        elif op[0] == "fork":
+            assert pool.fork(op[1], op[2]) == oracle.OK
+            records.append(None)
+        else:
+            assert pool.free(op[1]) == oracle.OK
+            records.append(None)
+    st, table, ctx = pool.block_table(wl.batch, wl.max_blocks)
+    assert st == oracle.OK
+    return dict(pool=pool, table=table, ctx=ctx, k_cache=kc, v_cache=vc, records=records)
+
+
+def attention(wl, state, rows=None, n_threads=None):
+    q = raw(wl.q())
+    return oracle.paged_decode_attention(q, state["k_cache"], state["v_cache"], state["table"],
+                                         state["ctx"], wl.scale, wl.dtype, rows=rows,
+                                         n_threads=n_threads)
+
+
+def contiguous_row(wl, b, heads=None):
+    """Oracle attention of batch row b from its logical (unpaged) key/value rows."""
+    seq = int(wl.batch[b])
+    q = raw(wl.q()[b])
+    if heads is None:
+        k = raw(wl.contiguous_kv(seq, 0))
+        v = raw(wl.contiguous_kv(seq, 1))
+        return oracle.contiguous_attention(q, k, v, wl.scale, wl.dtype)
+    # only the KV heads the listed query heads read
+    kvh = sorted({h // wl.G for h in heads})
+    k = raw(wl.contiguous_kv(seq, 0, heads=kvh))
+    v = raw(wl.contiguous_kv(seq, 1, heads=kvh))
+    out = np.full((wl.Hq, wl.D), np.nan)
+    for h in heads:
+        j = kvh.index(h // wl.G)
+        o = oracle.contiguous_attention(q[h:h + 1], k[:, j:j + 1], v[:, j:j + 1], wl.scale,
+                                        wl.dtype)
+        out[h] = o[0]
+    return out
