@@ -1,0 +1,430 @@
+"""Benchmark of the paged decode hot path on B200.
+
+One step = one decode step of one layer for the whole batch: append each
+sequence's new token to the paged cache (pa_reshape_and_cache; block copies
+when a shared block must be copied first), then paged decode attention
+(pa_decode_attention: decode kernel + log-sum-exp combine).
+
+  value  : decode tokens/s (batch / step time), inputs resident in HBM, summed
+           over ranks (each rank is an independent replica: weak scaling)
+  e2e    : the same metric through the public API from host buffers: the host
+           pool allocates each new token's slot (contexts grow by one token per
+           step), pinned host q / k / v / slots / tables go to the device, the
+           kernels run and the output comes back, all inside the timed region
+  roofline: the decode call's algorithmic bytes / its CUDA-event duration
+           against the measured HBM copy bandwidth
+  cpu_baseline: the fp64 oracle on the host cores, on a bounded sample
+
+``--impl reference`` times the oracle alone as the reference arm.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention tokens/s and KV-read GB/s as % of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def _peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _kernel_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_486_b200", "csrc")
+    for name in ("decode_tc.cu", "decode_common.cuh", "decode_simt.cu"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(config):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(config)
+        if e and e.get("kernel_sha") == _kernel_sha():
+            return e["dram_bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return dist, dist.get_rank(), ws
+    return None, 0, 1
+
+
+def _max_over_ranks(dist, x):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(dist, x):
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- our arm
+def _setup(wl):
+    from paged_kv_cache_486_b200.engine import PagedKVCache
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda")
+
+    def tokens(seq, pos0, n):
+        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
+
+    eng.apply_ops(wl.ops[:wl.n_prefill_ops], tokens)
+    # the decode step's slots (and any block copies) for the resident-input loop
+    slots, keys, vals, copies = [], [], [], []
+    for op in wl.decode_ops():
+        _, seq, n, pos0, _w = op
+        s, cow = eng.alloc(seq, n)
+        slots.append(s)
+        copies.extend(cow.tolist())
+        k, v = tokens(seq, pos0, n)
+        keys.append(k)
+        vals.append(v)
+    step = dict(slots=torch.from_numpy(np.concatenate(slots)).cuda(),
+                key=torch.cat(keys), value=torch.cat(vals),
+                pairs=torch.tensor(copies, dtype=torch.int32, device="cuda").reshape(-1, 2))
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    step.update(bt=bt, ctx=ctx, q=wl.q("cuda"), out=torch.empty_like(wl.q("cuda")))
+    torch.cuda.synchronize()
+    return eng, step
+
+
+def run_ours(args, dist, rank, world):
+    import paged_kv_cache_486_b200 as pa
+    wl = workloads.make(args.config)
+    eng, st = _setup(wl)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    launches_per_step = 1 + 2 + (1 if st["pairs"].shape[0] else 0)
+
+    def step():
+        if st["pairs"].shape[0]:
+            pa.pa_copy_blocks([eng.k_cache], [eng.v_cache], st["pairs"], eng.dev_error)
+        eng.write(st["key"], st["value"], st["slots"])
+        e_mid.record(stream)
+        eng.decode(st["q"], st["bt"], st["ctx"], wl.scale, out=st["out"])
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e_mid = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    step_ms, decode_ms = [], []
+    for _ in range(args.steps):
+        flush.zero_()  # L2 flushed between timed steps, outside the events
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        step_ms.append(e0.elapsed_time(e1))
+        decode_ms.append(e_mid.elapsed_time(e1))
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if dist:
+        dist.barrier()
+    assert eng.device_errors() == 0, "device guards fired"
+
+    total_ms = _max_over_ranks(dist, sum(step_ms))
+    tokens_all = _sum_over_ranks(dist, wl.B * args.steps)
+    value = tokens_all / (total_ms / 1e3)
+    alg = wl.kv_read_bytes()
+    dec_ms = statistics.mean(decode_ms)
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    peak, peak_kind = _peak_hbm()
+
+    e2e = run_e2e(args, wl, eng, dist)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded counter-based N(0,1) stand-in values, shuffled block pool)",
+        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+                   "head_dim": wl.D, "block_size": wl.bs, "layers_per_step": 1,
+                   "context_tokens": int(wl.context_lens().sum()),
+                   "kv_read_bytes_per_step": alg, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write outside the events)"},
+        "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
+                     "traffic": _traffic(wl.name),
+                     "timed": "pa_decode_attention call: decode + combine kernels"},
+        "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, wl, eng, dist):
+    """Public-API decode steps from pinned host buffers; contexts grow one token per step."""
+    import paged_kv_cache_486_b200 as pa
+    stream = torch.cuda.current_stream()
+    B, Hkv, D, Hq = wl.B, wl.Hkv, wl.D, wl.Hq
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    h_q = wl.q("cpu").pin_memory()
+    h_k = torch.empty(B, Hkv, D, dtype=dt).pin_memory()
+    h_v = torch.empty(B, Hkv, D, dtype=dt).pin_memory()
+    h_k.copy_(wl.tokens(1 << 50, 0, B, 0))
+    h_v.copy_(wl.tokens(1 << 50, 0, B, 1))
+    h_slots = torch.empty(B, dtype=torch.int64).pin_memory()
+    h_table = torch.empty(B, wl.max_blocks, dtype=torch.int32).pin_memory()
+    h_ctx = torch.empty(B, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(B, Hq, D, dtype=dt).pin_memory()
+    d = {k: torch.empty_like(v, device="cuda") for k, v in
+         dict(q=h_q, k=h_k, v=h_v, slots=h_slots, table=h_table, ctx=h_ctx, out=h_out).items()}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    seqs = [int(s) for s in wl.batch]
+    np_slots = h_slots.numpy()
+    np_table, np_ctx = h_table.numpy(), h_ctx.numpy()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_table, h_ctx))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def one():
+        copies = []
+        for i, s in enumerate(seqs):
+            sl, cow = eng.pool.pa_alloc(s, 1)
+            np_slots[i] = sl[0]
+            copies.extend(cow.tolist())
+        eng.pool.pa_block_table(seqs, wl.max_blocks, out_table=np_table, out_ctx=np_ctx)
+        for name, h in (("q", h_q), ("k", h_k), ("v", h_v), ("slots", h_slots),
+                        ("table", h_table), ("ctx", h_ctx)):
+            d[name].copy_(h, non_blocking=True)
+        if copies:
+            pairs = torch.tensor(copies, dtype=torch.int32).reshape(-1, 2).cuda()
+            pa.pa_copy_blocks([eng.k_cache], [eng.v_cache], pairs, eng.dev_error)
+        pa.pa_reshape_and_cache(d["k"], d["v"], eng.k_cache, eng.v_cache, d["slots"],
+                                eng.dev_error)
+        pa.pa_decode_attention(d["out"], d["q"], eng.k_cache, eng.v_cache, d["table"], d["ctx"],
+                               wl.scale, eng.workspace, eng.dev_error)
+        h_out.copy_(d["out"], non_blocking=True)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    total = _max_over_ranks(dist, sum(ms))
+    tokens_all = _sum_over_ranks(dist, wl.B * args.steps)
+    assert torch.isfinite(h_out.float()).all()
+    return {"value": tokens_all / (total / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": total / args.steps}
+
+
+# ---------------------------------------------------------- oracle timings
+def cpu_baseline(wl, target_s=10.0):
+    import oracle
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_side import raw
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    # lay the first S sequences' logical rows out in a shuffled pool of wl.bs blocks
+    rng = np.random.default_rng(wl.seed)
+    ctx_all = wl.context_lens()
+    S = 1
+    t_one = None
+    pools = {}
+
+    def make(S):
+        ctx = ctx_all[:S]
+        nblk = (ctx + wl.bs - 1) // wl.bs
+        nb = int(nblk.sum())
+        perm = rng.permutation(nb).astype(np.int32)
+        kc = np.zeros((nb, wl.Hkv, wl.bs, wl.D), dtype=np.float32 if wl.dtype == "f32"
+                      else np.uint16)
+        vc = np.zeros_like(kc)
+        table = np.full((S, int(nblk.max())), -1, np.int32)
+        off = 0
+        for b in range(S):
+            blocks = perm[off:off + nblk[b]]
+            off += nblk[b]
+            table[b, :nblk[b]] = blocks
+            seq = int(wl.batch[b])
+            for kind, cache in ((0, kc), (1, vc)):
+                rows = raw(wl.contiguous_kv(seq, kind, dev))  # [n, Hkv, D]
+                pad = np.zeros((nblk[b] * wl.bs,) + rows.shape[1:], rows.dtype)
+                pad[:len(rows)] = rows
+                cache[blocks] = pad.reshape(nblk[b], wl.bs, wl.Hkv, wl.D).transpose(0, 2, 1, 3)
+        q = raw(wl.q(dev)[:S])
+        return q, kc, vc, table, ctx.astype(np.int32)
+
+    threads = os.cpu_count() or 1
+    q, kc, vc, table, ctx = make(S)
+    t0 = time.perf_counter()
+    oracle.paged_decode_attention(q, kc, vc, table, ctx, wl.scale, wl.dtype, n_threads=threads)
+    t_one = time.perf_counter() - t0
+    S = int(min(wl.B, max(1, target_s / max(t_one, 1e-3) / 4)))
+    q, kc, vc, table, ctx = make(S)
+    reps, elapsed = 0, 0.0
+    while elapsed < target_s and reps < 50:
+        t0 = time.perf_counter()
+        oracle.paged_decode_attention(q, kc, vc, table, ctx, wl.scale, wl.dtype,
+                                      n_threads=threads)
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    return {"value": S * reps / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {S} of {wl.B} sequences ({int(ctx.sum())} context tokens) of "
+                      f"{wl.name}, fp64 oracle, {reps} passes, {elapsed:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    wl = workloads.make(args.config)
+    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(wl, target_s=min(per_step, 2.0))
+    vals = [cpu_baseline(wl, target_s=per_step) for _ in range(args.steps)]
+    v = statistics.mean(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * wl.B / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq,
+                       "kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": wl.bs},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, rank, world)
+        if line:
+            print(json.dumps(line), flush=True)
+        return
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist, rank, world = _dist()
+    try:
+        line = run_ours(args, dist, rank, world)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,244 @@
+/*
+ * pa.h -- C ABI of libpagedattn: a paged KV cache and single-query decode
+ * attention over it, for NVIDIA B200 (sm_100a).
+ *
+ * What the pages define (cited by page title and section):
+ *  [P1] "PagedAttention for professionals: how vLLM serves more requests on the
+ *       same H100", sections "Beginner example: library shelves" and "The
+ *       scientific explanation: why PagedAttention is a breakthrough" (+ its
+ *       results list).
+ *  [P2] "KV Cache and PagedAttention: Why Your LLM Server Slows Down", sections
+ *       "What is the KV cache?", "How PagedAttention solves this", "How does
+ *       PagedAttention work?".
+ *  [P5] "KV Cache for intermediates: why long context eats the GPU and how to cut
+ *       it 4x", sections "The precise scientific definition" and "The four
+ *       solutions".
+ * The pages describe the data structure (fixed-size blocks anywhere in one pool,
+ * a per-sequence block table, on-demand growth, shared blocks with copy-on-write)
+ * and the KV-size formula; they print no kernel, memory layout or attention
+ * formula.  The readings taken where they are silent are stated at each call.
+ *
+ * Conventions for every call:
+ *  - Sizes are int32 unless noted; pointers named *_host point to host memory,
+ *    all other buffer pointers to device memory on the device of `stream`.
+ *  - Every device buffer is owned by the caller.  The library never allocates
+ *    or frees device memory.  Pool metadata (host) is owned by the pool object.
+ *  - Device calls are asynchronous on `stream` (NULL = the legacy default
+ *    stream).  They return PA_ERR_CUDA if the launch fails.
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns PA_ERR_INVALID and changes nothing.  Values that live in
+ *    device memory (slots, block ids, pairs, context lengths) are checked by the
+ *    kernels: an out-of-range value is skipped, never dereferenced, and its
+ *    PA_DEVERR_* bit is OR-ed into *dev_error (when dev_error is non-NULL).
+ *    No kernel traps.  Host-side validators for the same data are provided.
+ *  - On any error, pa_last_error() returns a message (thread-local).
+ *  - The pool object is not thread-safe; use one pool per thread or lock it.
+ */
+#ifndef PAGED_ATTN_PA_H
+#define PAGED_ATTN_PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,   /* bad argument; nothing changed */
+  PA_ERR_OOM = 2,       /* pool has too few free blocks; nothing changed */
+  PA_ERR_NOT_FOUND = 3, /* unknown sequence id */
+  PA_ERR_CUDA = 4,      /* a CUDA runtime call failed */
+  PA_ERR_DEVICE = 5     /* a kernel reported PA_DEVERR_* bits (pa_check_device_error) */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Bits a kernel may OR into *dev_error. */
+#define PA_DEVERR_BAD_SLOT 1    /* slot_mapping entry >= num_blocks * block_size */
+#define PA_DEVERR_BAD_BLOCK 2   /* block table / copy pair entry outside [0, num_blocks) */
+#define PA_DEVERR_BAD_CTX 4     /* context length < 0 or > max_blocks * block_size */
+#define PA_DEVERR_TIMEOUT 8     /* a bounded wait for a tile copy gave up */
+
+/* == cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* pa_stream;
+
+typedef struct pa_pool pa_pool;
+
+/* ------------------------------------------------------------------------
+ * Block pool (host).  [P1] "The scientific explanation": the cache is split
+ * into fixed-size blocks (default 16 tokens) stored anywhere in GPU memory,
+ * and a block table per request maps its logical blocks to physical ones.
+ * [P1] "Beginner example": a request takes a new block only when its 17th
+ * token arrives; a finished request's blocks go back to the pool and are taken
+ * again at once.  [P2] "How PagedAttention solves this": on-demand pages, and
+ * shared prefix pages with copy-on-write.
+ * Readings: the free list is a stack (the last block freed is the first
+ * reused; a fresh pool hands out 0, 1, 2, ...); growing into a partially filled
+ * last block that other sequences also hold copies it first (one copy pair);
+ * full shared blocks stay shared; the last holder writes in place.
+ * ---------------------------------------------------------------------- */
+
+/* Create a pool of num_blocks (>= 0) blocks of block_size (>= 1) tokens. */
+pa_status pa_pool_create(int32_t num_blocks, int32_t block_size, pa_pool** pool_out);
+void pa_pool_destroy(pa_pool* pool);
+
+/* Grow sequence seq_id by n_new (>= 0) tokens, creating it if unknown.
+ * slot_mapping_out_host[n_new] receives each new token's slot:
+ *   physical_block * block_size + offset_in_block   (int64).
+ * If the sequence's last block was partially filled and shared, it is first
+ * replaced by a fresh copy: one (src, dst) pair of physical block ids is written
+ * to cow_pairs_out_host[0..1] and *n_cow_out = 1 (else 0).  The caller must run
+ * pa_copy_blocks on returned pairs before writing the new tokens.
+ * max_cow is the capacity of cow_pairs_out_host in pairs (>= 1 if a copy can
+ * happen; PA_ERR_INVALID if a copy is needed and max_cow < 1).
+ * All or nothing: PA_ERR_OOM (too few free blocks) leaves the pool unchanged. */
+pa_status pa_alloc(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slot_mapping_out_host,
+                   int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out);
+
+/* Drop seq_id: each of its blocks loses one holder, in logical order; a block
+ * with no holder left goes on top of the free stack.  PA_ERR_NOT_FOUND if unknown. */
+pa_status pa_free(pa_pool* pool, int64_t seq_id);
+
+/* child_id becomes a copy of parent_id sharing all of its blocks ([P1] results:
+ * parallel sampling with n=4 costs about the memory of n=1).
+ * PA_ERR_NOT_FOUND: unknown parent; PA_ERR_INVALID: child exists. */
+pa_status pa_fork(pa_pool* pool, int64_t parent_id, int64_t child_id);
+
+/* Block-table rows for n_seqs sequences: table_out_host[i * max_blocks + j] is
+ * the physical block of logical block j of seq_ids_host[i], -1 past the end;
+ * ctx_lens_out_host[i] is its token count.  PA_ERR_INVALID if a sequence holds
+ * more than max_blocks blocks; PA_ERR_NOT_FOUND if one is unknown. */
+pa_status pa_block_table(const pa_pool* pool, const int64_t* seq_ids_host, int32_t n_seqs,
+                         int32_t max_blocks, int32_t* table_out_host, int32_t* ctx_lens_out_host);
+
+int32_t pa_num_free_blocks(const pa_pool* pool);
+/* Number of sequences holding `block` (0 if free, -1 if out of range). */
+int32_t pa_refcount(const pa_pool* pool, int32_t block);
+/* Token count of seq_id, or -1 if unknown. */
+int64_t pa_seq_len(const pa_pool* pool, int64_t seq_id);
+
+/* [P5] "The precise scientific definition": KV bytes of a model =
+ * 2 (key and value) x layers x tokens x kv_heads x head_dim x bytes per element. */
+uint64_t pa_kv_bytes(int32_t num_layers, int64_t num_tokens, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t dtype_bytes);
+
+/* ------------------------------------------------------------------------
+ * Cache layout (reading; the pages fix none): one key pool and one value pool
+ * per layer, each [num_blocks, num_kv_heads, block_size, head_dim] row-major in
+ * `dtype`, so the (block, kv head) tile of block_size x head_dim is contiguous.
+ * ---------------------------------------------------------------------- */
+
+/* Append new tokens' keys and values to the cache ([P2] "What is the KV cache?":
+ * the engine stores each token's K and V instead of recomputing them).
+ * key, value: [n_tokens, num_kv_heads, head_dim] contiguous, `dtype`.
+ * slot_mapping: [n_tokens] int64, device; -1 = skip the token.
+ * Byte-exact copy.  An entry >= num_blocks * block_size is skipped and sets
+ * PA_DEVERR_BAD_SLOT.  Duplicate slots in one call are invalid input (which copy
+ * lands is unspecified).  head_dim * element size must be a multiple of 16. */
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int32_t n_tokens,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                               pa_stream stream);
+
+/* Copy-on-write block copies ([P2] "How PagedAttention solves this").
+ * k_caches_host / v_caches_host: host arrays of num_layers (1..128) device
+ * pointers, one key pool and one value pool per layer.
+ * pairs: [n_pairs, 2] int32 (src, dst) physical block ids, device.
+ * For every pair and layer, block dst of both pools becomes a byte copy of
+ * block src.  block_bytes = num_kv_heads * block_size * head_dim * element
+ * size (a multiple of 16).  A dst may not appear twice and may not be a src in
+ * the same call (check with pa_validate_copy_pairs); ids outside
+ * [0, num_blocks) are skipped with PA_DEVERR_BAD_BLOCK. */
+pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
+                         int32_t num_layers, const int32_t* pairs, int32_t n_pairs,
+                         int32_t num_blocks, int64_t block_bytes, int32_t* dev_error,
+                         pa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Decode attention.  [P5] "The precise scientific definition": the new token
+ * computes a new Q while the K and V of every earlier token must already be in
+ * memory.  Reading (the pages print no formula):
+ *   out[b, h, :] = sum_{j < ctx[b]} softmax_j(scale * q[b, h, :] . K_b[j, g, :]) V_b[j, g, :]
+ * with g = h / (num_q_heads / num_kv_heads) ([P5] "The four solutions", GQA: a
+ * group of query heads shares one K/V head; MQA is num_kv_heads = 1).  Token j
+ * of batch row b is slot (block_tables[b, j / block_size], j % block_size).
+ * ctx[b] counts the token the caller has just written with
+ * pa_reshape_and_cache.  ctx[b] = 0 gives a zero output row.
+ *
+ * q, out: [batch, num_q_heads, head_dim], `dtype`; out is rounded once, to
+ *   nearest even, from fp32 accumulators.
+ * block_tables: [batch, max_blocks] int32, device; context_lens: [batch] int32.
+ * head_dim in {64, 128}; block_size in {8, 16, 32, 64, 128}; batch <= 4096;
+ * num_blocks * num_kv_heads * block_size < 2^31.
+ * workspace: device scratch of at least pa_decode_workspace_size(...) bytes,
+ *   16-byte aligned, contents need no initialisation; calls that share a
+ *   workspace must be ordered on one stream.
+ * The work is split evenly across the GPU by KV blocks: a sequence that fits in
+ * one worker's share is done in a single pass; a longer one is cut into pieces
+ * whose (max, sum, partial output) are merged by a log-sum-exp combine kernel.
+ * ---------------------------------------------------------------------- */
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim);
+
+pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                              int32_t max_blocks, float scale, pa_dtype dtype, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_error, pa_stream stream);
+
+/* Kernel paths for pa_decode_attention_ex. */
+#define PA_PATH_AUTO 0   /* tensor-core path when it applies, else the CUDA-core path */
+#define PA_PATH_TC 1     /* fp16/bf16, G <= 8, block_size a multiple of 16 */
+#define PA_PATH_SIMT 2   /* every supported shape and dtype */
+
+/* As pa_decode_attention, with the path and the number of workers (warps that
+ * split the KV blocks; 0 = automatic, else clamped to the supported range)
+ * chosen by the caller.  Every choice gives the same result up to fp32
+ * rounding order. */
+pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, int32_t max_blocks, float scale,
+                                 pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                                 int32_t* dev_error, int32_t path, int32_t num_workers,
+                                 pa_stream stream);
+
+/* Path and worker count pa_decode_attention would use for these arguments. */
+pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* path_out,
+                         int32_t* num_workers_out);
+
+/* ------------------------------------------------------------------------
+ * Host-side validators (no device work): PA_OK or PA_ERR_INVALID + message.
+ * ---------------------------------------------------------------------- */
+/* Every slot is -1 or in [0, num_blocks * block_size), and no slot repeats. */
+pa_status pa_validate_slot_mapping(const int64_t* slot_mapping_host, int32_t n_tokens,
+                                   int32_t block_size, int32_t num_blocks);
+/* Each ctx in [0, max_blocks * block_size]; each of its ceil(ctx / block_size)
+ * leading table entries in [0, num_blocks). */
+pa_status pa_validate_block_table(const int32_t* block_tables_host,
+                                  const int32_t* context_lens_host, int32_t batch,
+                                  int32_t max_blocks, int32_t block_size, int32_t num_blocks);
+/* Ids in range, no dst repeated, no dst also used as a src. */
+pa_status pa_validate_copy_pairs(const int32_t* pairs_host, int32_t n_pairs, int32_t num_blocks);
+
+/* Copy the device error word to the host (synchronising `stream`), then clear
+ * it.  Returns PA_ERR_DEVICE with *flags_out set if any bit was set. */
+pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream);
+
+/* Message for the last failing call on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* Number of streaming multiprocessors on the current device (0 on failure). */
+int32_t pa_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTN_PA_H */

@@ -1,0 +1,347 @@
+// C ABI entry points for the device calls: argument checks, path and launch
+// choices, TMA tensor maps, and the device error word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "cache_ops.h"
+#include "decode_common.cuh"
+#include "decode_launch.h"
+#include "host_common.h"
+
+namespace {
+
+using pa::fail;
+
+int elem_bytes(pa_dtype d) { return d == PA_F32 ? 4 : 2; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool valid_dtype(pa_dtype d) { return d == PA_F32 || d == PA_F16 || d == PA_BF16; }
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return 0;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// ------------------------------ tensor maps --------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// A pool [num_blocks, Hkv, bs, D] seen as `rows` rows of D elements; one box is
+// 16 rows x D, delivered with 128-byte swizzle (D = 128: 3-d view 64 x 2 x rows).
+bool make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim, pa_dtype dt) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType t =
+      dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r;
+  if (head_dim == 128) {
+    cuuint64_t dims[3] = {64, 2, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[2] = {128, 256};
+    cuuint32_t box[3] = {64, 2, 16};
+    cuuint32_t es[3] = {1, 1, 1};
+    r = enc(map, t, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t es[2] = {1, 1};
+    r = enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  return r == CUDA_SUCCESS;
+}
+
+// Small per-thread cache: encoding is cheap but not free, and decode is called
+// with the same pools every step.
+struct MapEntry {
+  const void* base;
+  int64_t rows;
+  int head_dim;
+  int dtype;
+  CUtensorMap map;
+};
+thread_local MapEntry g_maps[8];
+thread_local int g_maps_next = 0;
+
+bool tile_map(CUtensorMap* out, const void* base, int64_t rows, int head_dim, pa_dtype dt) {
+  for (auto& e : g_maps) {
+    if (e.base == base && e.rows == rows && e.head_dim == head_dim && e.dtype == dt) {
+      *out = e.map;
+      return true;
+    }
+  }
+  MapEntry& e = g_maps[g_maps_next];
+  if (!make_tile_map(&e.map, base, rows, head_dim, dt)) return false;
+  e.base = base;
+  e.rows = rows;
+  e.head_dim = head_dim;
+  e.dtype = dt;
+  g_maps_next = (g_maps_next + 1) % 8;
+  *out = e.map;
+  return true;
+}
+
+// ------------------------------ decode plan --------------------------------
+int max_workers(int group) {
+  int w = pa::kPieceHeadBudget / group;
+  if (w > pa::kMaxWorkers) w = pa::kMaxWorkers;
+  return w < 1 ? 1 : w;
+}
+
+bool tc_applies(int group, int head_dim, int block_size, pa_dtype dt) {
+  return (dt == PA_F16 || dt == PA_BF16) && (head_dim == 64 || head_dim == 128) && group <= 8 &&
+         block_size % 16 == 0;
+}
+
+size_t pieces_offset(int batch) {
+  const size_t cum = (sizeof(int32_t) * (static_cast<size_t>(batch) + 1) + 255) & ~size_t(255);
+  return 256 + cum;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t pa_device_sm_count(void) { return sm_count(); }
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache, void* v_cache,
+                               const int64_t* slot_mapping, int32_t n_tokens,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                               pa_stream stream) {
+  if (!valid_dtype(dtype) || n_tokens < 0 || num_kv_heads < 1 || head_dim < 1 ||
+      block_size < 1 || num_blocks < 0)
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache: bad sizes (n_tokens=%d kv_heads=%d "
+                "head_dim=%d block_size=%d num_blocks=%d)", n_tokens, num_kv_heads, head_dim,
+                block_size, num_blocks);
+  const int row_bytes = head_dim * elem_bytes(dtype);
+  if (row_bytes % 16)
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache: head_dim * element size = %d bytes is "
+                "not a multiple of 16", row_bytes);
+  if (n_tokens == 0) return PA_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache: NULL pointer");
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache: misaligned pointer");
+  const cudaError_t e = pa::launch_reshape_and_cache(
+      key, value, k_cache, v_cache, slot_mapping, n_tokens, num_kv_heads, row_bytes, block_size,
+      num_blocks, dev_error, sm_count() ? sm_count() : 148, stream);
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_reshape_and_cache");
+}
+
+pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
+                         int32_t num_layers, const int32_t* pairs, int32_t n_pairs,
+                         int32_t num_blocks, int64_t block_bytes, int32_t* dev_error,
+                         pa_stream stream) {
+  if (num_layers < 1 || num_layers > pa::kMaxLayers || n_pairs < 0 || num_blocks < 0 ||
+      block_bytes <= 0 || block_bytes % 16)
+    return fail(PA_ERR_INVALID, "pa_copy_blocks: bad sizes (layers=%d pairs=%d block_bytes=%lld)",
+                num_layers, n_pairs, static_cast<long long>(block_bytes));
+  if (n_pairs == 0) return PA_OK;
+  if (!k_caches_host || !v_caches_host || !pairs)
+    return fail(PA_ERR_INVALID, "pa_copy_blocks: NULL pointer");
+  pa::LayerPtrs ptrs;
+  std::memset(&ptrs, 0, sizeof ptrs);
+  for (int i = 0; i < num_layers; ++i) {
+    if (!k_caches_host[i] || !v_caches_host[i] || !aligned(k_caches_host[i], 16) ||
+        !aligned(v_caches_host[i], 16))
+      return fail(PA_ERR_INVALID, "pa_copy_blocks: layer %d pointer NULL or misaligned", i);
+    ptrs.k[i] = k_caches_host[i];
+    ptrs.v[i] = v_caches_host[i];
+  }
+  const cudaError_t e = pa::launch_copy_blocks(ptrs, num_layers, pairs, n_pairs, num_blocks,
+                                               block_bytes, dev_error, stream);
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_copy_blocks");
+}
+
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim) {
+  if (batch < 0 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads || head_dim < 1)
+    return 0;
+  const int group = num_q_heads / num_kv_heads;
+  return pieces_offset(batch) +
+         sizeof(float) * 2 * static_cast<size_t>(max_workers(group)) * group * (head_dim + 2);
+}
+
+pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* path_out,
+                         int32_t* num_workers_out) {
+  if (num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID, "pa_decode_plan: bad head counts");
+  const int group = num_q_heads / num_kv_heads;
+  const int sms = sm_count() ? sm_count() : 148;
+  int path, workers;
+  if (tc_applies(group, head_dim, block_size, dtype)) {
+    path = PA_PATH_TC;
+    workers = sms * pa::decode_tc_workers_per_cta();
+  } else {
+    path = PA_PATH_SIMT;
+    workers = sms * 16;
+  }
+  const int cap = max_workers(group);
+  if (workers > cap) workers = cap;
+  (void)batch;
+  if (path_out) *path_out = path;
+  if (num_workers_out) *num_workers_out = workers;
+  return PA_OK;
+}
+
+pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
+                                 const void* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t num_blocks, int32_t max_blocks, float scale,
+                                 pa_dtype dtype, void* workspace, size_t workspace_bytes,
+                                 int32_t* dev_error, int32_t path, int32_t num_workers,
+                                 pa_stream stream) {
+  if (!valid_dtype(dtype))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: unknown dtype %d", static_cast<int>(dtype));
+  if (batch < 0 || batch > pa::kMaxBatch)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: batch %d outside [0, %d]", batch,
+                pa::kMaxBatch);
+  if (num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_q_heads %d not a multiple of "
+                "num_kv_heads %d", num_q_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: head_dim %d not in {64, 128}", head_dim);
+  if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
+      block_size != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: block_size %d not in {8,16,32,64,128}",
+                block_size);
+  if (num_blocks < 0 || max_blocks < 0)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: negative num_blocks or max_blocks");
+  const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  if (rows >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_blocks * num_kv_heads * block_size "
+                "= %lld >= 2^31", static_cast<long long>(rows));
+  if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention: scale is NaN");
+  if (path != PA_PATH_AUTO && path != PA_PATH_TC && path != PA_PATH_SIMT)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: unknown path %d", path);
+  if (batch == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: NULL pointer");
+  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(workspace, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: misaligned pointer");
+  const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: workspace %zu bytes < %zu needed",
+                workspace_bytes, need);
+
+  const int group = num_q_heads / num_kv_heads;
+  const bool tc_ok = tc_applies(group, head_dim, block_size, dtype);
+  if (path == PA_PATH_TC && !tc_ok)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: tensor-core path needs fp16/bf16, "
+                "group <= 8 and block_size a multiple of 16");
+  const bool use_tc = path == PA_PATH_TC || (path == PA_PATH_AUTO && tc_ok);
+  int32_t planned_path = 0, workers = 0;
+  pa_status st = pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, dtype,
+                                &planned_path, &workers);
+  if (st != PA_OK) return st;
+  if (!use_tc && planned_path == PA_PATH_TC) workers = (sm_count() ? sm_count() : 148) * 16;
+  if (num_workers > 0) workers = num_workers;
+  if (workers > max_workers(group)) workers = max_workers(group);
+
+  pa::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.dev_error = dev_error;
+  a.ws_cum = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + 256);
+  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) + pieces_offset(batch));
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks = max_blocks;
+  a.workers = workers;
+  a.scale_log2 = scale * 1.4426950408889634f;
+
+  cudaError_t e;
+  if (use_tc) {
+    CUtensorMap kmap, vmap;
+    if (!tile_map(&kmap, k_cache, rows, head_dim, dtype) ||
+        !tile_map(&vmap, v_cache, rows, head_dim, dtype))
+      return fail(PA_ERR_CUDA, "pa_decode_attention: cuTensorMapEncodeTiled failed");
+    const int per = pa::decode_tc_workers_per_cta();
+    e = pa::launch_decode_tc(a, dtype, kmap, vmap, (workers + per - 1) / per,
+                             static_cast<cudaStream_t>(stream));
+  } else {
+    e = pa::launch_decode_simt(a, dtype, static_cast<cudaStream_t>(stream));
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention (decode kernel)");
+  e = pa::launch_combine(a, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention (combine kernel)");
+  return PA_OK;
+}
+
+pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                              const int32_t* block_tables, const int32_t* context_lens,
+                              int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                              int32_t max_blocks, float scale, pa_dtype dtype, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_error, pa_stream stream) {
+  return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks, scale, dtype, workspace, workspace_bytes, dev_error,
+                                PA_PATH_AUTO, 0, stream);
+}
+
+pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {
+  if (!dev_error) return fail(PA_ERR_INVALID, "pa_check_device_error: NULL pointer");
+  int32_t h = 0;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&h, dev_error, sizeof h, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "pa_check_device_error");
+  if (flags_out) *flags_out = h;
+  if (h) {
+    e = cudaMemsetAsync(dev_error, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "pa_check_device_error");
+    return fail(PA_ERR_DEVICE, "device error bits 0x%x", h);
+  }
+  return PA_OK;
+}
+
+}  // extern "C"

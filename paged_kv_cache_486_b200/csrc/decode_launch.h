@@ -1,0 +1,24 @@
+// Launchers for the decode kernels (internal).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "decode_common.cuh"
+
+namespace pa {
+
+// CUDA-core path: every dtype, head_dim 64 or 128, any group size.
+cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream);
+
+// Tensor-core path: fp16 / bf16, head_dim 64 or 128, group <= 8, block_size a
+// multiple of 16.  kmap / vmap describe the key / value pools as rows of
+// head_dim elements (see make_tile_maps in api.cu).
+cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
+                             const CUtensorMap& vmap, int num_ctas, cudaStream_t stream);
+int decode_tc_workers_per_cta();
+size_t decode_tc_smem_bytes(int head_dim, int batch);
+
+// Merge pieces of split contexts and zero the rows of empty ones.
+cudaError_t launch_combine(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream);
+
+}  // namespace pa

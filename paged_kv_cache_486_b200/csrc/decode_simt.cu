@@ -1,0 +1,212 @@
+// Paged decode attention on CUDA cores (every dtype and head grouping), and the
+// log-sum-exp combine that merges pieces of a split context.
+//
+// Each warp is one worker of the even split described in decode_common.cuh.
+// Within a segment the warp walks the sequence's blocks through its block-table
+// row; for each token the 32 lanes hold head_dim / 32 elements of the key and
+// value rows (coalesced), reduce the dot products of up to 8 query heads with
+// shuffles and keep an online softmax per head in fp32.  Query heads beyond 8
+// per KV head are done in further passes over the same blocks.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "decode_common.cuh"
+#include "decode_launch.h"
+
+namespace pa {
+
+constexpr int kSimtWarps = 8;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs a) {
+  extern __shared__ int32_t simt_smem[];
+  int32_t* cum = simt_smem;
+  int32_t* ctx_s = simt_smem + a.batch + 1;
+  scan_context(a, cum, ctx_s);
+
+  const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
+  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
+  if (U == 0) return;
+  const int64_t W = U < a.workers ? U : a.workers;
+  const int lane = threadIdx.x & 31;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kSimtWarps + (threadIdx.x >> 5);
+  if (w >= W) return;
+  const int64_t u0 = split_start(w, U, W), u1 = split_start(w + 1, U, W);
+
+  constexpr int PER = D / 32;
+  const T* q = static_cast<const T*>(a.q);
+  const T* kc = static_cast<const T*>(a.k_cache);
+  const T* vc = static_cast<const T*>(a.v_cache);
+  T* out = static_cast<T*>(a.out);
+  const int bs = a.block_size;
+  const int piece_floats = G * (D + 2);
+
+  UnitCursor c;
+  cursor_seek(c, u0, u1, cum, B, Hkv);
+  bool first_seg = true;
+  while (c.u < c.u_end) {
+    const int b = c.b, kvh = c.kvh, j0 = c.j;
+    const int64_t left = c.u_end - c.u;
+    const int seg = static_cast<int>(left < c.nblk - c.j ? left : c.nblk - c.j);
+    const int j1 = j0 + seg;
+    const bool complete = j0 == 0 && j1 == c.nblk;
+    const int slot = first_seg ? 0 : 1;
+    const int ctx = ctx_s[b];
+    for (int hg = 0; hg < G; hg += 8) {
+      const int nh = G - hg < 8 ? G - hg : 8;
+      float qv[8][PER], o[8][PER], m[8], l[8];
+#pragma unroll
+      for (int hh = 0; hh < 8; ++hh) {
+        m[hh] = -INFINITY;
+        l[hh] = 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+          o[hh][i] = 0.f;
+          qv[hh][i] = hh < nh ? Num<T>::to_f(q[(static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) *
+                                                    D + lane + 32 * i])
+                              : 0.f;
+        }
+      }
+      for (int j = j0; j < j1; ++j) {
+        const int32_t phys = a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j];
+        if (phys < 0 || phys >= a.num_blocks) {
+          if (lane == 0) report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+          continue;
+        }
+        const int rem = ctx - j * bs;
+        const int ntok = rem < bs ? rem : bs;
+        const int64_t tile = ((static_cast<int64_t>(phys) * Hkv + kvh) * bs) * D;
+        for (int t = 0; t < ntok; ++t) {
+          float kr[PER], vr[PER];
+#pragma unroll
+          for (int i = 0; i < PER; ++i) {
+            kr[i] = Num<T>::to_f(kc[tile + t * D + lane + 32 * i]);
+            vr[i] = Num<T>::to_f(vc[tile + t * D + lane + 32 * i]);
+          }
+          float s[8];
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh) {
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) acc = fmaf(qv[hh][i], kr[i], acc);
+            s[hh] = acc;
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+            for (int hh = 0; hh < 8; ++hh) s[hh] += __shfl_xor_sync(0xffffffffu, s[hh], off);
+          }
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh) {
+            const float t2 = s[hh] * a.scale_log2;
+            const float mn = fmaxf(m[hh], t2);
+            const float alpha = exp2f(m[hh] - mn);
+            const float p = exp2f(t2 - mn);
+            l[hh] = l[hh] * alpha + p;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) o[hh][i] = fmaf(o[hh][i], alpha, p * vr[i]);
+            m[hh] = mn;
+          }
+        }
+      }
+      if (complete) {
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          if (hh < nh) {
+            const float inv = 1.f / l[hh];
+            T* orow = out + (static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) * D;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = Num<T>::from_f(o[hh][i] * inv);
+          }
+        }
+      } else {
+        float* piece = a.ws_pieces + (w * 2 + slot) * piece_floats;
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          if (hh < nh) {
+            if (lane == 0) {
+              piece[hg + hh] = m[hh];
+              piece[G + hg + hh] = l[hh];
+            }
+#pragma unroll
+            for (int i = 0; i < PER; ++i) piece[2 * G + (hg + hh) * D + lane + 32 * i] = o[hh][i];
+          }
+        }
+      }
+    }
+    first_seg = false;
+    c.u += seg - 1;
+    c.j = j1 - 1;
+    cursor_next(c, cum, Hkv);
+  }
+}
+
+// One CTA per (b, kv head): zero rows of empty contexts; merge the pieces of a
+// split context:  M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
+  const int Hkv = a.num_kv_heads, G = a.group, D = a.head_dim, B = a.batch;
+  const int b = blockIdx.x / Hkv, kvh = blockIdx.x % Hkv;
+  const int32_t* cum = a.ws_cum;
+  const int nblk = cum[b + 1] - cum[b];
+  T* out = static_cast<T*>(a.out) + (static_cast<int64_t>(b) * a.num_q_heads + kvh * G) * D;
+  if (nblk == 0) {
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[i] = Num<T>::from_f(0.f);
+    return;
+  }
+  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
+  const int64_t W = U < a.workers ? U : a.workers;
+  const int64_t u0 = static_cast<int64_t>(Hkv) * cum[b] + static_cast<int64_t>(kvh) * nblk;
+  const int64_t wf = split_worker_of(u0, U, W);
+  const int64_t wl = split_worker_of(u0 + nblk - 1, U, W);
+  if (wf == wl) return;  // done in one pass by one worker
+  const int piece_floats = G * (D + 2);
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int h = i / D, d = i - h * D;
+    float M = -INFINITY;
+    for (int64_t w = wf; w <= wl; ++w) {
+      const int slot = split_start(w, U, W) >= u0 ? 0 : 1;
+      M = fmaxf(M, a.ws_pieces[(w * 2 + slot) * piece_floats + h]);
+    }
+    float L = 0.f, O = 0.f;
+    for (int64_t w = wf; w <= wl; ++w) {
+      const int slot = split_start(w, U, W) >= u0 ? 0 : 1;
+      const float* piece = a.ws_pieces + (w * 2 + slot) * piece_floats;
+      const float e = exp2f(piece[h] - M);
+      L = fmaf(e, piece[G + h], L);
+      O = fmaf(e, piece[2 * G + h * D + d], O);
+    }
+    out[h * D + d] = Num<T>::from_f(O / L);
+  }
+}
+
+template <typename T, int D>
+static cudaError_t launch_simt_t(const DecodeArgs& a, cudaStream_t stream) {
+  const int ctas = (a.workers + kSimtWarps - 1) / kSimtWarps;
+  const size_t smem = sizeof(int32_t) * (2 * a.batch + 1);
+  decode_simt_kernel<T, D><<<ctas, kSimtWarps * 32, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream) {
+  if (a.head_dim == 64) {
+    if (dtype == PA_F32) return launch_simt_t<float, 64>(a, stream);
+    if (dtype == PA_F16) return launch_simt_t<__half, 64>(a, stream);
+    return launch_simt_t<__nv_bfloat16, 64>(a, stream);
+  }
+  if (dtype == PA_F32) return launch_simt_t<float, 128>(a, stream);
+  if (dtype == PA_F16) return launch_simt_t<__half, 128>(a, stream);
+  return launch_simt_t<__nv_bfloat16, 128>(a, stream);
+}
+
+cudaError_t launch_combine(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream) {
+  const int grid = a.batch * a.num_kv_heads;
+  if (grid == 0) return cudaSuccess;
+  if (dtype == PA_F32) combine_kernel<float><<<grid, 256, 0, stream>>>(a);
+  else if (dtype == PA_F16) combine_kernel<__half><<<grid, 256, 0, stream>>>(a);
+  else combine_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,491 @@
+// Paged decode attention on B200 tensor cores, K/V tiles staged by TMA.
+//
+// Shape of the work.  For one (sequence b, kv head) the G query heads that
+// share the KV head ("KV Cache for intermediates..." / "The four solutions",
+// GQA) form an 8-column operand, so each 16-token tile of keys and values is
+// read from HBM once per KV head and used by all G heads:
+//   S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]          (mma m16n8k16)
+//   O^T[D x 8 heads]     += V^T[D x 16] . P^T[16 x 8]       (mma m16n8k16)
+// Heads beyond G (G < 8) are zero query rows whose results are not stored.
+// Scores are kept in base-2 units (scale * log2 e) with an online softmax in
+// fp32 registers.  The exchange of P^T between the two products is a register
+// transpose (movmatrix), so P never goes through shared memory.
+//
+// Data movement.  Every warp is an independent worker (see decode_common.cuh)
+// with its own ring of kStages stage buffers.  Lane 0 issues, kStages stages
+// ahead of the consumer, two TMA tile loads per stage: 16 rows x D of the key
+// pool and of the value pool, rows (block * Hkv + kv_head) * block_size + 16s,
+// landing 128-byte-swizzled so ldmatrix reads them without bank conflicts.
+// Block ids come from the block table through a per-warp window of 32 ids
+// held one per lane and loaded one window ahead.  Each stage signals an
+// mbarrier with its byte count; every wait on it is bounded in time.
+//
+// Roofline.  Per context token and KV head the kernel must read D*2 bytes of
+// key and D*2 of value; tensor-core work is ~4*8*D flops per token and KV head
+// (8 padded heads), far below the tensor rate, so HBM bandwidth bounds it.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "decode_common.cuh"
+#include "decode_launch.h"
+
+namespace pa {
+namespace tc {
+
+constexpr int kTok = 16;     // tokens per stage (one mma tile of keys)
+constexpr int kWarps = 8;    // workers per CTA
+constexpr int kStages = 3;   // ring depth per worker
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct Geo {
+  static constexpr int kTileBytes = kTok * D * 2;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with `parity` to complete; false after ~2^31 clock
+// cycles (about a second) or 2^24 polls, whichever comes first.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  for (uint32_t i = 0; i < (1u << 24); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > (1ll << 31)) break;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int D>
+__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row,
+                                         uint32_t bar) {
+  if constexpr (D == 128) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(row), "r"(bar)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(bar)
+        : "memory");
+  }
+}
+
+// Byte address of 16-byte chunk `chunk` (0 .. D/8-1) of token row `tok` in a
+// tile written by TMA with 128-byte swizzle: row `tok` occupies D/64 lines of
+// 128 bytes; chunk c of line L sits at position c ^ (L mod 8).
+template <int D>
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int tok, int chunk) {
+  const int line = tok * (D / 64) + (chunk >> 3);
+  return tile + line * 128 + (((chunk & 7) ^ (line & 7)) << 4);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+template <typename T>
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4],
+                                         const uint32_t (&b)[2]);
+
+template <>
+__device__ __forceinline__ void mma16816<__half>(float (&c)[4], const uint32_t (&a)[4],
+                                                 const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+template <>
+__device__ __forceinline__ void mma16816<__nv_bfloat16>(float (&c)[4], const uint32_t (&a)[4],
+                                                        const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Block id of unit u (or -1 past the worker's range), for the id window.
+__device__ __forceinline__ int32_t unit_block_id(const DecodeArgs& a, const int32_t* cum,
+                                                 int64_t u, int64_t u1) {
+  if (u >= u1) return -1;
+  const int b = find_seq(cum, a.batch, u, a.num_kv_heads);
+  const int nblk = cum[b + 1] - cum[b];
+  const int64_t rem = u - static_cast<int64_t>(a.num_kv_heads) * cum[b];
+  const int j = static_cast<int>(rem % nblk);
+  return __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j]);
+}
+
+__device__ __forceinline__ int stages_in_block(int ctx, int j, int bs) {
+  const int rem = ctx - j * bs;
+  const int n = rem < bs ? rem : bs;
+  return (n + kTok - 1) / kTok;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, DecodeArgs a) {
+  using G_ = Geo<D>;
+  constexpr int KC = D / 16;  // 16-wide chunks of head_dim
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t ring0 = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (ring0 - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + G_::kRingBytes);
+  int32_t* slot_ok = reinterpret_cast<int32_t*>(bars + kWarps * kStages);
+  int32_t* cum = slot_ok + kWarps * kStages;
+  int32_t* ctx_s = cum + a.batch + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+  }
+  scan_context(a, cum, ctx_s);  // ends with __syncthreads()
+
+  const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
+  const int bs = a.block_size;
+  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
+  if (U == 0) return;
+  const int64_t W = U < a.workers ? U : a.workers;
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+  if (w >= W) return;
+  const int64_t u0 = split_start(w, U, W), u1 = split_start(w + 1, U, W);
+
+  const uint32_t ring = ring0 + warp * kStages * G_::kStageBytes;
+  const uint32_t bar0 = smem_u32(&bars[warp * kStages]);
+  int32_t* ok = slot_ok + warp * kStages;
+
+  // ---------------- producer state (uniform across the warp) ----------------
+  UnitCursor pc;
+  cursor_seek(pc, u0, u1, cum, B, Hkv);
+  int psub = 0;
+  int pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+  int64_t win = u0;
+  int32_t ids_cur = unit_block_id(a, cum, u0 + lane, u1);
+  int32_t ids_next = unit_block_id(a, cum, u0 + 32 + lane, u1);
+
+  auto produce = [&](int slot) {
+    if (pc.u >= win + 32) {
+      win += 32;
+      ids_cur = ids_next;
+      ids_next = unit_block_id(a, cum, win + 32 + lane, u1);
+    }
+    const int32_t id = __shfl_sync(kFull, ids_cur, static_cast<int>(pc.u - win));
+    if (lane == 0) {
+      const uint32_t bar = bar0 + slot * 8;
+      if (id >= 0 && id < a.num_blocks) {
+        ok[slot] = 1;
+        mbar_arrive_expect_tx(bar, G_::kStageBytes);
+        const int row = (id * Hkv + pc.kvh) * bs + psub * kTok;
+        const uint32_t dst = ring + slot * G_::kStageBytes;
+        tma_tile<D>(dst, &kmap, row, bar);
+        tma_tile<D>(dst + G_::kTileBytes, &vmap, row, bar);
+      } else {
+        ok[slot] = 0;
+        report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+        mbar_arrive(bar);
+      }
+    }
+    if (++psub == pnsub) {
+      psub = 0;
+      cursor_next(pc, cum, Hkv);
+      if (pc.u < pc.u_end) pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+    }
+  };
+
+  int issued = 0;
+  for (; issued < kStages && pc.u < u1; ++issued) produce(issued);
+
+  // ---------------- consumer state ----------------
+  UnitCursor cc;
+  cursor_seek(cc, u0, u1, cum, B, Hkv);
+  int csub = 0;
+  bool seg_start = true, first_seg = true, timed_out = false;
+  int seg_j0 = 0;
+  int slot = 0;
+  uint32_t phases = 0;
+  int consumed = 0;
+  const int g = lane >> 2, cq = lane & 3;
+  uint32_t qf[KC][2];
+  float o[KC][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  while (cc.u < u1) {
+    if (seg_start) {
+      const T* qb = static_cast<const T*>(a.q) + (static_cast<int64_t>(cc.b) * Hq + cc.kvh * G) * D;
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+        if (g < G) {
+          qf[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 2 * cq));
+          qf[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 8 + 2 * cq));
+        } else {
+          qf[kc][0] = qf[kc][1] = 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[kc][i] = 0.f;
+      }
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+      seg_j0 = cc.j;
+      seg_start = false;
+    }
+
+    const uint32_t bar = bar0 + slot * 8;
+    // all lanes take the same decision, so the warp never splits on a timeout
+    if (!__all_sync(kFull, mbar_wait_bounded(bar, (phases >> slot) & 1u))) {
+      if (lane == 0) report(a.dev_error, PA_DEVERR_TIMEOUT);
+      timed_out = true;
+      break;
+    }
+    phases ^= 1u << slot;
+    ++consumed;
+
+    const int ctx = ctx_s[cc.b];
+    const int tok0 = cc.j * bs + csub * kTok;
+    const int n_valid = ctx - tok0 < kTok ? ctx - tok0 : kTok;
+    const uint32_t kt = ring + slot * G_::kStageBytes;
+    const uint32_t vt = kt + G_::kTileBytes;
+    if (ok[slot]) {
+      if (n_valid < kTok) {
+        // rows past the context may hold anything (even NaN): clear them in V
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        for (int off = n_valid * D * 2 + lane * 16; off < G_::kTileBytes; off += 512) {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vt + off), "r"(z.x),
+                       "r"(z.y), "r"(z.z), "r"(z.w)
+                       : "memory");
+        }
+        __syncwarp();
+      }
+      // S^T = K . Q^T  (two accumulators to halve the dependent chain)
+      float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int mi = lane >> 3;
+        const int tok = ((mi & 1) << 3) + (lane & 7);
+#pragma unroll
+        for (int kc = 0; kc < KC; ++kc) {
+          uint32_t ka[4];
+          ldsm_x4(swz<D>(kt, tok, 2 * kc + (mi >> 1)), ka);
+          if (kc & 1) mma16816<T>(s2, ka, qf[kc]); else mma16816<T>(s, ka, qf[kc]);
+        }
+      }
+      // scores of (tok g, head 2cq), (g, 2cq+1), (g+8, 2cq), (g+8, 2cq+1)
+      float t0 = (s[0] + s2[0]) * a.scale_log2, t1 = (s[1] + s2[1]) * a.scale_log2;
+      float t2 = (s[2] + s2[2]) * a.scale_log2, t3 = (s[3] + s2[3]) * a.scale_log2;
+      if (g >= n_valid) t0 = t1 = -INFINITY;
+      if (g + 8 >= n_valid) t2 = t3 = -INFINITY;
+      float x0 = fmaxf(t0, t2), x1 = fmaxf(t1, t3);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, off));
+        x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, off));
+      }
+      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+      const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
+      const float p0 = exp2f(t0 - n0), p1 = exp2f(t1 - n1);
+      const float p2 = exp2f(t2 - n0), p3 = exp2f(t3 - n1);
+      l0 = l0 * a0 + p0 + p2;
+      l1 = l1 * a1 + p1 + p3;
+      m0 = n0;
+      m1 = n1;
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+        o[kc][0] *= a0;
+        o[kc][1] *= a1;
+        o[kc][2] *= a0;
+        o[kc][3] *= a1;
+      }
+      const uint32_t pb[2] = {transpose8x8(pack2<T>(p0, p1)), transpose8x8(pack2<T>(p2, p3))};
+      // O^T += V^T . P^T
+      {
+        const int mi = lane >> 3;
+        const int tok = ((mi >> 1) << 3) + (lane & 7);
+#pragma unroll
+        for (int mt = 0; mt < KC; ++mt) {
+          uint32_t va[4];
+          ldsm_x4_trans(swz<D>(vt, tok, 2 * mt + (mi & 1)), va);
+          mma16816<T>(o[mt], va, pb);
+        }
+      }
+    }
+
+    // hand the slot back to TMA
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (pc.u < u1) {
+      produce(slot);
+      ++issued;
+    }
+
+    const int nsub = stages_in_block(ctx, cc.j, bs);
+    if (csub + 1 == nsub) {
+      const bool seg_end = (cc.u + 1 == u1) || (cc.j + 1 == cc.nblk);
+      if (seg_end) {
+        float L0 = l0, L1 = l1;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          L0 += __shfl_xor_sync(kFull, L0, off);
+          L1 += __shfl_xor_sync(kFull, L1, off);
+        }
+        const int h0 = 2 * cq, h1 = 2 * cq + 1;
+        const bool complete = seg_j0 == 0 && cc.j + 1 == cc.nblk;
+        if (complete) {
+          T* ob = static_cast<T*>(a.out) + (static_cast<int64_t>(cc.b) * Hq + cc.kvh * G) * D;
+          const float i0 = 1.f / L0, i1 = 1.f / L1;
+#pragma unroll
+          for (int mt = 0; mt < KC; ++mt) {
+            const int d = mt * 16 + g;
+            if (h0 < G) {
+              ob[h0 * D + d] = Num<T>::from_f(o[mt][0] * i0);
+              ob[h0 * D + d + 8] = Num<T>::from_f(o[mt][2] * i0);
+            }
+            if (h1 < G) {
+              ob[h1 * D + d] = Num<T>::from_f(o[mt][1] * i1);
+              ob[h1 * D + d + 8] = Num<T>::from_f(o[mt][3] * i1);
+            }
+          }
+        } else {
+          float* piece = a.ws_pieces + (w * 2 + (first_seg ? 0 : 1)) * (G * (D + 2));
+          if (g == 0) {
+            if (h0 < G) { piece[h0] = m0; piece[G + h0] = L0; }
+            if (h1 < G) { piece[h1] = m1; piece[G + h1] = L1; }
+          }
+          float* po = piece + 2 * G;
+#pragma unroll
+          for (int mt = 0; mt < KC; ++mt) {
+            const int d = mt * 16 + g;
+            if (h0 < G) {
+              po[h0 * D + d] = o[mt][0];
+              po[h0 * D + d + 8] = o[mt][2];
+            }
+            if (h1 < G) {
+              po[h1 * D + d] = o[mt][1];
+              po[h1 * D + d + 8] = o[mt][3];
+            }
+          }
+        }
+        first_seg = false;
+        seg_start = true;
+      }
+      csub = 0;
+      cursor_next(cc, cum, Hkv);
+    } else {
+      ++csub;
+    }
+    slot = slot + 1 == kStages ? 0 : slot + 1;
+  }
+
+  if (timed_out) {
+    // let copies already in flight land before the CTA's shared memory goes away
+    for (int k = consumed; k < issued; ++k) {
+      const int s_ = k % kStages;
+      mbar_wait_bounded(bar0 + s_ * 8, (phases >> s_) & 1u);
+      phases ^= 1u << s_;
+    }
+  }
+}
+
+template <typename T, int D>
+static cudaError_t launch_t(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
+                            int num_ctas, cudaStream_t stream) {
+  const size_t smem = decode_tc_smem_bytes(D, a.batch);
+  auto kern = decode_tc_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<num_ctas, kWarps * 32, smem, stream>>>(kmap, vmap, a);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+int decode_tc_workers_per_cta() { return tc::kWarps; }
+
+size_t decode_tc_smem_bytes(int head_dim, int batch) {
+  const size_t ring = static_cast<size_t>(tc::kWarps) * tc::kStages * 2 * tc::kTok * head_dim * 2;
+  const size_t meta = tc::kWarps * tc::kStages * (8 + 4) + sizeof(int32_t) * (2 * batch + 1);
+  return 1024 + ring + meta;
+}
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
+                             const CUtensorMap& vmap, int num_ctas, cudaStream_t stream) {
+  if (a.head_dim == 128) {
+    return dtype == PA_F16 ? tc::launch_t<__half, 128>(a, kmap, vmap, num_ctas, stream)
+                           : tc::launch_t<__nv_bfloat16, 128>(a, kmap, vmap, num_ctas, stream);
+  }
+  return dtype == PA_F16 ? tc::launch_t<__half, 64>(a, kmap, vmap, num_ctas, stream)
+                         : tc::launch_t<__nv_bfloat16, 64>(a, kmap, vmap, num_ctas, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,68 @@
+"""Runs a workload through the CUDA library (test infrastructure)."""
+import numpy as np
+import torch
+
+import workloads
+from paged_kv_cache_486_b200.engine import PagedKVCache
+
+NAN_BITS = {"f32": 0x7FC00000, "f16": 0x7E00, "bf16": 0x7FC0}
+
+
+def tol_ok(got, ref, dtype):
+    """Spec bar for fp16/bf16: |got - ref| <= 2e-3 + 1e-2 |ref|; fp32: 1e-5 + 1e-4 |ref|."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    atol, rtol = (1e-5, 1e-4) if dtype == "f32" else (2e-3, 1e-2)
+    err = np.abs(got - ref)
+    bound = atol + rtol * np.abs(ref)
+    ok = bool(np.all(err <= bound)) and bool(np.all(np.isfinite(got)))
+    worst = float(np.max(err / bound)) if err.size else 0.0
+    return ok, worst
+
+
+def build(wl, poison=True, batched_step=True, path=0, workers=0, stream=None):
+    """Prefill the pools from the op script, then run the decode step: one new
+    token per sequence (one batched cache write), then decode attention."""
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda",
+                       fill_bits=NAN_BITS[wl.dtype] if poison else None)
+
+    def tokens(seq, pos0, n):
+        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
+
+    pre = eng.apply_ops(wl.ops[:wl.n_prefill_ops], tokens, stream)
+    step_ops = wl.ops[wl.n_prefill_ops:]
+    if batched_step:
+        slots, keys, vals, step = [], [], [], []
+        for op in step_ops:
+            _, seq, n, pos0, _w = op
+            s, cow = eng.alloc(seq, n, stream)
+            step.append((s, cow))
+            slots.append(s)
+            k, v = tokens(seq, pos0, n)
+            keys.append(k)
+            vals.append(v)
+        eng.write(torch.cat(keys), torch.cat(vals), np.concatenate(slots), stream)
+    else:
+        step = eng.apply_ops(step_ops, tokens, stream)
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    q = wl.q("cuda")
+    out = eng.decode(q, bt, ctx, wl.scale, path=path, num_workers=workers, stream=stream)
+    torch.cuda.synchronize()
+    return dict(eng=eng, records=pre + step, bt=bt, ctx=ctx, q=q, out=out)
+
+
+def gathered(eng, bt, ctx, b, kind, heads=None):
+    """Cache rows of batch row b in logical order, read back through its table (torch indexing)."""
+    cache = eng.k_cache if kind == 0 else eng.v_cache
+    n = int(ctx[b])
+    bs = cache.shape[2]
+    pos = torch.arange(n, device=cache.device)
+    blocks = bt[b].long()[pos // bs]
+    rows = cache[blocks, :, pos % bs, :]  # [n, Hkv, D]
+    return rows if heads is None else rows[:, heads, :]
+
+
+def bits(t):
+    t = t.contiguous()
+    return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)

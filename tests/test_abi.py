@@ -1,0 +1,107 @@
+"""The C ABI library loads without a GPU, exports every function include/*.h
+declares, and rejects bad arguments on the host before any device work."""
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_486_b200 as pa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(pa_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    declared = _declared()
+    assert len(declared) >= 20
+    raw = C.CDLL(pa.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+        assert name in pa.SIGNATURES, f"binding lacks {name}"
+
+
+def test_loaded_library_is_the_in_tree_build():
+    assert os.path.dirname(pa.LIB_PATH) == os.path.join(ROOT, "paged_kv_cache_486_b200")
+    assert os.path.exists(pa.LIB_PATH)
+
+
+def test_kv_bytes():
+    assert pa.pa_kv_bytes(80, 1, 8, 128, 2) == 327680
+    assert pa.pa_kv_bytes(32, 4096, 8, 128, 2) == 2 * 32 * 4096 * 8 * 128 * 2
+
+
+def _decode_args(**kw):
+    args = dict(out=C.c_void_p(16), q=C.c_void_p(16), k=C.c_void_p(16), v=C.c_void_p(16),
+                bt=C.c_void_p(16), ctx=C.c_void_p(16), B=4, Hq=8, Hkv=2, D=128, bs=16, NB=10,
+                MB=4, scale=0.1, dtype=pa.PA_F16, ws=C.c_void_p(16), ws_bytes=1 << 30, err=None,
+                path=0, workers=0, stream=None)
+    args.update(kw)
+    return args
+
+
+def _call_decode(a):
+    return pa.lib.pa_decode_attention_ex(a["out"], a["q"], a["k"], a["v"], a["bt"], a["ctx"],
+                                         a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"],
+                                         a["MB"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"],
+                                         a["err"], a["path"], a["workers"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(D=96), dict(Hq=7), dict(Hkv=0), dict(bs=12), dict(B=-1), dict(B=5000), dict(dtype=7),
+    dict(ws_bytes=16), dict(q=None), dict(k=C.c_void_p(8)), dict(path=9),
+    dict(path=pa.PA_PATH_TC, dtype=pa.PA_F32), dict(path=pa.PA_PATH_TC, Hq=32, Hkv=2),
+    dict(path=pa.PA_PATH_TC, bs=8), dict(NB=1 << 24, Hkv=16, Hq=16), dict(scale=float("nan")),
+])
+def test_decode_rejects_bad_arguments_on_host(bad):
+    st = _call_decode(_decode_args(**bad))
+    assert st == pa.PA_ERR_INVALID, pa.pa_last_error()
+    assert pa.pa_last_error()
+
+
+def test_empty_batch_is_a_no_op():
+    assert _call_decode(_decode_args(B=0, q=None, out=None)) == pa.PA_OK
+
+
+def test_cache_write_and_copy_reject_bad_arguments():
+    p = C.c_void_p(16)
+    assert pa.lib.pa_reshape_and_cache(p, p, p, p, p, 4, 8, 100, 16, 10, pa.PA_F16, None,
+                                       None) == pa.PA_ERR_INVALID  # 200-byte rows
+    assert pa.lib.pa_reshape_and_cache(p, p, p, p, p, -1, 8, 128, 16, 10, pa.PA_F16, None,
+                                       None) == pa.PA_ERR_INVALID
+    assert pa.lib.pa_reshape_and_cache(C.c_void_p(8), p, p, p, p, 4, 8, 128, 16, 10, pa.PA_F16,
+                                       None, None) == pa.PA_ERR_INVALID
+    assert pa.lib.pa_reshape_and_cache(p, p, p, p, p, 0, 8, 128, 16, 10, pa.PA_F16, None,
+                                       None) == pa.PA_OK
+    arr = (C.c_void_p * 1)(16)
+    assert pa.lib.pa_copy_blocks(arr, arr, 0, p, 1, 10, 4096, None, None) == pa.PA_ERR_INVALID
+    assert pa.lib.pa_copy_blocks(arr, arr, 129, p, 1, 10, 4096, None, None) == pa.PA_ERR_INVALID
+    assert pa.lib.pa_copy_blocks(arr, arr, 1, p, 1, 10, 4100, None, None) == pa.PA_ERR_INVALID
+    assert pa.lib.pa_copy_blocks(arr, arr, 1, p, 0, 10, 4096, None, None) == pa.PA_OK
+
+
+def test_workspace_size_is_independent_of_context_and_grows_with_group():
+    a = pa.pa_decode_workspace_size(64, 32, 8, 128)
+    b = pa.pa_decode_workspace_size(256, 64, 8, 128)
+    assert 0 < a < b < (64 << 20)
+    assert pa.pa_decode_workspace_size(4, 7, 2, 128) == 0
+
+
+def test_plan_chooses_tensor_cores_where_they_apply():
+    import torch
+    assert pa.pa_decode_plan(64, 32, 8, 128, 16, torch.float16)[0] == pa.PA_PATH_TC
+    assert pa.pa_decode_plan(64, 64, 8, 128, 16, torch.bfloat16)[0] == pa.PA_PATH_TC
+    assert pa.pa_decode_plan(64, 64, 64, 128, 32, torch.float16)[0] == pa.PA_PATH_TC
+    assert pa.pa_decode_plan(4, 4, 2, 64, 16, torch.float32)[0] == pa.PA_PATH_SIMT
+    assert pa.pa_decode_plan(4, 32, 2, 128, 16, torch.float16)[0] == pa.PA_PATH_SIMT
+    assert pa.pa_decode_plan(4, 8, 2, 128, 8, torch.float16)[0] == pa.PA_PATH_SIMT

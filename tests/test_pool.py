@@ -1,0 +1,132 @@
+"""The product's host block pool against the oracle's pool model: identical
+slots, copy pairs, block tables, free counts and holder counts, bit for bit,
+on every workload script and on random op scripts; plus the validators."""
+import numpy as np
+import pytest
+
+import oracle
+import paged_kv_cache_486_b200 as pa
+import workloads
+
+
+def _same_state(p, o, nb, seqs, max_blocks):
+    assert p.pa_num_free_blocks() == o.num_free()
+    for b in range(nb):
+        assert p.pa_refcount(b) == o.holders(b)
+    if seqs:
+        t1, c1 = p.pa_block_table(seqs, max_blocks)
+        st, t2, c2 = o.block_table(seqs, max_blocks)
+        assert st == oracle.OK
+        assert np.array_equal(t1, t2) and np.array_equal(c1, c2)
+
+
+def _run_both(wl):
+    p = pa.Pool(wl.num_blocks, wl.bs)
+    o = oracle.Pool(wl.num_blocks, wl.bs)
+    for op in wl.ops:
+        if op[0] == "alloc":
+            slots, cow = p.pa_alloc(op[1], op[2])
+            st, slots2, cow2 = o.alloc(op[1], op[2])
+            assert st == oracle.OK
+            assert np.array_equal(slots, slots2) and np.array_equal(cow, cow2)
+        elif op[0] == "fork":
+            p.pa_fork(op[1], op[2])
+            assert o.fork(op[1], op[2]) == oracle.OK
+        else:
+            p.pa_free(op[1])
+            assert o.free(op[1]) == oracle.OK
+    _same_state(p, o, wl.num_blocks, list(wl.batch), wl.max_blocks)
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama3_8b", "shared_prefix", "llama3_70b"])
+def test_workload_scripts_match_the_oracle(name):
+    _run_both(workloads.make(name))
+
+
+def test_random_scripts_match_the_oracle():
+    rng = np.random.default_rng(99)
+    for trial in range(30):
+        nb, bs = int(rng.integers(1, 50)), int(rng.choice([1, 3, 8, 16]))
+        p, o = pa.Pool(nb, bs), oracle.Pool(nb, bs)
+        live = set()
+        for _ in range(250):
+            r = rng.random()
+            if r < 0.5 or not live:
+                s, n = int(rng.integers(0, 10)), int(rng.integers(0, 3 * bs + 1))
+                st, slots2, cow2 = o.alloc(s, n)
+                try:
+                    slots, cow = p.pa_alloc(s, n)
+                    assert st == oracle.OK
+                    assert np.array_equal(slots, slots2) and np.array_equal(cow, cow2)
+                    live.add(s)
+                except pa.PagedAttnError as e:
+                    assert e.status == st == pa.PA_ERR_OOM
+            elif r < 0.7:
+                parent, child = int(rng.choice(sorted(live))), int(rng.integers(0, 10))
+                st = o.fork(parent, child)
+                try:
+                    p.pa_fork(parent, child)
+                    assert st == oracle.OK
+                    live.add(child)
+                except pa.PagedAttnError as e:
+                    assert e.status == st
+            else:
+                s = int(rng.choice(sorted(live)))
+                p.pa_free(s)
+                assert o.free(s) == oracle.OK
+                live.discard(s)
+            _same_state(p, o, nb, sorted(live), nb + 1)
+
+
+def test_errors_and_atomicity():
+    p = pa.Pool(4, 4)
+    with pytest.raises(pa.PagedAttnError) as e:
+        p.pa_free(1)
+    assert e.value.status == pa.PA_ERR_NOT_FOUND
+    p.pa_alloc(1, 10)
+    p.pa_fork(1, 2)
+    before = (p.pa_num_free_blocks(), [p.pa_refcount(b) for b in range(4)])
+    with pytest.raises(pa.PagedAttnError) as e:
+        p.pa_alloc(2, 7)
+    assert e.value.status == pa.PA_ERR_OOM
+    assert (p.pa_num_free_blocks(), [p.pa_refcount(b) for b in range(4)]) == before
+    with pytest.raises(pa.PagedAttnError) as e:
+        p.pa_fork(1, 2)
+    assert e.value.status == pa.PA_ERR_INVALID
+    with pytest.raises(pa.PagedAttnError):
+        p.pa_block_table([1], 2)
+    assert p.pa_refcount(-1) == -1 and p.pa_refcount(4) == -1
+    assert p.pa_seq_len(1) == 10 and p.pa_seq_len(9) == -1
+
+
+def test_validators():
+    assert pa.pa_validate_slot_mapping([0, 5, -1, 63], 16, 4) == pa.PA_OK
+    assert pa.pa_validate_slot_mapping([0, 64], 16, 4) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_slot_mapping([3, 3], 16, 4) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_slot_mapping([-2], 16, 4) == pa.PA_ERR_INVALID
+    t = np.array([[0, 1, -1], [2, -1, -1]], np.int32)
+    assert pa.pa_validate_block_table(t, np.array([20, 16], np.int32), 16, 3) == pa.PA_OK
+    assert pa.pa_validate_block_table(t, np.array([33, 16], np.int32), 16, 3) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_block_table(t, np.array([20, 17], np.int32), 16, 3) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_block_table(t, np.array([20, 16], np.int32), 16, 2) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_copy_pairs([[1, 2], [3, 4]], 5) == pa.PA_OK
+    assert pa.pa_validate_copy_pairs([[1, 2], [3, 2]], 5) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_copy_pairs([[1, 2], [2, 4]], 5) == pa.PA_ERR_INVALID
+    assert pa.pa_validate_copy_pairs([[1, 5]], 5) == pa.PA_ERR_INVALID
+
+
+def test_pool_slots_are_valid_for_the_kernels():
+    wl = workloads.make("shared_prefix")
+    p = pa.Pool(wl.num_blocks, wl.bs)
+    for op in wl.ops:
+        if op[0] == "alloc":
+            slots, cow = p.pa_alloc(op[1], op[2])
+            assert pa.pa_validate_slot_mapping(slots, wl.bs, wl.num_blocks) == pa.PA_OK
+            if len(cow):
+                assert pa.pa_validate_copy_pairs(cow, wl.num_blocks) == pa.PA_OK
+        elif op[0] == "fork":
+            p.pa_fork(op[1], op[2])
+        else:
+            p.pa_free(op[1])
+    t, c = p.pa_block_table(wl.batch, wl.max_blocks)
+    assert pa.pa_validate_block_table(t, c, wl.bs, wl.num_blocks) == pa.PA_OK
