@@ -173,6 +173,27 @@ __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+template <typename T>
+__device__ __forceinline__ float2 unpack2(uint32_t x);
+template <>
+__device__ __forceinline__ float2 unpack2<__half>(uint32_t x) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&x));
+}
+template <>
+__device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t x) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
+}
+
+// Softmax weights as a head + tail pair of 16-bit values (p = head + tail up to
+// ~16 significant bits), so that P . V keeps fp32-like accuracy even for bf16,
+// whose 8-bit significand alone would cost ~2^-9 |v| wherever outputs cancel.
+template <typename T>
+__device__ __forceinline__ void split2(float a, float b, uint32_t& head, uint32_t& tail) {
+  head = pack2<T>(a, b);
+  const float2 h = unpack2<T>(head);
+  tail = pack2<T>(a - h.x, b - h.y);
+}
+
 // Block id of unit u (or -1 past the worker's range), for the id window.
 __device__ __forceinline__ int32_t unit_block_id(const DecodeArgs& a, const int32_t* cum,
                                                  int64_t u, int64_t u1) {
@@ -366,8 +387,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         o[kc][2] *= a0;
         o[kc][3] *= a1;
       }
-      const uint32_t pb[2] = {transpose8x8(pack2<T>(p0, p1)), transpose8x8(pack2<T>(p2, p3))};
-      // O^T += V^T . P^T
+      uint32_t h01, t01, h23, t23;
+      split2<T>(p0, p1, h01, t01);
+      split2<T>(p2, p3, h23, t23);
+      const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
+      const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
+      // O^T += V^T . (P_head + P_tail)^T
       {
         const int mi = lane >> 3;
         const int tok = ((mi >> 1) << 3) + (lane & 7);
@@ -376,6 +401,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
           uint32_t va[4];
           ldsm_x4_trans(swz<D>(vt, tok, 2 * mt + (mi & 1)), va);
           mma16816<T>(o[mt], va, pb);
+          mma16816<T>(o[mt], va, pt);
         }
       }
     }
