@@ -208,6 +208,29 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                                  int32_t* dev_error, int32_t path, int32_t num_workers,
                                  pa_stream stream);
 
+/* pa_decode_attention without a caller-provided workspace.  The pages have
+ * no counterpart to this call; it exists for callers that cannot allocate
+ * device memory (an embedding host that hands out none, a serving loop that
+ * must not call cudaMalloc while requests run, a process whose memory another
+ * runtime has reserved).  The scratch is one area of 18 MiB that the library
+ * declares in device memory; every GPU that loads the library holds it until
+ * the process exits.  Arguments, results and errors are those of
+ * pa_decode_attention, plus PA_ERR_INVALID if a shape would need more scratch
+ * than the area holds.  Nothing is allocated by this call.
+ * The first call on a device looks up the area's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins.  All calls share the one area, which keeps whatever the last
+ * call left in it: calls whose work overlaps on the GPU (different streams,
+ * or different host threads on one device) race on it and must be ordered by
+ * the caller. */
+pa_status pa_decode_attention_static_ws(void* out, const void* q, const void* k_cache,
+                                        const void* v_cache, const int32_t* block_tables,
+                                        const int32_t* context_lens, int32_t batch,
+                                        int32_t num_q_heads, int32_t num_kv_heads,
+                                        int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                        int32_t max_blocks, float scale, pa_dtype dtype,
+                                        int32_t* dev_error, pa_stream stream);
+
 /* Path and worker count pa_decode_attention would use for these arguments. */
 pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                          int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* path_out,

@@ -49,6 +49,8 @@ SIGNATURES = {
     "pa_decode_attention_ex": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                       _I32, _I32, C.c_float, C.c_int, _P, C.c_size_t, _P, _I32,
                                       _I32, _P]),
+    "pa_decode_attention_static_ws": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
+                                             _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
     "pa_decode_plan": (_I32, [_I32, _I32, _I32, _I32, _I32, C.c_int, _P, _P]),
     "pa_validate_slot_mapping": (_I32, [_P, _I32, _I32, _I32]),
     "pa_validate_block_table": (_I32, [_P, _P, _I32, _I32, _I32, _I32]),
@@ -225,6 +227,25 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, sc
         workspace.numel() * workspace.element_size(),
         _dev_ptr(dev_error, "dev_error", torch.int32), path, num_workers, _stream(stream))
     _check(st, "pa_decode_attention")
+
+
+def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                                  dev_error=None, stream=None):
+    """pa_decode_attention for callers that cannot allocate device memory: the
+    library's own fixed 18 MiB device scratch replaces the workspace.  Calls that
+    overlap on the GPU share that scratch and race; order them on one stream."""
+    B, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    MB = block_tables.shape[1]
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    st = lib.pa_decode_attention_static_ws(
+        _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache", q.dtype),
+        _dev_ptr(v_cache, "v_cache", q.dtype), _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(context_lens, "context_lens", torch.int32), B, Hq, Hkv, D, bs, NB, MB,
+        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32),
+        _stream(stream))
+    _check(st, "pa_decode_attention_static_ws")
 
 
 def pa_check_device_error(dev_error, stream=None) -> int:

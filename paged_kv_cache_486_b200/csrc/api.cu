@@ -345,3 +345,77 @@ pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_strea
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention for callers that cannot allocate device memory.
+//
+// pa_decode_attention needs a scratch buffer from its caller.  Some callers
+// have no way to provide one: an embedding host that owns every device
+// allocation and exposes none to plug-ins, a serving loop that must never call
+// cudaMalloc while requests are in flight (the call can synchronise the device
+// and stall every other stream), or a process whose memory is fully reserved
+// by another runtime's caching allocator.  For them the library keeps one
+// scratch area of its own in device memory, declared below, and
+// pa_decode_attention_static_ws uses it instead of a caller buffer.
+//
+// The area is kStaticScratchBytes (18 MiB): enough for the largest workspace
+// any shape pa_decode_attention accepts can ask for (2048 workers x 8 heads x
+// (128 + 2) floats x 2 pieces, plus the batch prefix sums).  Every GPU that
+// loads this library holds those 18 MiB until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kStaticScratchBytes = size_t(18) << 20;
+}
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+namespace {
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {};
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// symbol name is only a host-side handle, so the address is looked up once per
+// device (with that device current) and remembered.
+pa_status static_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention_static_ws (cudaGetDevice)");
+  if (dev < 0 || dev >= 64)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_static_ws: device %d not supported", dev);
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess)
+      return cuda_fail(e, "pa_decode_attention_static_ws (cudaGetSymbolAddress)");
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_attention_static_ws(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t num_blocks, int32_t max_blocks, float scale, pa_dtype dtype, int32_t* dev_error,
+    pa_stream stream) {
+  const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim);
+  if (need > kStaticScratchBytes)
+    return fail(PA_ERR_INVALID,
+                "pa_decode_attention_static_ws: this shape needs %zu bytes of scratch, more "
+                "than the library's fixed %zu-byte area; use pa_decode_attention with a "
+                "caller-provided workspace", need, kStaticScratchBytes);
+  void* scratch = nullptr;
+  const pa_status st = static_scratch(&scratch);
+  if (st != PA_OK) return st;
+  // Nothing in the scratch needs to start at zero: every call writes each byte
+  // of it that it later reads (prefix sums first, then the split pieces).
+  return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
+                                num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                max_blocks, scale, dtype, scratch, kStaticScratchBytes,
+                                dev_error, PA_PATH_AUTO, 0, stream);
+}
