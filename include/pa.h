@@ -172,13 +172,14 @@ pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
  *   nearest even, from fp32 accumulators.
  * block_tables: [batch, max_blocks] int32, device; context_lens: [batch] int32.
  * head_dim in {64, 128}; block_size in {8, 16, 32, 64, 128}; batch <= 4096;
- * num_blocks * num_kv_heads * block_size < 2^31.
+ * batch * num_kv_heads <= 262144; num_blocks * num_kv_heads * block_size < 2^31.
  * workspace: device scratch of at least pa_decode_workspace_size(...) bytes,
  *   16-byte aligned, contents need no initialisation; calls that share a
  *   workspace must be ordered on one stream.
  * The work is split evenly across the GPU by KV blocks: a sequence that fits in
  * one worker's share is done in a single pass; a longer one is cut into pieces
- * whose (max, sum, partial output) are merged by a log-sum-exp combine kernel.
+ * whose (max, sum, partial output) are merged with a log-sum-exp combine by the
+ * worker that finishes the last piece.  One kernel launch per call.
  * ---------------------------------------------------------------------- */
 size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                 int32_t head_dim);
@@ -212,7 +213,7 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
  * no counterpart to this call; it exists for callers that cannot allocate
  * device memory (an embedding host that hands out none, a serving loop that
  * must not call cudaMalloc while requests run, a process whose memory another
- * runtime has reserved).  The scratch is one area of 18 MiB that the library
+ * runtime has reserved).  The scratch is one area of 20 MiB that the library
  * declares in device memory; every GPU that loads the library holds it until
  * the process exits.  Arguments, results and errors are those of
  * pa_decode_attention, plus PA_ERR_INVALID if a shape would need more scratch

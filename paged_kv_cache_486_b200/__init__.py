@@ -232,7 +232,7 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, sc
 def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                                   dev_error=None, stream=None):
     """pa_decode_attention for callers that cannot allocate device memory: the
-    library's own fixed 18 MiB device scratch replaces the workspace.  Calls that
+    library's own fixed 20 MiB device scratch replaces the workspace.  Calls that
     overlap on the GPU share that scratch and race; order them on one stream."""
     B, Hq, D = q.shape
     NB, Hkv, bs, _ = k_cache.shape

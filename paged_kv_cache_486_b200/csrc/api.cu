@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -56,30 +57,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // A pool [num_blocks, Hkv, bs, D] seen as `rows` rows of D elements; one box is
-// 16 rows x D, delivered with 128-byte swizzle (D = 128: 3-d view 64 x 2 x rows).
+// 16 rows x 64 columns (128 bytes, the 128-byte swizzle span).
 bool make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim, pa_dtype dt) {
   auto enc = encode_fn();
   if (!enc) return false;
   const CUtensorMapDataType t =
       dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  CUresult r;
-  if (head_dim == 128) {
-    cuuint64_t dims[3] = {64, 2, static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[2] = {128, 256};
-    cuuint32_t box[3] = {64, 2, 16};
-    cuuint32_t es[3] = {1, 1, 1};
-    r = enc(map, t, 3, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  } else {
-    cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, 16};
-    cuuint32_t es[2] = {1, 1};
-    r = enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  }
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -125,9 +115,19 @@ bool tc_applies(int group, int head_dim, int block_size, pa_dtype dt) {
          block_size % 16 == 0;
 }
 
-size_t pieces_offset(int batch) {
-  const size_t cum = (sizeof(int32_t) * (static_cast<size_t>(batch) + 1) + 255) & ~size_t(255);
-  return 256 + cum;
+// Workspace: [256 reserved][arrival words: B * Hkv x 8 bytes][pieces].
+size_t pieces_offset(int batch, int num_kv_heads) {
+  const size_t arrivals = (sizeof(unsigned long long) * static_cast<size_t>(batch) * num_kv_heads +
+                           255) & ~size_t(255);
+  return 256 + arrivals;
+}
+
+// Nonzero tag per decode call for the arrival words.
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> epoch{0};
+  uint32_t e = ++epoch;
+  while (e == 0) e = ++epoch;
+  return e;
 }
 
 }  // namespace
@@ -193,7 +193,7 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_
       num_q_heads % num_kv_heads || head_dim < 1)
     return 0;
   const int group = num_q_heads / num_kv_heads;
-  return pieces_offset(batch) +
+  return pieces_offset(batch, num_kv_heads) +
          sizeof(float) * 2 * static_cast<size_t>(max_workers(group)) * group * (head_dim + 2);
 }
 
@@ -249,6 +249,9 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_INVALID, "pa_decode_attention: num_blocks * num_kv_heads * block_size "
                 "= %lld >= 2^31", static_cast<long long>(rows));
   if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention: scale is NaN");
+  if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: batch * num_kv_heads = %lld > %d",
+                static_cast<long long>(batch) * num_kv_heads, pa::kMaxArrivals);
   if (path != PA_PATH_AUTO && path != PA_PATH_TC && path != PA_PATH_SIMT)
     return fail(PA_ERR_INVALID, "pa_decode_attention: unknown path %d", path);
   if (batch == 0) return PA_OK;
@@ -284,8 +287,10 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.dev_error = dev_error;
-  a.ws_cum = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + 256);
-  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) + pieces_offset(batch));
+  a.ws_arrivals =
+      reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + 256);
+  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         pieces_offset(batch, num_kv_heads));
   a.batch = batch;
   a.num_q_heads = num_q_heads;
   a.num_kv_heads = num_kv_heads;
@@ -295,6 +300,7 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.num_blocks = num_blocks;
   a.max_blocks = max_blocks;
   a.workers = workers;
+  a.epoch = next_epoch();
   a.scale_log2 = scale * 1.4426950408889634f;
 
   cudaError_t e;
@@ -310,8 +316,6 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
     e = pa::launch_decode_simt(a, dtype, static_cast<cudaStream_t>(stream));
   }
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention (decode kernel)");
-  e = pa::launch_combine(a, dtype, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention (combine kernel)");
   return PA_OK;
 }
 
@@ -358,13 +362,14 @@ pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_strea
 // scratch area of its own in device memory, declared below, and
 // pa_decode_attention_static_ws uses it instead of a caller buffer.
 //
-// The area is kStaticScratchBytes (18 MiB): enough for the largest workspace
+// The area is kStaticScratchBytes (20 MiB): enough for the largest workspace
 // any shape pa_decode_attention accepts can ask for (2048 workers x 8 heads x
-// (128 + 2) floats x 2 pieces, plus the batch prefix sums).  Every GPU that
-// loads this library holds those 18 MiB until the process exits.
+// (128 + 2) floats x 2 pieces, plus one 8-byte arrival word for each of at most
+// 262144 (sequence, kv head) pairs).  Every GPU that loads this library holds
+// those 20 MiB until the process exits.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr size_t kStaticScratchBytes = size_t(18) << 20;
+constexpr size_t kStaticScratchBytes = size_t(20) << 20;
 }
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
@@ -412,8 +417,10 @@ extern "C" pa_status pa_decode_attention_static_ws(
   void* scratch = nullptr;
   const pa_status st = static_scratch(&scratch);
   if (st != PA_OK) return st;
-  // Nothing in the scratch needs to start at zero: every call writes each byte
-  // of it that it later reads (prefix sums first, then the split pieces).
+  // Nothing in the scratch needs to start at zero: the split pieces are written
+  // before they are read, and each arrival word is tagged with its call's epoch
+  // (a word from an earlier call reads as zero) and cleared by the call that
+  // completes it.
   return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, scratch, kStaticScratchBytes,

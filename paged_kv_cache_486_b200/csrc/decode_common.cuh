@@ -8,7 +8,9 @@
 // gets the same number of KV bytes to within one block.  A run of units of
 // one (b, kv head) inside one worker is a "segment".  A segment that holds a
 // whole (b, kv head) writes the output directly (single pass); otherwise it is
-// a piece of a longer context that a log-sum-exp combine merges.  Only a
+// a piece of a longer context: the worker stores the piece's (max, sum,
+// unnormalised output) and the worker whose piece arrives last merges all of
+// them with a log-sum-exp combine (piece_done below).  Only a
 // worker's first and last segments can be pieces, so each worker owns two
 // piece slots: slot 0 for the segment that contains start(w), slot 1 for its
 // last segment.
@@ -29,6 +31,7 @@ namespace pa {
 constexpr int kMaxBatch = 4096;
 constexpr int kMaxWorkers = 2048;
 constexpr int kPieceHeadBudget = 16384;  // workers x G kept in the workspace
+constexpr int kMaxArrivals = 262144;     // batch x kv heads (arrival words)
 
 struct DecodeArgs {
   void* out;
@@ -38,11 +41,12 @@ struct DecodeArgs {
   const int32_t* block_tables;
   const int32_t* context_lens;
   int32_t* dev_error;
-  int32_t* ws_cum;      // [B + 1] written by CTA 0
+  unsigned long long* ws_arrivals;  // [B * Hkv] piece arrival words (epoch << 32 | count)
   float* ws_pieces;     // [2 * max_workers][G * (D + 2)]
   int32_t batch, num_q_heads, num_kv_heads, group, head_dim, block_size;
   int32_t num_blocks, max_blocks;
   int32_t workers;      // workers launched (the split uses min(workers, U))
+  uint32_t epoch;       // nonzero tag of this call for the arrival words
   float scale_log2;     // scale * log2(e)
 };
 
@@ -108,8 +112,16 @@ __device__ inline void scan_context(const DecodeArgs& a, int32_t* cum, int32_t* 
   }
   if (threadIdx.x == nt - 1) cum[B] = run;
   __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int b = threadIdx.x; b <= B; b += nt) a.ws_cum[b] = cum[b];
+}
+
+// Rows of sequences with an empty context are zero; CTA (b mod grid) writes them.
+template <typename T>
+__device__ inline void zero_empty_rows(const DecodeArgs& a, const int32_t* ctx_s) {
+  const int per_row = a.num_q_heads * a.head_dim;
+  for (int b = blockIdx.x; b < a.batch; b += gridDim.x) {
+    if (ctx_s[b] != 0) continue;
+    T* o = static_cast<T*>(a.out) + static_cast<int64_t>(b) * per_row;
+    for (int i = threadIdx.x; i < per_row; i += blockDim.x) o[i] = T(0.f);
   }
 }
 
@@ -158,8 +170,132 @@ __device__ inline void cursor_next(UnitCursor& c, const int32_t* cum, int Hkv) {
   }
 }
 
-// ------------------------------- dtypes ------------------------------------
+// ------------------------- merging split contexts --------------------------
+// A worker that has written a piece of (b, kv head) announces it on the pair's
+// arrival word; the warp whose piece completes the set merges all pieces:
+//   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,
+// then clears the word.  Words carry the call's epoch in their high half, so a
+// word left by an earlier call counts as zero.
+__device__ inline uint32_t arrive_piece(unsigned long long* word, uint32_t epoch,
+                                        int32_t* dev_error) {
+  unsigned long long old = atomicAdd(word, 0ull);
+  for (int i = 0; i < (1 << 20); ++i) {
+    const uint32_t e = static_cast<uint32_t>(old >> 32);
+    const uint32_t n = (e == epoch) ? static_cast<uint32_t>(old) : 0u;
+    const unsigned long long want = (static_cast<unsigned long long>(epoch) << 32) | (n + 1u);
+    const unsigned long long seen = atomicCAS(word, old, want);
+    if (seen == old) return n + 1u;
+    old = seen;
+  }
+  report(dev_error, PA_DEVERR_TIMEOUT);
+  return 0u;
+}
+
+__device__ inline float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__device__ inline float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
 template <typename T> struct Num;
+
+// Whole warp, after its piece of (b, kvh) is stored.  cum: block prefix sums.
+// The merge keeps many loads in flight: pass 1 spreads the pieces over the
+// lanes to find each head's max and sum; pass 2 gives every lane the columns
+// d = lane + 32k of a few heads and walks the pieces, each step issuing all of
+// that piece's loads for the lane at once.
+template <typename T, int D>
+__device__ inline void piece_done(const DecodeArgs& a, const int32_t* cum, int b, int kvh,
+                                  int64_t U, int64_t W, int lane) {
+  constexpr int PER = D / 32;
+  constexpr int HG = 16 / PER;  // heads merged per pass (16 accumulators per lane)
+  const int Hkv = a.num_kv_heads, G = a.group;
+  const int nblk = cum[b + 1] - cum[b];
+  const int64_t u0 = static_cast<int64_t>(Hkv) * cum[b] + static_cast<int64_t>(kvh) * nblk;
+  const int64_t wf = split_worker_of(u0, U, W);
+  const int64_t wl = split_worker_of(u0 + nblk - 1, U, W);
+  __syncwarp();
+  __threadfence();  // this warp's piece is visible before it is announced
+  __syncwarp();
+  uint32_t n = 0;
+  if (lane == 0) n = arrive_piece(&a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh], a.epoch,
+                                  a.dev_error);
+  n = __shfl_sync(0xffffffffu, n, 0);
+  const int np = static_cast<int>(wl - wf + 1);
+  if (n != static_cast<uint32_t>(np)) return;
+  __threadfence();  // every other piece is visible to this warp
+  // only the first piece can sit in slot 1 (its worker started before u0)
+  const int first_slot = split_start(wf, U, W) >= u0 ? 0 : 1;
+  const int pf = G * (D + 2);
+  const float* base = a.ws_pieces + (wf * 2 + first_slot) * pf;  // piece 0
+  const float* rest = a.ws_pieces + (wf + 1) * 2 * pf;            // piece p >= 1: rest + 2 pf (p - 1)
+  auto piece = [&](int p) { return p == 0 ? base : rest + static_cast<int64_t>(2 * pf) * (p - 1); };
+  T* out = static_cast<T*>(a.out) + (static_cast<int64_t>(b) * a.num_q_heads + kvh * G) * D;
+  for (int h0 = 0; h0 < G; h0 += HG) {
+    const int nh = G - h0 < HG ? G - h0 : HG;
+    float M[HG], L[HG], O[HG][PER];
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) {
+      M[hh] = -INFINITY;
+      L[hh] = 0.f;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) O[hh][k] = 0.f;
+    }
+    for (int p = lane; p < np; p += 32) {
+      const float* pc = piece(p);
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh)
+        if (hh < nh) M[hh] = fmaxf(M[hh], __ldcg(pc + h0 + hh));
+    }
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) M[hh] = warp_max(M[hh]);
+    for (int p = lane; p < np; p += 32) {
+      const float* pc = piece(p);
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh)
+        if (hh < nh) L[hh] = fmaf(exp2f(__ldcg(pc + h0 + hh) - M[hh]), __ldcg(pc + G + h0 + hh),
+                                  L[hh]);
+    }
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) L[hh] = warp_sum(L[hh]);
+#pragma unroll 1
+    for (int p = 0; p < np; ++p) {
+      const float* pc = piece(p);
+      float e[HG], v[HG][PER];
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh) {
+        e[hh] = hh < nh ? __ldcg(pc + h0 + hh) : 0.f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k)
+          v[hh][k] = hh < nh ? __ldcg(pc + 2 * G + (h0 + hh) * D + lane + 32 * k) : 0.f;
+      }
+#pragma unroll
+      for (int hh = 0; hh < HG; ++hh) {
+        const float wgt = hh < nh ? exp2f(e[hh] - M[hh]) : 0.f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) O[hh][k] = fmaf(wgt, v[hh][k], O[hh][k]);
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < HG; ++hh) {
+      if (hh < nh) {
+        const float inv = 1.f / L[hh];
+#pragma unroll
+        for (int k = 0; k < PER; ++k)
+          out[(h0 + hh) * D + lane + 32 * k] = Num<T>::from_f(O[hh][k] * inv);
+      }
+    }
+  }
+  if (lane == 0) a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh] = 0ull;
+}
+
+// ------------------------------- dtypes ------------------------------------
 template <> struct Num<float> {
   __device__ static float to_f(float x) { return x; }
   __device__ static float from_f(float x) { return x; }

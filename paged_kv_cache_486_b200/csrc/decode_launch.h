@@ -18,7 +18,4 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensor
 int decode_tc_workers_per_cta();
 size_t decode_tc_smem_bytes(int head_dim, int batch);
 
-// Merge pieces of split contexts and zero the rows of empty ones.
-cudaError_t launch_combine(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream);
-
 }  // namespace pa

@@ -1,5 +1,4 @@
-// Paged decode attention on CUDA cores (every dtype and head grouping), and the
-// log-sum-exp combine that merges pieces of a split context.
+// Paged decode attention on CUDA cores (every dtype and head grouping).
 //
 // Each warp is one worker of the even split described in decode_common.cuh.
 // Within a segment the warp walks the sequence's blocks through its block-table
@@ -24,6 +23,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
   int32_t* cum = simt_smem;
   int32_t* ctx_s = simt_smem + a.batch + 1;
   scan_context(a, cum, ctx_s);
+  zero_empty_rows<T>(a, ctx_s);
 
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
   const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
@@ -135,49 +135,11 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
         }
       }
     }
+    if (!complete) piece_done<T, D>(a, cum, b, kvh, U, W, lane);
     first_seg = false;
     c.u += seg - 1;
     c.j = j1 - 1;
     cursor_next(c, cum, Hkv);
-  }
-}
-
-// One CTA per (b, kv head): zero rows of empty contexts; merge the pieces of a
-// split context:  M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-template <typename T>
-__global__ void __launch_bounds__(256) combine_kernel(DecodeArgs a) {
-  const int Hkv = a.num_kv_heads, G = a.group, D = a.head_dim, B = a.batch;
-  const int b = blockIdx.x / Hkv, kvh = blockIdx.x % Hkv;
-  const int32_t* cum = a.ws_cum;
-  const int nblk = cum[b + 1] - cum[b];
-  T* out = static_cast<T*>(a.out) + (static_cast<int64_t>(b) * a.num_q_heads + kvh * G) * D;
-  if (nblk == 0) {
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[i] = Num<T>::from_f(0.f);
-    return;
-  }
-  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
-  const int64_t W = U < a.workers ? U : a.workers;
-  const int64_t u0 = static_cast<int64_t>(Hkv) * cum[b] + static_cast<int64_t>(kvh) * nblk;
-  const int64_t wf = split_worker_of(u0, U, W);
-  const int64_t wl = split_worker_of(u0 + nblk - 1, U, W);
-  if (wf == wl) return;  // done in one pass by one worker
-  const int piece_floats = G * (D + 2);
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int h = i / D, d = i - h * D;
-    float M = -INFINITY;
-    for (int64_t w = wf; w <= wl; ++w) {
-      const int slot = split_start(w, U, W) >= u0 ? 0 : 1;
-      M = fmaxf(M, a.ws_pieces[(w * 2 + slot) * piece_floats + h]);
-    }
-    float L = 0.f, O = 0.f;
-    for (int64_t w = wf; w <= wl; ++w) {
-      const int slot = split_start(w, U, W) >= u0 ? 0 : 1;
-      const float* piece = a.ws_pieces + (w * 2 + slot) * piece_floats;
-      const float e = exp2f(piece[h] - M);
-      L = fmaf(e, piece[G + h], L);
-      O = fmaf(e, piece[2 * G + h * D + d], O);
-    }
-    out[h * D + d] = Num<T>::from_f(O / L);
   }
 }
 
@@ -198,15 +160,6 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, cudaStream_t
   if (dtype == PA_F32) return launch_simt_t<float, 128>(a, stream);
   if (dtype == PA_F16) return launch_simt_t<__half, 128>(a, stream);
   return launch_simt_t<__nv_bfloat16, 128>(a, stream);
-}
-
-cudaError_t launch_combine(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream) {
-  const int grid = a.batch * a.num_kv_heads;
-  if (grid == 0) return cudaSuccess;
-  if (dtype == PA_F32) combine_kernel<float><<<grid, 256, 0, stream>>>(a);
-  else if (dtype == PA_F16) combine_kernel<__half><<<grid, 256, 0, stream>>>(a);
-  else combine_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a);
-  return cudaGetLastError();
 }
 
 }  // namespace pa

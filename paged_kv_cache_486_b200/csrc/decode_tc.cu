@@ -13,9 +13,12 @@
 //
 // Data movement.  Every warp is an independent worker (see decode_common.cuh)
 // with its own ring of kStages stage buffers.  Lane 0 issues, kStages stages
-// ahead of the consumer, two TMA tile loads per stage: 16 rows x D of the key
-// pool and of the value pool, rows (block * Hkv + kv_head) * block_size + 16s,
-// landing 128-byte-swizzled so ldmatrix reads them without bank conflicts.
+// ahead of the consumer, the TMA loads of a stage: 16 rows x D of the key pool
+// and of the value pool, rows (block * Hkv + kv_head) * block_size + 16s, each
+// as D/64 boxes of 16 rows x 64 columns.  A box lands 128-byte-swizzled with
+// one row per 128-byte line, so the eight rows an ldmatrix reads sit in eight
+// different bank groups (with whole 256-byte rows in one box, rows t and t+4
+// would share banks).
 // Block ids come from the block table through a per-warp window of 32 ids
 // held one per lane and loaded one window ahead.  Each stage signals an
 // mbarrier with its byte count; every wait on it is bounded in time.
@@ -91,31 +94,26 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+constexpr int kBoxBytes = kTok * 64 * 2;  // one 16 x 64 box of 16-bit elements
+
+// The tile of 16 rows x D: D/64 boxes, box h holding columns [64h, 64h + 64).
 template <int D>
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row,
                                          uint32_t bar) {
-  if constexpr (D == 128) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(row), "r"(bar)
-        : "memory");
-  } else {
+#pragma unroll
+  for (int h = 0; h < D / 64; ++h) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(bar)
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst + h * kBoxBytes),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(64 * h), "r"(row), "r"(bar)
         : "memory");
   }
 }
 
-// Byte address of 16-byte chunk `chunk` (0 .. D/8-1) of token row `tok` in a
-// tile written by TMA with 128-byte swizzle: row `tok` occupies D/64 lines of
-// 128 bytes; chunk c of line L sits at position c ^ (L mod 8).
-template <int D>
+// Byte address of 16-byte chunk `chunk` (0 .. D/8-1) of token row `tok`: box
+// chunk / 8, line tok, position (chunk mod 8) ^ (tok mod 8) (128-byte swizzle).
 __device__ __forceinline__ uint32_t swz(uint32_t tile, int tok, int chunk) {
-  const int line = tok * (D / 64) + (chunk >> 3);
-  return tile + line * 128 + (((chunk & 7) ^ (line & 7)) << 4);
+  return tile + (chunk >> 3) * kBoxBytes + tok * 128 + (((chunk & 7) ^ (tok & 7)) << 4);
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -234,6 +232,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
   }
   scan_context(a, cum, ctx_s);  // ends with __syncthreads()
+  zero_empty_rows<T>(a, ctx_s);
 
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
   const int bs = a.block_size;
@@ -299,21 +298,32 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   uint32_t phases = 0;
   int consumed = 0;
   const int g = lane >> 2, cq = lane & 3;
-  uint32_t qf[KC][2];
+  uint32_t qf[KC][2], qn[KC][2];
   float o[KC][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
+  // Query fragments (B operand, k = head_dim, n = head) of pair (b, kvh):
+  // lane (g, cq) holds q[g][16kc + 2cq, +1] and q[g][16kc + 8 + 2cq, +1].
+  auto load_q = [&](uint32_t (&dst)[KC][2], int b, int kvh) {
+    const T* qb = static_cast<const T*>(a.q) + (static_cast<int64_t>(b) * Hq + kvh * G) * D;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+      if (g < G) {
+        dst[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 2 * cq));
+        dst[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 8 + 2 * cq));
+      } else {
+        dst[kc][0] = dst[kc][1] = 0u;
+      }
+    }
+  };
+  load_q(qn, cc.b, cc.kvh);
+
   while (cc.u < u1) {
     if (seg_start) {
-      const T* qb = static_cast<const T*>(a.q) + (static_cast<int64_t>(cc.b) * Hq + cc.kvh * G) * D;
 #pragma unroll
       for (int kc = 0; kc < KC; ++kc) {
-        if (g < G) {
-          qf[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 2 * cq));
-          qf[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 8 + 2 * cq));
-        } else {
-          qf[kc][0] = qf[kc][1] = 0u;
-        }
+        qf[kc][0] = qn[kc][0];
+        qf[kc][1] = qn[kc][1];
 #pragma unroll
         for (int i = 0; i < 4; ++i) o[kc][i] = 0.f;
       }
@@ -321,6 +331,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       l0 = l1 = 0.f;
       seg_j0 = cc.j;
       seg_start = false;
+      // start fetching the next segment's queries now; they are used only then
+      const int64_t next_u = cc.u + (cc.nblk - cc.j);
+      if (next_u < u1) {
+        int nb = cc.b, nk = cc.kvh + 1;
+        if (nk == Hkv) {
+          nk = 0;
+          do {
+            ++nb;
+          } while (cum[nb + 1] == cum[nb]);
+        }
+        load_q(qn, nb, nk);
+      }
     }
 
     const uint32_t bar = bar0 + slot * 8;
@@ -338,28 +360,44 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     const int n_valid = ctx - tok0 < kTok ? ctx - tok0 : kTok;
     const uint32_t kt = ring + slot * G_::kStageBytes;
     const uint32_t vt = kt + G_::kTileBytes;
-    if (ok[slot]) {
+    const bool have = ok[slot] != 0;
+    // Move the stage into registers first and hand the slot straight back to
+    // TMA, so the ring keeps loading while this warp computes.
+    uint32_t ka[KC][4], va[KC][4];
+    if (have) {
       if (n_valid < kTok) {
         // rows past the context may hold anything (even NaN): clear them in V
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-        for (int off = n_valid * D * 2 + lane * 16; off < G_::kTileBytes; off += 512) {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vt + off), "r"(z.x),
-                       "r"(z.y), "r"(z.z), "r"(z.w)
+        const int per_box = (kTok - n_valid) * 8;  // 16-byte chunks past the context
+        for (int i = lane; i < per_box * (D / 64); i += 32) {
+          const int h = i / per_box, r = i - h * per_box;
+          const uint32_t addr = vt + h * kBoxBytes + n_valid * 128 + r * 16;
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
                        : "memory");
         }
         __syncwarp();
       }
+      const int mi = lane >> 3;
+      const int ktok = ((mi & 1) << 3) + (lane & 7);
+      const int vtok = ((mi >> 1) << 3) + (lane & 7);
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        ldsm_x4(swz(kt, ktok, 2 * c + (mi >> 1)), ka[c]);
+        ldsm_x4_trans(swz(vt, vtok, 2 * c + (mi & 1)), va[c]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (pc.u < u1) {
+      produce(slot);
+      ++issued;
+    }
+
+    if (have) {
       // S^T = K . Q^T  (two accumulators to halve the dependent chain)
       float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const int mi = lane >> 3;
-        const int tok = ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
-          uint32_t ka[4];
-          ldsm_x4(swz<D>(kt, tok, 2 * kc + (mi >> 1)), ka);
-          if (kc & 1) mma16816<T>(s2, ka, qf[kc]); else mma16816<T>(s, ka, qf[kc]);
-        }
+      for (int kc = 0; kc < KC; ++kc) {
+        if (kc & 1) mma16816<T>(s2, ka[kc], qf[kc]); else mma16816<T>(s, ka[kc], qf[kc]);
       }
       // scores of (tok g, head 2cq), (g, 2cq+1), (g+8, 2cq), (g+8, 2cq+1)
       float t0 = (s[0] + s2[0]) * a.scale_log2, t1 = (s[1] + s2[1]) * a.scale_log2;
@@ -373,45 +411,36 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, off));
       }
       const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
       const float p0 = exp2f(t0 - n0), p1 = exp2f(t1 - n1);
       const float p2 = exp2f(t2 - n0), p3 = exp2f(t3 - n1);
-      l0 = l0 * a0 + p0 + p2;
-      l1 = l1 * a1 + p1 + p3;
-      m0 = n0;
-      m1 = n1;
+      // rescale the running sums only when some head's maximum moved
+      if (__any_sync(kFull, n0 > m0 || n1 > m1)) {
+        const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
+        l0 *= a0;
+        l1 *= a1;
 #pragma unroll
-      for (int kc = 0; kc < KC; ++kc) {
-        o[kc][0] *= a0;
-        o[kc][1] *= a1;
-        o[kc][2] *= a0;
-        o[kc][3] *= a1;
+        for (int kc = 0; kc < KC; ++kc) {
+          o[kc][0] *= a0;
+          o[kc][1] *= a1;
+          o[kc][2] *= a0;
+          o[kc][3] *= a1;
+        }
+        m0 = n0;
+        m1 = n1;
       }
+      l0 += p0 + p2;
+      l1 += p1 + p3;
       uint32_t h01, t01, h23, t23;
       split2<T>(p0, p1, h01, t01);
       split2<T>(p2, p3, h23, t23);
       const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
       const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
       // O^T += V^T . (P_head + P_tail)^T
-      {
-        const int mi = lane >> 3;
-        const int tok = ((mi >> 1) << 3) + (lane & 7);
 #pragma unroll
-        for (int mt = 0; mt < KC; ++mt) {
-          uint32_t va[4];
-          ldsm_x4_trans(swz<D>(vt, tok, 2 * mt + (mi & 1)), va);
-          mma16816<T>(o[mt], va, pb);
-          mma16816<T>(o[mt], va, pt);
-        }
+      for (int mt = 0; mt < KC; ++mt) {
+        mma16816<T>(o[mt], va[mt], pb);
+        mma16816<T>(o[mt], va[mt], pt);
       }
-    }
-
-    // hand the slot back to TMA
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (pc.u < u1) {
-      produce(slot);
-      ++issued;
     }
 
     const int nsub = stages_in_block(ctx, cc.j, bs);
@@ -460,6 +489,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
               po[h1 * D + d + 8] = o[mt][3];
             }
           }
+          piece_done<T, D>(a, cum, cc.b, cc.kvh, U, W, lane);
         }
         first_seg = false;
         seg_start = true;
@@ -487,9 +517,18 @@ static cudaError_t launch_t(const DecodeArgs& a, const CUtensorMap& kmap, const 
                             int num_ctas, cudaStream_t stream) {
   const size_t smem = decode_tc_smem_bytes(D, a.batch);
   auto kern = decode_tc_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  // the opt-in shared-memory limit is per device; raise it once to the most any
+  // batch can ask for
+  static bool raised[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !raised[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(decode_tc_smem_bytes(D, kMaxBatch)));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) raised[dev] = true;
+  }
   kern<<<num_ctas, kWarps * 32, smem, stream>>>(kmap, vmap, a);
   return cudaGetLastError();
 }
