@@ -137,20 +137,29 @@ def _dist():
     return None, 0, 1
 
 
-def _max_over_ranks(dist, x):
+def _reduce(dist, x, op):
     if dist is None:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def _max_over_ranks(dist, x):
+    return _reduce(dist, x, None if dist is None else dist.ReduceOp.MAX)
 
 
 def _sum_over_ranks(dist, x):
-    if dist is None:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(dist, x, None if dist is None else dist.ReduceOp.SUM)
+
+
+def aggregate(dist, local_ms, local_tokens):
+    """Whole-job throughput of independent replicas: tokens summed over ranks divided
+    by the slowest rank's device time.  Returns (max_ms, tokens, tokens/s)."""
+    total_ms = _max_over_ranks(dist, local_ms)
+    tokens = _sum_over_ranks(dist, local_tokens)
+    return total_ms, tokens, tokens / (total_ms / 1e3)
 
 
 # --------------------------------------------------------------- our arm
@@ -240,9 +249,7 @@ def run_ours(args, dist, rank, world):
     torch.cuda.synchronize()
     assert eng.device_errors() == 0, "device guards fired"
 
-    total_ms = _max_over_ranks(dist, sum(step_ms))
-    tokens_all = _sum_over_ranks(dist, wl.B * args.steps)
-    value = tokens_all / (total_ms / 1e3)
+    total_ms, _, value = aggregate(dist, sum(step_ms), wl.B * args.steps)
     alg = wl.kv_read_bytes()
     dec_ms = statistics.mean(decode_ms)
     achieved = alg / (dec_ms / 1e3) / 1e9
@@ -333,10 +340,9 @@ def run_e2e(args, wl, eng, dist):
         e1.record(stream)
         e1.synchronize()
         ms.append(e0.elapsed_time(e1))
-    total = _max_over_ranks(dist, sum(ms))
-    tokens_all = _sum_over_ranks(dist, wl.B * args.steps)
+    total, _, e2e_value = aggregate(dist, sum(ms), wl.B * args.steps)
     assert torch.isfinite(h_out.float()).all()
-    return {"value": tokens_all / (total / 1e3), "unit": "tokens/s",
+    return {"value": e2e_value, "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": total / args.steps}
 
