@@ -196,10 +196,20 @@ pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, con
 #define PA_PATH_TC 1     /* fp16/bf16, G <= 8, block_size a multiple of 16 */
 #define PA_PATH_SIMT 2   /* every supported shape and dtype */
 
-/* As pa_decode_attention, with the path and the number of workers (warps that
- * split the KV blocks; 0 = automatic, else clamped to the supported range)
- * chosen by the caller.  Every choice gives the same result up to fp32
- * rounding order. */
+/* Flags for pa_decode_attention_ex.
+ * PA_DECODE_OVERLAP_PROLOGUE: launch the decode kernel so that its prologue runs
+ * while the kernel before it on `stream` finishes (programmatic dependent
+ * launch).  The prologue reads context_lens, block_tables and q; everything
+ * else (the caches, out, the workspace) is touched only after the preceding
+ * kernel has completed.  Use it only when that preceding kernel does not write
+ * context_lens, block_tables or q -- e.g. right after pa_reshape_and_cache or
+ * pa_copy_blocks, which write only the caches. */
+#define PA_DECODE_OVERLAP_PROLOGUE 1
+
+/* As pa_decode_attention, with the path, the number of workers (warps that
+ * split the KV blocks; 0 = automatic, else clamped to the supported range) and
+ * flags chosen by the caller.  Every path and worker count gives the same result
+ * up to fp32 rounding order. */
 pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                                  const void* v_cache, const int32_t* block_tables,
                                  const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
@@ -207,7 +217,7 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                                  int32_t num_blocks, int32_t max_blocks, float scale,
                                  pa_dtype dtype, void* workspace, size_t workspace_bytes,
                                  int32_t* dev_error, int32_t path, int32_t num_workers,
-                                 pa_stream stream);
+                                 int32_t flags, pa_stream stream);
 
 /* pa_decode_attention without a caller-provided workspace.  The pages have
  * no counterpart to this call; it exists for callers that cannot allocate

@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
 PA_OK, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_NOT_FOUND, PA_ERR_CUDA, PA_ERR_DEVICE = range(6)
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 PA_PATH_AUTO, PA_PATH_TC, PA_PATH_SIMT = 0, 1, 2
+PA_DECODE_OVERLAP_PROLOGUE = 1
 PA_DEVERR_BAD_SLOT, PA_DEVERR_BAD_BLOCK, PA_DEVERR_BAD_CTX, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 DTYPE_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
@@ -48,7 +49,7 @@ SIGNATURES = {
                                    _I32, C.c_float, C.c_int, _P, C.c_size_t, _P, _P]),
     "pa_decode_attention_ex": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                       _I32, _I32, C.c_float, C.c_int, _P, C.c_size_t, _P, _I32,
-                                      _I32, _P]),
+                                      _I32, _I32, _P]),
     "pa_decode_attention_static_ws": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                              _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
     "pa_decode_plan": (_I32, [_I32, _I32, _I32, _I32, _I32, C.c_int, _P, _P]),
@@ -211,7 +212,7 @@ def pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, dtype
 
 
 def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, scale, workspace,
-                        dev_error=None, path=PA_PATH_AUTO, num_workers=0, stream=None):
+                        dev_error=None, path=PA_PATH_AUTO, num_workers=0, flags=0, stream=None):
     """q/out [B, Hq, D]; caches [NB, Hkv, bs, D]; block_tables int32 [B, MB];
     context_lens int32 [B]; workspace uint8 [>= pa_decode_workspace_size] (all CUDA)."""
     B, Hq, D = q.shape
@@ -225,7 +226,7 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, sc
         _dev_ptr(context_lens, "context_lens", torch.int32), B, Hq, Hkv, D, bs, NB, MB,
         float(scale), DTYPE_CODE[q.dtype], _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(),
-        _dev_ptr(dev_error, "dev_error", torch.int32), path, num_workers, _stream(stream))
+        _dev_ptr(dev_error, "dev_error", torch.int32), path, num_workers, flags, _stream(stream))
     _check(st, "pa_decode_attention")
 
 

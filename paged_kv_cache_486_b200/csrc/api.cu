@@ -227,7 +227,7 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                                  int32_t num_blocks, int32_t max_blocks, float scale,
                                  pa_dtype dtype, void* workspace, size_t workspace_bytes,
                                  int32_t* dev_error, int32_t path, int32_t num_workers,
-                                 pa_stream stream) {
+                                 int32_t flags, pa_stream stream) {
   if (!valid_dtype(dtype))
     return fail(PA_ERR_INVALID, "pa_decode_attention: unknown dtype %d", static_cast<int>(dtype));
   if (batch < 0 || batch > pa::kMaxBatch)
@@ -254,6 +254,9 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                 static_cast<long long>(batch) * num_kv_heads, pa::kMaxArrivals);
   if (path != PA_PATH_AUTO && path != PA_PATH_TC && path != PA_PATH_SIMT)
     return fail(PA_ERR_INVALID, "pa_decode_attention: unknown path %d", path);
+  if (flags & ~PA_DECODE_OVERLAP_PROLOGUE)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: unknown flags 0x%x", flags);
+  const bool overlap = (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0;
   if (batch == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
     return fail(PA_ERR_INVALID, "pa_decode_attention: NULL pointer");
@@ -310,10 +313,10 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
         !tile_map(&vmap, v_cache, rows, head_dim, dtype))
       return fail(PA_ERR_CUDA, "pa_decode_attention: cuTensorMapEncodeTiled failed");
     const int per = pa::decode_tc_workers_per_cta();
-    e = pa::launch_decode_tc(a, dtype, kmap, vmap, (workers + per - 1) / per,
+    e = pa::launch_decode_tc(a, dtype, kmap, vmap, (workers + per - 1) / per, overlap,
                              static_cast<cudaStream_t>(stream));
   } else {
-    e = pa::launch_decode_simt(a, dtype, static_cast<cudaStream_t>(stream));
+    e = pa::launch_decode_simt(a, dtype, overlap, static_cast<cudaStream_t>(stream));
   }
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention (decode kernel)");
   return PA_OK;
@@ -328,7 +331,7 @@ pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, con
   return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, workspace, workspace_bytes, dev_error,
-                                PA_PATH_AUTO, 0, stream);
+                                PA_PATH_AUTO, 0, 0, stream);
 }
 
 pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {
@@ -424,5 +427,5 @@ extern "C" pa_status pa_decode_attention_static_ws(
   return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, scratch, kStaticScratchBytes,
-                                dev_error, PA_PATH_AUTO, 0, stream);
+                                dev_error, PA_PATH_AUTO, 0, 0, stream);
 }

@@ -23,6 +23,9 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
                                          int64_t total_chunks, int32_t row_chunks,
                                          int32_t num_kv_heads, int32_t block_size,
                                          int64_t num_slots, int32_t* dev_error) {
+  // a decode launched to overlap its prologue with this kernel may start now; it
+  // waits for this grid before it reads the cache
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int32_t token_chunks = row_chunks * num_kv_heads;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total_chunks;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -54,6 +57,7 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant_
                                                           const int32_t* __restrict__ pairs,
                                                           int32_t num_blocks, int64_t block_chunks,
                                                           int32_t* dev_error) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int32_t pair = blockIdx.x;
   const int32_t layer = blockIdx.y >> 1;
   const bool is_v = blockIdx.y & 1;

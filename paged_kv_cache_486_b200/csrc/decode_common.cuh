@@ -59,6 +59,10 @@ __host__ __device__ inline int64_t split_worker_of(int64_t u, int64_t U, int64_t
   return ((u + 1) * W - 1) / U;
 }
 
+// Waits for the grid this launch depends on (a no-op unless the decode was
+// launched to overlap its prologue with the preceding kernel).
+__device__ inline void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ inline void report(int32_t* dev_error, int32_t bits) {
   if (dev_error) atomicOr(dev_error, bits);
 }
@@ -207,14 +211,15 @@ template <typename T> struct Num;
 
 // Whole warp, after its piece of (b, kvh) is stored.  cum: block prefix sums.
 // The merge keeps many loads in flight: pass 1 spreads the pieces over the
-// lanes to find each head's max and sum; pass 2 gives every lane the columns
-// d = lane + 32k of a few heads and walks the pieces, each step issuing all of
-// that piece's loads for the lane at once.
+// lanes and finds each head's max and sum in one round of loads; pass 2 gives
+// every lane the columns d = lane + 32k of a few heads and walks the pieces two
+// at a time, each round issuing all of their loads for the lane at once.
 template <typename T, int D>
 __device__ inline void piece_done(const DecodeArgs& a, const int32_t* cum, int b, int kvh,
                                   int64_t U, int64_t W, int lane) {
   constexpr int PER = D / 32;
   constexpr int HG = 16 / PER;  // heads merged per pass (16 accumulators per lane)
+  constexpr int PQ = 2;         // pieces loaded per round in pass 2
   const int Hkv = a.num_kv_heads, G = a.group;
   const int nblk = cum[b + 1] - cum[b];
   const int64_t u0 = static_cast<int64_t>(Hkv) * cum[b] + static_cast<int64_t>(kvh) * nblk;
@@ -247,39 +252,48 @@ __device__ inline void piece_done(const DecodeArgs& a, const int32_t* cum, int b
 #pragma unroll
       for (int k = 0; k < PER; ++k) O[hh][k] = 0.f;
     }
-    for (int p = lane; p < np; p += 32) {
-      const float* pc = piece(p);
-#pragma unroll
-      for (int hh = 0; hh < HG; ++hh)
-        if (hh < nh) M[hh] = fmaxf(M[hh], __ldcg(pc + h0 + hh));
-    }
-#pragma unroll
-    for (int hh = 0; hh < HG; ++hh) M[hh] = warp_max(M[hh]);
-    for (int p = lane; p < np; p += 32) {
-      const float* pc = piece(p);
-#pragma unroll
-      for (int hh = 0; hh < HG; ++hh)
-        if (hh < nh) L[hh] = fmaf(exp2f(__ldcg(pc + h0 + hh) - M[hh]), __ldcg(pc + G + h0 + hh),
-                                  L[hh]);
-    }
-#pragma unroll
-    for (int hh = 0; hh < HG; ++hh) L[hh] = warp_sum(L[hh]);
-#pragma unroll 1
-    for (int p = 0; p < np; ++p) {
-      const float* pc = piece(p);
-      float e[HG], v[HG][PER];
+    // pass 1: (max, sum) of every head; one round of loads when np <= 32
+    for (int p0 = 0; p0 < np; p0 += 32) {
+      const int p = p0 + lane;
+      float pm[HG], pl[HG];
 #pragma unroll
       for (int hh = 0; hh < HG; ++hh) {
-        e[hh] = hh < nh ? __ldcg(pc + h0 + hh) : 0.f;
-#pragma unroll
-        for (int k = 0; k < PER; ++k)
-          v[hh][k] = hh < nh ? __ldcg(pc + 2 * G + (h0 + hh) * D + lane + 32 * k) : 0.f;
+        const bool on = p < np && hh < nh;
+        pm[hh] = on ? __ldcg(piece(p) + h0 + hh) : -INFINITY;
+        pl[hh] = on ? __ldcg(piece(p) + G + h0 + hh) : 0.f;
       }
 #pragma unroll
       for (int hh = 0; hh < HG; ++hh) {
-        const float wgt = hh < nh ? exp2f(e[hh] - M[hh]) : 0.f;
+        const float mx = fmaxf(M[hh], warp_max(pm[hh]));
+        const float part = pl[hh] == 0.f ? 0.f : pl[hh] * exp2f(pm[hh] - mx);
+        L[hh] = L[hh] * exp2f(M[hh] - mx) + warp_sum(part);
+        M[hh] = mx;
+      }
+    }
+    // pass 2: weighted sum of the pieces' outputs, PQ pieces per round of loads
+    for (int p0 = 0; p0 < np; p0 += PQ) {
+      float e[PQ][HG], v[PQ][HG][PER];
 #pragma unroll
-        for (int k = 0; k < PER; ++k) O[hh][k] = fmaf(wgt, v[hh][k], O[hh][k]);
+      for (int q = 0; q < PQ; ++q) {
+        const bool in = p0 + q < np;
+        const float* pc = piece(in ? p0 + q : 0);
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+          const bool on = in && hh < nh;
+          e[q][hh] = on ? __ldcg(pc + h0 + hh) : -INFINITY;
+#pragma unroll
+          for (int k = 0; k < PER; ++k)
+            v[q][hh][k] = on ? __ldcg(pc + 2 * G + (h0 + hh) * D + lane + 32 * k) : 0.f;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < PQ; ++q) {
+#pragma unroll
+        for (int hh = 0; hh < HG; ++hh) {
+          const float wgt = exp2f(e[q][hh] - M[hh]);
+#pragma unroll
+          for (int k = 0; k < PER; ++k) O[hh][k] = fmaf(wgt, v[q][hh][k], O[hh][k]);
+        }
       }
     }
 #pragma unroll

@@ -8,13 +8,18 @@
 namespace pa {
 
 // CUDA-core path: every dtype, head_dim 64 or 128, any group size.
-cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream);
+// overlap: launch with programmatic stream serialisation, so the prologue (which
+// reads only context_lens, block_tables and q) runs while the preceding kernel
+// finishes; the kernel waits for that kernel before touching anything else.
+cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, bool overlap,
+                               cudaStream_t stream);
 
 // Tensor-core path: fp16 / bf16, head_dim 64 or 128, group <= 8, block_size a
 // multiple of 16.  kmap / vmap describe the key / value pools as rows of
 // head_dim elements (see make_tile_maps in api.cu).
 cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
-                             const CUtensorMap& vmap, int num_ctas, cudaStream_t stream);
+                             const CUtensorMap& vmap, int num_ctas, bool overlap,
+                             cudaStream_t stream);
 int decode_tc_workers_per_cta();
 size_t decode_tc_smem_bytes(int head_dim, int batch);
 

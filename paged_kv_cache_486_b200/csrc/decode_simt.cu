@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
   int32_t* cum = simt_smem;
   int32_t* ctx_s = simt_smem + a.batch + 1;
   scan_context(a, cum, ctx_s);
+  wait_prior_grid();  // the cache, the output and the workspace are touched only after this
   zero_empty_rows<T>(a, ctx_s);
 
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
@@ -144,22 +145,32 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
 }
 
 template <typename T, int D>
-static cudaError_t launch_simt_t(const DecodeArgs& a, cudaStream_t stream) {
+static cudaError_t launch_simt_t(const DecodeArgs& a, bool overlap, cudaStream_t stream) {
   const int ctas = (a.workers + kSimtWarps - 1) / kSimtWarps;
   const size_t smem = sizeof(int32_t) * (2 * a.batch + 1);
-  decode_simt_kernel<T, D><<<ctas, kSimtWarps * 32, smem, stream>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kSimtWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_simt_kernel<T, D>, a);
 }
 
-cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, cudaStream_t stream) {
+cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, bool overlap,
+                               cudaStream_t stream) {
   if (a.head_dim == 64) {
-    if (dtype == PA_F32) return launch_simt_t<float, 64>(a, stream);
-    if (dtype == PA_F16) return launch_simt_t<__half, 64>(a, stream);
-    return launch_simt_t<__nv_bfloat16, 64>(a, stream);
+    if (dtype == PA_F32) return launch_simt_t<float, 64>(a, overlap, stream);
+    if (dtype == PA_F16) return launch_simt_t<__half, 64>(a, overlap, stream);
+    return launch_simt_t<__nv_bfloat16, 64>(a, overlap, stream);
   }
-  if (dtype == PA_F32) return launch_simt_t<float, 128>(a, stream);
-  if (dtype == PA_F16) return launch_simt_t<__half, 128>(a, stream);
-  return launch_simt_t<__nv_bfloat16, 128>(a, stream);
+  if (dtype == PA_F32) return launch_simt_t<float, 128>(a, overlap, stream);
+  if (dtype == PA_F16) return launch_simt_t<__half, 128>(a, overlap, stream);
+  return launch_simt_t<__nv_bfloat16, 128>(a, overlap, stream);
 }
 
 }  // namespace pa

@@ -232,16 +232,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
   }
   scan_context(a, cum, ctx_s);  // ends with __syncthreads()
-  zero_empty_rows<T>(a, ctx_s);
 
+  // Until wait_prior_grid() below the kernel reads only its inputs
+  // (context_lens, block_tables, q): with overlap enabled this prologue runs
+  // while the preceding kernel (typically the cache write) is still finishing.
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
   const int bs = a.block_size;
   const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
-  if (U == 0) return;
   const int64_t W = U < a.workers ? U : a.workers;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  if (w >= W) return;
-  const int64_t u0 = split_start(w, U, W), u1 = split_start(w + 1, U, W);
+  const bool active = w < W;  // false for every warp when U == 0
+  const int64_t u0 = active ? split_start(w, U, W) : 0;
+  const int64_t u1 = active ? split_start(w + 1, U, W) : 0;
 
   const uint32_t ring = ring0 + warp * kStages * G_::kStageBytes;
   const uint32_t bar0 = smem_u32(&bars[warp * kStages]);
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   UnitCursor pc;
   cursor_seek(pc, u0, u1, cum, B, Hkv);
   int psub = 0;
-  int pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+  int pnsub = active ? stages_in_block(ctx_s[pc.b], pc.j, bs) : 0;
   int64_t win = u0;
   int32_t ids_cur = unit_block_id(a, cum, u0 + lane, u1);
   int32_t ids_next = unit_block_id(a, cum, u0 + 32 + lane, u1);
@@ -285,9 +287,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
   };
 
-  int issued = 0;
-  for (; issued < kStages && pc.u < u1; ++issued) produce(issued);
-
   // ---------------- consumer state ----------------
   UnitCursor cc;
   cursor_seek(cc, u0, u1, cum, B, Hkv);
@@ -316,7 +315,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
     }
   };
-  load_q(qn, cc.b, cc.kvh);
+  if (active) load_q(qn, cc.b, cc.kvh);
+
+  wait_prior_grid();  // from here on the cache, the output and the workspace are used
+  zero_empty_rows<T>(a, ctx_s);
+  if (!active) return;
+
+  int issued = 0;
+  for (; issued < kStages && pc.u < u1; ++issued) produce(issued);
 
   while (cc.u < u1) {
     if (seg_start) {
@@ -514,7 +520,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 
 template <typename T, int D>
 static cudaError_t launch_t(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                            int num_ctas, cudaStream_t stream) {
+                            int num_ctas, bool overlap, cudaStream_t stream) {
   const size_t smem = decode_tc_smem_bytes(D, a.batch);
   auto kern = decode_tc_kernel<T, D>;
   // the opt-in shared-memory limit is per device; raise it once to the most any
@@ -529,8 +535,17 @@ static cudaError_t launch_t(const DecodeArgs& a, const CUtensorMap& kmap, const 
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) raised[dev] = true;
   }
-  kern<<<num_ctas, kWarps * 32, smem, stream>>>(kmap, vmap, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_ctas);
+  cfg.blockDim = dim3(kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a);
 }
 
 }  // namespace tc
@@ -544,13 +559,16 @@ size_t decode_tc_smem_bytes(int head_dim, int batch) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
-                             const CUtensorMap& vmap, int num_ctas, cudaStream_t stream) {
+                             const CUtensorMap& vmap, int num_ctas, bool overlap,
+                             cudaStream_t stream) {
   if (a.head_dim == 128) {
-    return dtype == PA_F16 ? tc::launch_t<__half, 128>(a, kmap, vmap, num_ctas, stream)
-                           : tc::launch_t<__nv_bfloat16, 128>(a, kmap, vmap, num_ctas, stream);
+    return dtype == PA_F16
+               ? tc::launch_t<__half, 128>(a, kmap, vmap, num_ctas, overlap, stream)
+               : tc::launch_t<__nv_bfloat16, 128>(a, kmap, vmap, num_ctas, overlap, stream);
   }
-  return dtype == PA_F16 ? tc::launch_t<__half, 64>(a, kmap, vmap, num_ctas, stream)
-                         : tc::launch_t<__nv_bfloat16, 64>(a, kmap, vmap, num_ctas, stream);
+  return dtype == PA_F16
+             ? tc::launch_t<__half, 64>(a, kmap, vmap, num_ctas, overlap, stream)
+             : tc::launch_t<__nv_bfloat16, 64>(a, kmap, vmap, num_ctas, overlap, stream);
 }
 
 }  // namespace pa

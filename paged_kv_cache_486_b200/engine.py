@@ -79,11 +79,11 @@ class PagedKVCache:
         return (torch.from_numpy(table).to(self.device), torch.from_numpy(ctx).to(self.device))
 
     def decode(self, q, block_tables, context_lens, scale, out=None, path=PA_PATH_AUTO,
-               num_workers=0, stream=None):
+               num_workers=0, flags=0, stream=None):
         if out is None:
             out = torch.empty_like(q)
         pa_decode_attention(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
-                            self.workspace, self.dev_error, path, num_workers, stream)
+                            self.workspace, self.dev_error, path, num_workers, flags, stream)
         return out
 
     def device_errors(self, stream=None):

@@ -45,7 +45,7 @@ def _decode_args(**kw):
     args = dict(out=C.c_void_p(16), q=C.c_void_p(16), k=C.c_void_p(16), v=C.c_void_p(16),
                 bt=C.c_void_p(16), ctx=C.c_void_p(16), B=4, Hq=8, Hkv=2, D=128, bs=16, NB=10,
                 MB=4, scale=0.1, dtype=pa.PA_F16, ws=C.c_void_p(16), ws_bytes=1 << 30, err=None,
-                path=0, workers=0, stream=None)
+                path=0, workers=0, flags=0, stream=None)
     args.update(kw)
     return args
 
@@ -54,7 +54,8 @@ def _call_decode(a):
     return pa.lib.pa_decode_attention_ex(a["out"], a["q"], a["k"], a["v"], a["bt"], a["ctx"],
                                          a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["NB"],
                                          a["MB"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"],
-                                         a["err"], a["path"], a["workers"], a["stream"])
+                                         a["err"], a["path"], a["workers"], a["flags"],
+                                         a["stream"])
 
 
 @pytest.mark.parametrize("bad", [
@@ -62,6 +63,7 @@ def _call_decode(a):
     dict(ws_bytes=16), dict(q=None), dict(k=C.c_void_p(8)), dict(path=9),
     dict(path=pa.PA_PATH_TC, dtype=pa.PA_F32), dict(path=pa.PA_PATH_TC, Hq=32, Hkv=2),
     dict(path=pa.PA_PATH_TC, bs=8), dict(NB=1 << 24, Hkv=16, Hq=16), dict(scale=float("nan")),
+    dict(flags=2), dict(B=4096, Hkv=128, Hq=128),
 ])
 def test_decode_rejects_bad_arguments_on_host(bad):
     st = _call_decode(_decode_args(**bad))

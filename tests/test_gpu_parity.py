@@ -212,3 +212,27 @@ def test_device_guards_report_instead_of_faulting():
     out = eng.decode(g["q"], g["bt"], g["ctx"], wl.scale)
     torch.cuda.synchronize()
     assert torch.equal(bits(out), bits(g["out"]))
+
+
+def test_overlapped_prologue_gives_the_same_bits():
+    wl = workloads.custom("ovl", "bf16", B=5, Hq=64, Hkv=8, D=128, bs=16,
+                          ctx=[3, 100, 700, 1600, 2500], seed=41)
+    g = build(wl)
+    eng = g["eng"]
+    k = wl.tokens(7, 0, wl.B, 0, "cuda")
+    v = wl.tokens(7, 0, wl.B, 1, "cuda")
+    # rewrite each sequence's last token, then decode right behind the cache write
+    last = []
+    for b in range(wl.B):
+        n = int(g["ctx"][b])
+        blk = int(g["bt"][b, (n - 1) // wl.bs])
+        last.append(blk * wl.bs + (n - 1) % wl.bs)
+    slots = torch.tensor(last, dtype=torch.int64, device="cuda")
+    outs = []
+    for flags in (0, pa.PA_DECODE_OVERLAP_PROLOGUE, pa.PA_DECODE_OVERLAP_PROLOGUE):
+        pa.pa_reshape_and_cache(k, v, eng.k_cache, eng.v_cache, slots, eng.dev_error)
+        outs.append(eng.decode(g["q"], g["bt"], g["ctx"], wl.scale, flags=flags))
+    torch.cuda.synchronize()
+    assert torch.equal(bits(outs[0]), bits(outs[1])) and torch.equal(bits(outs[1]), bits(outs[2]))
+    assert not torch.equal(bits(outs[0]), bits(g["out"]))  # the rewritten tokens were seen
+    assert eng.device_errors() == 0
