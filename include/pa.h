@@ -97,6 +97,17 @@ void pa_pool_destroy(pa_pool* pool);
 pa_status pa_alloc(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slot_mapping_out_host,
                    int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out);
 
+/* pa_alloc for a batch: grows each of n_seqs sequences (in order; a sequence may
+ * appear more than once) by n_new_each tokens, exactly as n_seqs calls of
+ * pa_alloc would, in one call.  slot_mapping_out_host[n_seqs * n_new_each] is
+ * sequence-major; copy pairs (at most one per sequence) go to
+ * cow_pairs_out_host[2 * max_cow], their count to *n_cow_out.  All or nothing:
+ * on PA_ERR_OOM, or PA_ERR_INVALID because more than max_cow pairs are needed,
+ * the pool is restored exactly to its state before the call. */
+pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_seqs,
+                         int32_t n_new_each, int64_t* slot_mapping_out_host,
+                         int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out);
+
 /* Drop seq_id: each of its blocks loses one holder, in logical order; a block
  * with no holder left goes on top of the free stack.  PA_ERR_NOT_FOUND if unknown. */
 pa_status pa_free(pa_pool* pool, int64_t seq_id);

@@ -124,8 +124,9 @@ class Pool:
         self.block_size = block_size
 
     def __del__(self):
-        if getattr(self, "h", None):
-            lib().orc_pool_delete(self.h)
+        h = getattr(self, "h", None)
+        if h and _lib is not None:  # the library may be gone at interpreter shutdown
+            _lib.orc_pool_delete(h)
             self.h = None
 
     def alloc(self, seq, n):

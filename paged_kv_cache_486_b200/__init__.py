@@ -34,6 +34,7 @@ SIGNATURES = {
     "pa_pool_create": (_I32, [_I32, _I32, C.POINTER(_P)]),
     "pa_pool_destroy": (None, [_P]),
     "pa_alloc": (_I32, [_P, _I64, _I32, _P, _P, _I32, _P]),
+    "pa_alloc_batch": (_I32, [_P, _P, _I32, _I32, _P, _P, _I32, _P]),
     "pa_free": (_I32, [_P, _I64]),
     "pa_fork": (_I32, [_P, _I64, _I64]),
     "pa_block_table": (_I32, [_P, _P, _I32, _I32, _P, _P]),
@@ -125,7 +126,7 @@ class Pool:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h:
+        if h and lib is not None:  # the library may be gone at interpreter shutdown
             lib.pa_pool_destroy(h)
             self._h = None
 
@@ -136,6 +137,18 @@ class Pool:
                           _np_ptr(self._ncow))
         _check(st, "pa_alloc")
         return slots[:n_new], self._pair.reshape(1, 2)[: int(self._ncow[0])].copy()
+
+    def pa_alloc_batch(self, seq_ids, n_new_each: int, slots_out=None):
+        """-> (slot_mapping int64[n * n_new_each], cow_pairs int32[k, 2]); all or nothing."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = len(ids)
+        slots = slots_out if slots_out is not None else np.empty(max(n * n_new_each, 1),
+                                                                 dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int32)
+        st = lib.pa_alloc_batch(self._h, _np_ptr(ids), n, n_new_each, _np_ptr(slots),
+                                _np_ptr(pairs), n, _np_ptr(self._ncow))
+        _check(st, "pa_alloc_batch")
+        return slots[:n * n_new_each], pairs[: int(self._ncow[0])].copy()
 
     def pa_free(self, seq_id: int):
         _check(lib.pa_free(self._h, seq_id), "pa_free")

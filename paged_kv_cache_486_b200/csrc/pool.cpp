@@ -102,6 +102,92 @@ pa_status pa_alloc(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slot_m
   return PA_OK;
 }
 
+// Batched growth: the same effect as n_seqs calls of pa_alloc in order, but one
+// call, and all or nothing -- on failure every sequence already grown in this
+// batch is restored exactly (blocks go back on the free stack in the order
+// they left it), so the pool is unchanged.
+pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_seqs,
+                         int32_t n_new_each, int64_t* slot_mapping_out_host,
+                         int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out) {
+  if (!pool || n_seqs < 0 || n_new_each < 0 || !n_cow_out || max_cow < 0 ||
+      (n_seqs > 0 && !seq_ids_host) ||
+      (n_seqs > 0 && n_new_each > 0 && !slot_mapping_out_host) || (max_cow > 0 && !cow_pairs_out_host))
+    return pa::fail(PA_ERR_INVALID, "pa_alloc_batch: bad arguments");
+  struct Undo {
+    int64_t seq;
+    bool created;
+    int64_t old_len;
+    int32_t cow_src, cow_dst;
+    int64_t fresh;
+  };
+  std::vector<Undo> log;
+  log.reserve(n_seqs);
+  int32_t n_cow = 0;
+  pa_status st = PA_OK;
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const int64_t id = seq_ids_host[i];
+    auto it = pool->seqs.find(id);
+    const bool known = it != pool->seqs.end();
+    const int64_t bs = pool->block_size;
+    const int64_t len = known ? it->second.len : 0;
+    const int64_t tail = len % bs;
+    const int64_t fill = tail ? std::min<int64_t>(bs - tail, n_new_each) : 0;
+    const bool copy = fill > 0 && pool->refs[it->second.blocks.back()] > 1;
+    const int64_t fresh = (n_new_each - fill + bs - 1) / bs;
+    if (copy && n_cow >= max_cow) {
+      st = pa::fail(PA_ERR_INVALID, "pa_alloc_batch: more than max_cow=%d copy pairs", max_cow);
+      break;
+    }
+    if ((copy ? 1 : 0) + fresh > static_cast<int64_t>(pool->free_stack.size())) {
+      st = pa::fail(PA_ERR_OOM, "pa_alloc_batch: sequence %d of %d needs %lld blocks, %zu free",
+                    i, n_seqs, static_cast<long long>((copy ? 1 : 0) + fresh),
+                    pool->free_stack.size());
+      break;
+    }
+    pa_pool::Seq& s = known ? it->second : pool->seqs[id];
+    Undo u{id, !known, len, -1, -1, fresh};
+    if (copy) {
+      u.cow_src = s.blocks.back();
+      u.cow_dst = pool->pop();
+      pool->unref(u.cow_src);
+      s.blocks.back() = u.cow_dst;
+      cow_pairs_out_host[2 * n_cow] = u.cow_src;
+      cow_pairs_out_host[2 * n_cow + 1] = u.cow_dst;
+      ++n_cow;
+    }
+    for (int64_t k = 0; k < fresh; ++k) s.blocks.push_back(pool->pop());
+    int64_t* slots = slot_mapping_out_host + static_cast<int64_t>(i) * n_new_each;
+    for (int64_t k = 0; k < n_new_each; ++k) {
+      const int64_t pos = len + k;
+      slots[k] = static_cast<int64_t>(s.blocks[pos / bs]) * bs + pos % bs;
+    }
+    s.len = len + n_new_each;
+    log.push_back(u);
+  }
+  if (st != PA_OK) {
+    for (auto r = log.rbegin(); r != log.rend(); ++r) {
+      pa_pool::Seq& s = pool->seqs[r->seq];
+      for (int64_t k = 0; k < r->fresh; ++k) {
+        const int32_t b = s.blocks.back();
+        s.blocks.pop_back();
+        pool->refs[b] = 0;
+        pool->free_stack.push_back(b);
+      }
+      if (r->cow_dst >= 0) {
+        s.blocks.back() = r->cow_src;
+        pool->refs[r->cow_src] += 1;
+        pool->refs[r->cow_dst] = 0;
+        pool->free_stack.push_back(r->cow_dst);
+      }
+      s.len = r->old_len;
+      if (r->created) pool->seqs.erase(r->seq);
+    }
+    return st;
+  }
+  *n_cow_out = n_cow;
+  return PA_OK;
+}
+
 pa_status pa_free(pa_pool* pool, int64_t seq_id) {
   if (!pool) return pa::fail(PA_ERR_INVALID, "pa_free: NULL pool");
   auto it = pool->seqs.find(seq_id);

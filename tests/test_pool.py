@@ -130,3 +130,46 @@ def test_pool_slots_are_valid_for_the_kernels():
             p.pa_free(op[1])
     t, c = p.pa_block_table(wl.batch, wl.max_blocks)
     assert pa.pa_validate_block_table(t, c, wl.bs, wl.num_blocks) == pa.PA_OK
+
+
+def test_batched_alloc_equals_sequential_and_rolls_back():
+    rng = np.random.default_rng(5)
+    for trial in range(40):
+        nb, bs = int(rng.integers(4, 60)), int(rng.choice([1, 4, 16]))
+        a, b = pa.Pool(nb, bs), pa.Pool(nb, bs)
+        live = []
+        for _ in range(30):
+            r = rng.random()
+            if r < 0.2 and live:
+                p, c = int(rng.choice(live)), int(rng.integers(100, 200))
+                if c not in live:
+                    a.pa_fork(p, c)
+                    b.pa_fork(p, c)
+                    live.append(c)
+                continue
+            ids = [int(x) for x in rng.integers(0, 8, size=int(rng.integers(1, 6)))]
+            n = int(rng.integers(0, 2 * bs + 1))
+            before = ([a.pa_refcount(i) for i in range(nb)], a.pa_num_free_blocks(),
+                      {s: a.pa_seq_len(s) for s in range(8)})
+            try:
+                slots, cow = a.pa_alloc_batch(ids, n)
+            except pa.PagedAttnError as e:
+                assert e.status == pa.PA_ERR_OOM
+                after = ([a.pa_refcount(i) for i in range(nb)], a.pa_num_free_blocks(),
+                         {s: a.pa_seq_len(s) for s in range(8)})
+                assert before == after  # all or nothing
+                # and the free stack order is intact: the next allocations agree
+                continue
+            exp_slots, exp_cow = [], []
+            for s in ids:
+                sl, cw = b.pa_alloc(s, n)
+                exp_slots.append(sl)
+                exp_cow.extend(cw.tolist())
+            assert np.array_equal(slots, np.concatenate(exp_slots) if exp_slots else slots)
+            assert cow.tolist() == exp_cow
+            live = sorted(set(live) | set(ids))
+            assert a.pa_num_free_blocks() == b.pa_num_free_blocks()
+            assert [a.pa_refcount(i) for i in range(nb)] == [b.pa_refcount(i) for i in range(nb)]
+            t1, c1 = a.pa_block_table(live, nb + 1)
+            t2, c2 = b.pa_block_table(live, nb + 1)
+            assert np.array_equal(t1, t2) and np.array_equal(c1, c2)
