@@ -185,12 +185,16 @@ pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
  * head_dim in {64, 128}; block_size in {8, 16, 32, 64, 128}; batch <= 4096;
  * batch * num_kv_heads <= 262144; num_blocks * num_kv_heads * block_size < 2^31.
  * workspace: device scratch of at least pa_decode_workspace_size(...) bytes,
- *   16-byte aligned, contents need no initialisation; calls that share a
- *   workspace must be ordered on one stream.
- * The work is split evenly across the GPU by KV blocks: a sequence that fits in
- * one worker's share is done in a single pass; a longer one is cut into pieces
- * whose (max, sum, partial output) are merged with a log-sum-exp combine by the
- * worker that finishes the last piece.  One kernel launch per call.
+ *   16-byte aligned, zero-filled once before its first use (e.g. cudaMemset);
+ *   every call that completes leaves it zero-filled again, so it is reused
+ *   without clearing.  After a call that reported PA_DEVERR_TIMEOUT, zero it
+ *   again.  Calls that share a workspace must be ordered on one stream.
+ * The work is split across the GPU by KV blocks: 7/8 of them evenly over the
+ * workers, the rest in chunks claimed by whichever workers finish first.  A
+ * sequence that fits in one worker's share is done in a single pass; a longer
+ * one is cut into pieces whose (max, sum, partial output) are merged with a
+ * log-sum-exp combine by the worker that finishes the last piece.  One kernel
+ * launch per call.
  * ---------------------------------------------------------------------- */
 size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                 int32_t head_dim);
@@ -234,14 +238,14 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
  * no counterpart to this call; it exists for callers that cannot allocate
  * device memory (an embedding host that hands out none, a serving loop that
  * must not call cudaMalloc while requests run, a process whose memory another
- * runtime has reserved).  The scratch is one area of 20 MiB that the library
+ * runtime has reserved).  The scratch is one area of 28 MiB that the library
  * declares in device memory; every GPU that loads the library holds it until
  * the process exits.  Arguments, results and errors are those of
  * pa_decode_attention, plus PA_ERR_INVALID if a shape would need more scratch
  * than the area holds.  Nothing is allocated by this call.
- * The first call on a device looks up the area's device address (once per
- * device, with that device current); make that first call before any stream
- * capture begins.  All calls share the one area, which keeps whatever the last
+ * The first call on a device looks up the area's device address and zero-fills
+ * the area, waiting for the device to finish (once per device, with that device
+ * current); make that first call before any stream capture begins.  All calls share the one area, which keeps whatever the last
  * call left in it: calls whose work overlaps on the GPU (different streams,
  * or different host threads on one device) race on it and must be ordered by
  * the caller. */

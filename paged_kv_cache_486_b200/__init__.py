@@ -227,7 +227,8 @@ def pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, dtype
 def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, scale, workspace,
                         dev_error=None, path=PA_PATH_AUTO, num_workers=0, flags=0, stream=None):
     """q/out [B, Hq, D]; caches [NB, Hkv, bs, D]; block_tables int32 [B, MB];
-    context_lens int32 [B]; workspace uint8 [>= pa_decode_workspace_size] (all CUDA)."""
+    context_lens int32 [B]; workspace uint8 [>= pa_decode_workspace_size], zero-filled
+    before its first use (all CUDA)."""
     B, Hq, D = q.shape
     NB, Hkv, bs, _ = k_cache.shape
     MB = block_tables.shape[1]
@@ -246,7 +247,7 @@ def pa_decode_attention(out, q, k_cache, v_cache, block_tables, context_lens, sc
 def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                                   dev_error=None, stream=None):
     """pa_decode_attention for callers that cannot allocate device memory: the
-    library's own fixed 20 MiB device scratch replaces the workspace.  Calls that
+    library's own fixed 28 MiB device scratch replaces the workspace.  Calls that
     overlap on the GPU share that scratch and race; order them on one stream."""
     B, Hq, D = q.shape
     NB, Hkv, bs, _ = k_cache.shape

@@ -4,7 +4,6 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -115,19 +114,12 @@ bool tc_applies(int group, int head_dim, int block_size, pa_dtype dt) {
          block_size % 16 == 0;
 }
 
-// Workspace: [256 reserved][arrival words: B * Hkv x 8 bytes][pieces].
+// Workspace: [256-byte header: chunk counter, finished-worker counter]
+//            [arrival counts: B * Hkv x 4 bytes][piece slots].
 size_t pieces_offset(int batch, int num_kv_heads) {
-  const size_t arrivals = (sizeof(unsigned long long) * static_cast<size_t>(batch) * num_kv_heads +
-                           255) & ~size_t(255);
+  const size_t arrivals =
+      (sizeof(uint32_t) * static_cast<size_t>(batch) * num_kv_heads + 255) & ~size_t(255);
   return 256 + arrivals;
-}
-
-// Nonzero tag per decode call for the arrival words.
-uint32_t next_epoch() {
-  static std::atomic<uint32_t> epoch{0};
-  uint32_t e = ++epoch;
-  while (e == 0) e = ++epoch;
-  return e;
 }
 
 }  // namespace
@@ -194,7 +186,8 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_
     return 0;
   const int group = num_q_heads / num_kv_heads;
   return pieces_offset(batch, num_kv_heads) +
-         sizeof(float) * 2 * static_cast<size_t>(max_workers(group)) * group * (head_dim + 2);
+         sizeof(float) * 2 * static_cast<size_t>(pa::max_ranges(max_workers(group))) * group *
+             (head_dim + 2);
 }
 
 pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
@@ -290,8 +283,8 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.dev_error = dev_error;
-  a.ws_arrivals =
-      reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + 256);
+  a.ws_ctrl = static_cast<uint32_t*>(workspace);
+  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + 256);
   a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                          pieces_offset(batch, num_kv_heads));
   a.batch = batch;
@@ -303,7 +296,6 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.num_blocks = num_blocks;
   a.max_blocks = max_blocks;
   a.workers = workers;
-  a.epoch = next_epoch();
   a.scale_log2 = scale * 1.4426950408889634f;
 
   cudaError_t e;
@@ -365,14 +357,14 @@ pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_strea
 // scratch area of its own in device memory, declared below, and
 // pa_decode_attention_static_ws uses it instead of a caller buffer.
 //
-// The area is kStaticScratchBytes (20 MiB): enough for the largest workspace
-// any shape pa_decode_attention accepts can ask for (2048 workers x 8 heads x
-// (128 + 2) floats x 2 pieces, plus one 8-byte arrival word for each of at most
-// 262144 (sequence, kv head) pairs).  Every GPU that loads this library holds
-// those 20 MiB until the process exits.
+// The area is kStaticScratchBytes (28 MiB): enough for the largest workspace
+// any shape pa_decode_attention accepts can ask for (3073 ranges x 2 piece
+// slots x 8 heads x (128 + 2) floats, plus a 4-byte arrival count for each of
+// at most 262144 (sequence, kv head) pairs).  Every GPU that loads this
+// library holds those 28 MiB until the process exits.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr size_t kStaticScratchBytes = size_t(20) << 20;
+constexpr size_t kStaticScratchBytes = size_t(28) << 20;
 }
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
@@ -384,7 +376,10 @@ void* g_scratch_addr[64] = {};
 
 // Device address of g_decode_scratch on the current device.  In host code the
 // symbol name is only a host-side handle, so the address is looked up once per
-// device (with that device current) and remembered.
+// device (with that device current) and remembered.  The same one-time set-up
+// zero-fills the area (the decode keeps a few counters in its workspace that
+// must start at zero; every completed call leaves them at zero again) and waits
+// for that to finish.
 pa_status static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -397,6 +392,9 @@ pa_status static_scratch(void** out) {
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess)
       return cuda_fail(e, "pa_decode_attention_static_ws (cudaGetSymbolAddress)");
+    e = cudaMemset(p, 0, kStaticScratchBytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention_static_ws (zero-fill)");
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -420,10 +418,8 @@ extern "C" pa_status pa_decode_attention_static_ws(
   void* scratch = nullptr;
   const pa_status st = static_scratch(&scratch);
   if (st != PA_OK) return st;
-  // Nothing in the scratch needs to start at zero: the split pieces are written
-  // before they are read, and each arrival word is tagged with its call's epoch
-  // (a word from an earlier call reads as zero) and cleared by the call that
-  // completes it.
+  // The counters in the scratch were zeroed at set-up and every completed call
+  // returns them to zero; the split pieces are written before they are read.
   return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, scratch, kStaticScratchBytes,

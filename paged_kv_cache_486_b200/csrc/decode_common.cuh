@@ -3,21 +3,30 @@
 // The unit of work is one KV block of one (sequence b, kv head) pair.  Units
 // are numbered b-major, then kv head, then logical block j:
 //     u = Hkv * cum[b] + kvh * nblk[b] + j,   cum[b] = sum_{b' < b} nblk[b'],
-// nblk[b] = ceil(ctx[b] / block_size).  Worker w (one warp) takes the units
-// [start(w), start(w + 1)) with start(w) = floor(U * w / W), so every worker
-// gets the same number of KV bytes to within one block.  A run of units of
-// one (b, kv head) inside one worker is a "segment".  A segment that holds a
-// whole (b, kv head) writes the output directly (single pass); otherwise it is
-// a piece of a longer context: the worker stores the piece's (max, sum,
-// unnormalised output) and the worker whose piece arrives last merges all of
-// them with a log-sum-exp combine (piece_done below).  Only a
-// worker's first and last segments can be pieces, so each worker owns two
-// piece slots: slot 0 for the segment that contains start(w), slot 1 for its
-// last segment.
+// nblk[b] = ceil(ctx[b] / block_size).  The units are cut into ranges:
+//  * static ranges: the first Us units are split evenly over the W workers
+//    (one warp each): range w = [floor(Us w / W), floor(Us (w + 1) / W));
+//  * tail chunks: the last U - Us units (1/8 of them when there are at least
+//    16 per worker) are cut into NC chunks of CH units that workers claim one
+//    at a time, from a counter, when they run out of work.  An even split by
+//    bytes is not an even split by time (memory latency differs from warp to
+//    warp); the claimed tail evens out the finishing times.
+// A run of units of one (b, kv head) inside one range is a "segment".  A
+// segment that holds a whole (b, kv head) writes the output directly (single
+// pass); otherwise it is a piece of a longer context: the worker stores the
+// piece's (max, sum, unnormalised output) and the worker whose piece arrives
+// last merges all of them with a log-sum-exp combine (piece_done below).  Only
+// a range's first and last segments can be pieces, so each range owns two
+// piece slots: slot 0 for the segment that contains the range's first unit,
+// slot 1 for its last segment.
 //
 // Piece layout (fp32): m[G], l[G], o[G][D] where, for the piece's tokens j,
 //   m = max_j t_j, l = sum_j 2^(t_j - m), o = sum_j 2^(t_j - m) v_j,
 //   t_j = (q . k_j) * scale * log2(e)   (scores in base-2 units).
+//
+// Workspace words that must start at zero (the chunk counter, the finished-
+// worker counter and one arrival count per (b, kv head)) are returned to zero
+// by every call that completes, so a workspace zero-filled once stays usable.
 #pragma once
 #include <cstdint>
 
@@ -41,22 +50,48 @@ struct DecodeArgs {
   const int32_t* block_tables;
   const int32_t* context_lens;
   int32_t* dev_error;
-  unsigned long long* ws_arrivals;  // [B * Hkv] piece arrival words (epoch << 32 | count)
-  float* ws_pieces;     // [2 * max_workers][G * (D + 2)]
+  uint32_t* ws_ctrl;      // [0] next tail chunk, [1] workers finished
+  uint32_t* ws_arrivals;  // [B * Hkv] pieces arrived
+  float* ws_pieces;       // [2 * max_ranges][G * (D + 2)]
   int32_t batch, num_q_heads, num_kv_heads, group, head_dim, block_size;
   int32_t num_blocks, max_blocks;
-  int32_t workers;      // workers launched (the split uses min(workers, U))
-  uint32_t epoch;       // nonzero tag of this call for the arrival words
-  float scale_log2;     // scale * log2(e)
+  int32_t workers;        // workers launched (the split uses at most this many)
+  float scale_log2;       // scale * log2(e)
 };
 
-__host__ __device__ inline int64_t split_start(int64_t w, int64_t U, int64_t W) {
-  return (U * w) / W;
-}
+// Ranges of the unit sequence (see the header comment).  Every range is non-empty.
+struct Split {
+  int64_t U, Us, W, CH, NC;
+  __host__ __device__ int64_t start(int64_t r) const {
+    return r < W ? (Us * r) / W : Us + (r - W) * CH;
+  }
+  __host__ __device__ int64_t end(int64_t r) const {
+    const int64_t e = r + 1 < W ? (Us * (r + 1)) / W : Us + (r + 1 - W) * CH;
+    return e < U ? e : U;
+  }
+  __host__ __device__ int64_t range_of(int64_t u) const {
+    return u < Us ? ((u + 1) * W - 1) / Us : W + (u - Us) / CH;
+  }
+};
 
-// The worker whose range holds unit u (requires W <= U so no range is empty).
-__host__ __device__ inline int64_t split_worker_of(int64_t u, int64_t U, int64_t W) {
-  return ((u + 1) * W - 1) / U;
+// Maximum number of ranges for `workers` workers (piece slots are 2 per range).
+__host__ __device__ inline int64_t max_ranges(int64_t workers) { return workers + workers / 2 + 1; }
+
+__host__ __device__ inline Split make_split(int64_t U, int64_t workers) {
+  Split s;
+  s.U = U;
+  const int64_t T = U >= 16 * workers ? U / 8 : 0;
+  s.Us = U - T;
+  s.W = workers < s.Us ? workers : s.Us;
+  if (T > 0) {
+    const int64_t cap = s.W / 2 > 1 ? s.W / 2 : 1;
+    s.CH = (T + cap - 1) / cap;
+    s.NC = (T + s.CH - 1) / s.CH;
+  } else {
+    s.CH = 1;
+    s.NC = 0;
+  }
+  return s;
 }
 
 // Waits for the grid this launch depends on (a no-op unless the decode was
@@ -175,24 +210,28 @@ __device__ inline void cursor_next(UnitCursor& c, const int32_t* cum, int Hkv) {
 }
 
 // ------------------------- merging split contexts --------------------------
-// A worker that has written a piece of (b, kv head) announces it on the pair's
+// A worker that has written a piece of (b, kv head) counts it on the pair's
 // arrival word; the warp whose piece completes the set merges all pieces:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,
-// then clears the word.  Words carry the call's epoch in their high half, so a
-// word left by an earlier call counts as zero.
-__device__ inline uint32_t arrive_piece(unsigned long long* word, uint32_t epoch,
-                                        int32_t* dev_error) {
-  unsigned long long old = atomicAdd(word, 0ull);
-  for (int i = 0; i < (1 << 20); ++i) {
-    const uint32_t e = static_cast<uint32_t>(old >> 32);
-    const uint32_t n = (e == epoch) ? static_cast<uint32_t>(old) : 0u;
-    const unsigned long long want = (static_cast<unsigned long long>(epoch) << 32) | (n + 1u);
-    const unsigned long long seen = atomicCAS(word, old, want);
-    if (seen == old) return n + 1u;
-    old = seen;
+// then returns the word to zero for the next call.
+
+// Claims the next tail chunk (whole warp; lane 0 touches the counter).
+__device__ inline int64_t claim_chunk(const DecodeArgs& a, int lane) {
+  uint32_t c = 0;
+  if (lane == 0) c = atomicAdd(&a.ws_ctrl[0], 1u);
+  return __shfl_sync(0xffffffffu, c, 0);
+}
+
+// Whole warp, once it has claimed its last chunk: the last of the W workers
+// to finish returns both counters to zero.
+__device__ inline void worker_finished(const DecodeArgs& a, int64_t W, int lane) {
+  if (lane == 0) {
+    const uint32_t n = atomicAdd(&a.ws_ctrl[1], 1u) + 1u;
+    if (n == static_cast<uint32_t>(W)) {
+      a.ws_ctrl[0] = 0u;
+      a.ws_ctrl[1] = 0u;
+    }
   }
-  report(dev_error, PA_DEVERR_TIMEOUT);
-  return 0u;
 }
 
 __device__ inline float warp_max(float x) {
@@ -216,27 +255,27 @@ template <typename T> struct Num;
 // at a time, each round issuing all of their loads for the lane at once.
 template <typename T, int D>
 __device__ inline void piece_done(const DecodeArgs& a, const int32_t* cum, int b, int kvh,
-                                  int64_t U, int64_t W, int lane) {
+                                  const Split& sp, int lane) {
   constexpr int PER = D / 32;
   constexpr int HG = 16 / PER;  // heads merged per pass (16 accumulators per lane)
   constexpr int PQ = 2;         // pieces loaded per round in pass 2
   const int Hkv = a.num_kv_heads, G = a.group;
   const int nblk = cum[b + 1] - cum[b];
   const int64_t u0 = static_cast<int64_t>(Hkv) * cum[b] + static_cast<int64_t>(kvh) * nblk;
-  const int64_t wf = split_worker_of(u0, U, W);
-  const int64_t wl = split_worker_of(u0 + nblk - 1, U, W);
+  const int64_t rf = sp.range_of(u0);
+  const int64_t rl = sp.range_of(u0 + nblk - 1);
   __syncwarp();
-  __threadfence();  // this warp's piece is visible before it is announced
+  __threadfence();  // this warp's piece is visible before it is counted
   __syncwarp();
   uint32_t n = 0;
-  if (lane == 0) n = arrive_piece(&a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh], a.epoch,
-                                  a.dev_error);
+  if (lane == 0) n = atomicAdd(&a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh], 1u) + 1u;
   n = __shfl_sync(0xffffffffu, n, 0);
-  const int np = static_cast<int>(wl - wf + 1);
+  const int np = static_cast<int>(rl - rf + 1);
   if (n != static_cast<uint32_t>(np)) return;
   __threadfence();  // every other piece is visible to this warp
-  // only the first piece can sit in slot 1 (its worker started before u0)
-  const int first_slot = split_start(wf, U, W) >= u0 ? 0 : 1;
+  // only the first piece can sit in slot 1 (its range started before u0)
+  const int first_slot = sp.start(rf) >= u0 ? 0 : 1;
+  const int64_t wf = rf;
   const int pf = G * (D + 2);
   const float* base = a.ws_pieces + (wf * 2 + first_slot) * pf;  // piece 0
   const float* rest = a.ws_pieces + (wf + 1) * 2 * pf;            // piece p >= 1: rest + 2 pf (p - 1)
@@ -306,7 +345,7 @@ __device__ inline void piece_done(const DecodeArgs& a, const int32_t* cum, int b
       }
     }
   }
-  if (lane == 0) a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh] = 0ull;
+  if (lane == 0) a.ws_arrivals[static_cast<int64_t>(b) * Hkv + kvh] = 0u;
 }
 
 // ------------------------------- dtypes ------------------------------------

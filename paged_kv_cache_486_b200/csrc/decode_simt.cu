@@ -27,13 +27,10 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
   zero_empty_rows<T>(a, ctx_s);
 
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
-  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
-  if (U == 0) return;
-  const int64_t W = U < a.workers ? U : a.workers;
+  const Split sp = make_split(static_cast<int64_t>(Hkv) * cum[B], a.workers);
   const int lane = threadIdx.x & 31;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kSimtWarps + (threadIdx.x >> 5);
-  if (w >= W) return;
-  const int64_t u0 = split_start(w, U, W), u1 = split_start(w + 1, U, W);
+  if (w >= sp.W) return;
 
   constexpr int PER = D / 32;
   const T* q = static_cast<const T*>(a.q);
@@ -43,105 +40,114 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
   const int bs = a.block_size;
   const int piece_floats = G * (D + 2);
 
-  UnitCursor c;
-  cursor_seek(c, u0, u1, cum, B, Hkv);
-  bool first_seg = true;
-  while (c.u < c.u_end) {
-    const int b = c.b, kvh = c.kvh, j0 = c.j;
-    const int64_t left = c.u_end - c.u;
-    const int seg = static_cast<int>(left < c.nblk - c.j ? left : c.nblk - c.j);
-    const int j1 = j0 + seg;
-    const bool complete = j0 == 0 && j1 == c.nblk;
-    const int slot = first_seg ? 0 : 1;
-    const int ctx = ctx_s[b];
-    for (int hg = 0; hg < G; hg += 8) {
-      const int nh = G - hg < 8 ? G - hg : 8;
-      float qv[8][PER], o[8][PER], m[8], l[8];
+  // the worker's static range first, then tail chunks while any are left
+  for (int64_t r = w;;) {
+    UnitCursor c;
+    cursor_seek(c, sp.start(r), sp.end(r), cum, B, Hkv);
+    bool first_seg = true;
+    while (c.u < c.u_end) {
+      const int b = c.b, kvh = c.kvh, j0 = c.j;
+      const int64_t left = c.u_end - c.u;
+      const int seg = static_cast<int>(left < c.nblk - c.j ? left : c.nblk - c.j);
+      const int j1 = j0 + seg;
+      const bool complete = j0 == 0 && j1 == c.nblk;
+      const int slot = first_seg ? 0 : 1;
+      const int ctx = ctx_s[b];
+      for (int hg = 0; hg < G; hg += 8) {
+        const int nh = G - hg < 8 ? G - hg : 8;
+        float qv[8][PER], o[8][PER], m[8], l[8];
 #pragma unroll
-      for (int hh = 0; hh < 8; ++hh) {
-        m[hh] = -INFINITY;
-        l[hh] = 0.f;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-          o[hh][i] = 0.f;
-          qv[hh][i] = hh < nh ? Num<T>::to_f(q[(static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) *
-                                                    D + lane + 32 * i])
-                              : 0.f;
-        }
-      }
-      for (int j = j0; j < j1; ++j) {
-        const int32_t phys = a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j];
-        if (phys < 0 || phys >= a.num_blocks) {
-          if (lane == 0) report(a.dev_error, PA_DEVERR_BAD_BLOCK);
-          continue;
-        }
-        const int rem = ctx - j * bs;
-        const int ntok = rem < bs ? rem : bs;
-        const int64_t tile = ((static_cast<int64_t>(phys) * Hkv + kvh) * bs) * D;
-        for (int t = 0; t < ntok; ++t) {
-          float kr[PER], vr[PER];
+        for (int hh = 0; hh < 8; ++hh) {
+          m[hh] = -INFINITY;
+          l[hh] = 0.f;
 #pragma unroll
           for (int i = 0; i < PER; ++i) {
-            kr[i] = Num<T>::to_f(kc[tile + t * D + lane + 32 * i]);
-            vr[i] = Num<T>::to_f(vc[tile + t * D + lane + 32 * i]);
-          }
-          float s[8];
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh) {
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) acc = fmaf(qv[hh][i], kr[i], acc);
-            s[hh] = acc;
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-#pragma unroll
-            for (int hh = 0; hh < 8; ++hh) s[hh] += __shfl_xor_sync(0xffffffffu, s[hh], off);
-          }
-#pragma unroll
-          for (int hh = 0; hh < 8; ++hh) {
-            const float t2 = s[hh] * a.scale_log2;
-            const float mn = fmaxf(m[hh], t2);
-            const float alpha = exp2f(m[hh] - mn);
-            const float p = exp2f(t2 - mn);
-            l[hh] = l[hh] * alpha + p;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) o[hh][i] = fmaf(o[hh][i], alpha, p * vr[i]);
-            m[hh] = mn;
+            o[hh][i] = 0.f;
+            qv[hh][i] = hh < nh ? Num<T>::to_f(q[(static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) *
+                                                      D + lane + 32 * i])
+                                : 0.f;
           }
         }
-      }
-      if (complete) {
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          if (hh < nh) {
-            const float inv = 1.f / l[hh];
-            T* orow = out + (static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) * D;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = Num<T>::from_f(o[hh][i] * inv);
+        for (int j = j0; j < j1; ++j) {
+          const int32_t phys = a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j];
+          if (phys < 0 || phys >= a.num_blocks) {
+            if (lane == 0) report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+            continue;
           }
-        }
-      } else {
-        float* piece = a.ws_pieces + (w * 2 + slot) * piece_floats;
+          const int rem = ctx - j * bs;
+          const int ntok = rem < bs ? rem : bs;
+          const int64_t tile = ((static_cast<int64_t>(phys) * Hkv + kvh) * bs) * D;
+          for (int t = 0; t < ntok; ++t) {
+            float kr[PER], vr[PER];
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh) {
-          if (hh < nh) {
-            if (lane == 0) {
-              piece[hg + hh] = m[hh];
-              piece[G + hg + hh] = l[hh];
+            for (int i = 0; i < PER; ++i) {
+              kr[i] = Num<T>::to_f(kc[tile + t * D + lane + 32 * i]);
+              vr[i] = Num<T>::to_f(vc[tile + t * D + lane + 32 * i]);
+            }
+            float s[8];
+#pragma unroll
+            for (int hh = 0; hh < 8; ++hh) {
+              float acc = 0.f;
+#pragma unroll
+              for (int i = 0; i < PER; ++i) acc = fmaf(qv[hh][i], kr[i], acc);
+              s[hh] = acc;
             }
 #pragma unroll
-            for (int i = 0; i < PER; ++i) piece[2 * G + (hg + hh) * D + lane + 32 * i] = o[hh][i];
+            for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+              for (int hh = 0; hh < 8; ++hh) s[hh] += __shfl_xor_sync(0xffffffffu, s[hh], off);
+            }
+#pragma unroll
+            for (int hh = 0; hh < 8; ++hh) {
+              const float t2 = s[hh] * a.scale_log2;
+              const float mn = fmaxf(m[hh], t2);
+              const float alpha = exp2f(m[hh] - mn);
+              const float p = exp2f(t2 - mn);
+              l[hh] = l[hh] * alpha + p;
+#pragma unroll
+              for (int i = 0; i < PER; ++i) o[hh][i] = fmaf(o[hh][i], alpha, p * vr[i]);
+              m[hh] = mn;
+            }
+          }
+        }
+        if (complete) {
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh) {
+            if (hh < nh) {
+              const float inv = 1.f / l[hh];
+              T* orow = out + (static_cast<int64_t>(b) * Hq + kvh * G + hg + hh) * D;
+#pragma unroll
+              for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = Num<T>::from_f(o[hh][i] * inv);
+            }
+          }
+        } else {
+          float* piece = a.ws_pieces + (r * 2 + slot) * piece_floats;
+#pragma unroll
+          for (int hh = 0; hh < 8; ++hh) {
+            if (hh < nh) {
+              if (lane == 0) {
+                piece[hg + hh] = m[hh];
+                piece[G + hg + hh] = l[hh];
+              }
+#pragma unroll
+              for (int i = 0; i < PER; ++i)
+                piece[2 * G + (hg + hh) * D + lane + 32 * i] = o[hh][i];
+            }
           }
         }
       }
+      if (!complete) piece_done<T, D>(a, cum, b, kvh, sp, lane);
+      first_seg = false;
+      c.u += seg - 1;
+      c.j = j1 - 1;
+      cursor_next(c, cum, Hkv);
     }
-    if (!complete) piece_done<T, D>(a, cum, b, kvh, U, W, lane);
-    first_seg = false;
-    c.u += seg - 1;
-    c.j = j1 - 1;
-    cursor_next(c, cum, Hkv);
+    if (sp.NC == 0) break;
+    const int64_t chunk = claim_chunk(a, lane);
+    if (chunk >= sp.NC) break;
+    r = sp.W + chunk;
   }
+  worker_finished(a, sp.W, lane);
 }
 
 template <typename T, int D>

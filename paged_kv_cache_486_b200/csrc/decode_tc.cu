@@ -209,6 +209,21 @@ __device__ __forceinline__ int stages_in_block(int ctx, int j, int bs) {
   return (n + kTok - 1) / kTok;
 }
 
+// What the producer lane tells the consumer about a stage it issued.
+constexpr int kHasData = 1;       // the tile was loaded (its block id was in range)
+constexpr int kSegStart = 2;      // first stage of a segment
+constexpr int kSegEnd = 4;        // last stage of a segment
+constexpr int kComplete = 8;      // the segment is a whole (sequence, kv head)
+constexpr int kFirstInRange = 16; // the segment holds its range's first unit (piece slot 0)
+constexpr int kMoreInRange = 32;  // the range continues after this (sequence, kv head)
+
+struct StageMeta {
+  int32_t b;
+  int32_t kvh_flags;  // kv head << 16 | flags
+  int32_t tok0;       // first token of the stage in the sequence
+  int32_t range;      // range the stage belongs to (piece slots)
+};
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -220,8 +235,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   const uint32_t ring0 = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (ring0 - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + G_::kRingBytes);
-  int32_t* slot_ok = reinterpret_cast<int32_t*>(bars + kWarps * kStages);
-  int32_t* cum = slot_ok + kWarps * kStages;
+  StageMeta* meta = reinterpret_cast<StageMeta*>(bars + kWarps * kStages);
+  int32_t* cum = reinterpret_cast<int32_t*>(meta + kWarps * kStages);
   int32_t* ctx_s = cum + a.batch + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -238,66 +253,93 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   // while the preceding kernel (typically the cache write) is still finishing.
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
   const int bs = a.block_size;
-  const int64_t U = static_cast<int64_t>(Hkv) * cum[B];
-  const int64_t W = U < a.workers ? U : a.workers;
+  const Split sp = make_split(static_cast<int64_t>(Hkv) * cum[B], a.workers);
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const bool active = w < W;  // false for every warp when U == 0
-  const int64_t u0 = active ? split_start(w, U, W) : 0;
-  const int64_t u1 = active ? split_start(w + 1, U, W) : 0;
+  const bool active = w < sp.W;  // false for every warp when there is no work
 
   const uint32_t ring = ring0 + warp * kStages * G_::kStageBytes;
   const uint32_t bar0 = smem_u32(&bars[warp * kStages]);
-  int32_t* ok = slot_ok + warp * kStages;
+  StageMeta* wmeta = meta + warp * kStages;
 
   // ---------------- producer state (uniform across the warp) ----------------
+  int64_t prange = w;
+  int64_t pend = active ? sp.end(w) : 0;
   UnitCursor pc;
-  cursor_seek(pc, u0, u1, cum, B, Hkv);
+  cursor_seek(pc, active ? sp.start(w) : 0, pend, cum, B, Hkv);
   int psub = 0;
   int pnsub = active ? stages_in_block(ctx_s[pc.b], pc.j, bs) : 0;
-  int64_t win = u0;
-  int32_t ids_cur = unit_block_id(a, cum, u0 + lane, u1);
-  int32_t ids_next = unit_block_id(a, cum, u0 + 32 + lane, u1);
+  bool pdone = !active, pnew_seg = true, pfirst = true;
+  int pseg_j0 = 0;
+  int64_t win = active ? sp.start(w) : 0;
+  int32_t ids_cur = unit_block_id(a, cum, win + lane, pend);
+  int32_t ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
 
-  auto produce = [&](int slot) {
+  // Issues the next stage into `slot` (claiming a tail chunk when the current
+  // range is used up); false when there is nothing left to issue.
+  auto produce = [&](int slot) -> bool {
+    if (pdone) return false;
+    if (pc.u >= pend) {
+      const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
+      if (chunk >= sp.NC) {
+        pdone = true;
+        return false;
+      }
+      prange = sp.W + chunk;
+      win = sp.start(prange);
+      pend = sp.end(prange);
+      cursor_seek(pc, win, pend, cum, B, Hkv);
+      psub = 0;
+      pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+      pnew_seg = pfirst = true;
+      ids_cur = unit_block_id(a, cum, win + lane, pend);
+      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
+    }
     if (pc.u >= win + 32) {
       win += 32;
       ids_cur = ids_next;
-      ids_next = unit_block_id(a, cum, win + 32 + lane, u1);
+      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
     }
     const int32_t id = __shfl_sync(kFull, ids_cur, static_cast<int>(pc.u - win));
+    if (pnew_seg) pseg_j0 = pc.j;
+    const int64_t pair_end = pc.u - pc.j + pc.nblk;  // one past the pair's last unit
+    const bool last_sub = psub + 1 == pnsub;
+    const bool seg_end = last_sub && (pc.u + 1 == pend || pc.j + 1 == pc.nblk);
+    const bool ok = id >= 0 && id < a.num_blocks;
+    const int flags = (ok ? kHasData : 0) | (pnew_seg ? kSegStart : 0) | (seg_end ? kSegEnd : 0) |
+                      (pseg_j0 == 0 && pair_end <= pend ? kComplete : 0) |
+                      (pfirst ? kFirstInRange : 0) | (pair_end < pend ? kMoreInRange : 0);
     if (lane == 0) {
+      wmeta[slot] = StageMeta{pc.b, (pc.kvh << 16) | flags, pc.j * bs + psub * kTok,
+                              static_cast<int32_t>(prange)};
       const uint32_t bar = bar0 + slot * 8;
-      if (id >= 0 && id < a.num_blocks) {
-        ok[slot] = 1;
+      if (ok) {
         mbar_arrive_expect_tx(bar, G_::kStageBytes);
         const int row = (id * Hkv + pc.kvh) * bs + psub * kTok;
         const uint32_t dst = ring + slot * G_::kStageBytes;
         tma_tile<D>(dst, &kmap, row, bar);
         tma_tile<D>(dst + G_::kTileBytes, &vmap, row, bar);
       } else {
-        ok[slot] = 0;
         report(a.dev_error, PA_DEVERR_BAD_BLOCK);
         mbar_arrive(bar);
       }
     }
-    if (++psub == pnsub) {
+    if (seg_end) pfirst = false;
+    if (last_sub) {
       psub = 0;
       cursor_next(pc, cum, Hkv);
-      if (pc.u < pc.u_end) pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+      if (pc.u < pend) pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
+      pnew_seg = pc.j == 0;
+    } else {
+      ++psub;
+      pnew_seg = false;
     }
+    return true;
   };
 
   // ---------------- consumer state ----------------
-  UnitCursor cc;
-  cursor_seek(cc, u0, u1, cum, B, Hkv);
-  int csub = 0;
-  bool seg_start = true, first_seg = true, timed_out = false;
-  int seg_j0 = 0;
-  int slot = 0;
-  uint32_t phases = 0;
-  int consumed = 0;
   const int g = lane >> 2, cq = lane & 3;
   uint32_t qf[KC][2], qn[KC][2];
+  int qn_b = -1, qn_kvh = -1;
   float o[KC][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
@@ -315,42 +357,23 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
     }
   };
-  if (active) load_q(qn, cc.b, cc.kvh);
+  if (active) {
+    load_q(qn, pc.b, pc.kvh);
+    qn_b = pc.b;
+    qn_kvh = pc.kvh;
+  }
 
   wait_prior_grid();  // from here on the cache, the output and the workspace are used
   zero_empty_rows<T>(a, ctx_s);
   if (!active) return;
 
   int issued = 0;
-  for (; issued < kStages && pc.u < u1; ++issued) produce(issued);
+  while (issued < kStages && produce(issued)) ++issued;
 
-  while (cc.u < u1) {
-    if (seg_start) {
-#pragma unroll
-      for (int kc = 0; kc < KC; ++kc) {
-        qf[kc][0] = qn[kc][0];
-        qf[kc][1] = qn[kc][1];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o[kc][i] = 0.f;
-      }
-      m0 = m1 = -INFINITY;
-      l0 = l1 = 0.f;
-      seg_j0 = cc.j;
-      seg_start = false;
-      // start fetching the next segment's queries now; they are used only then
-      const int64_t next_u = cc.u + (cc.nblk - cc.j);
-      if (next_u < u1) {
-        int nb = cc.b, nk = cc.kvh + 1;
-        if (nk == Hkv) {
-          nk = 0;
-          do {
-            ++nb;
-          } while (cum[nb + 1] == cum[nb]);
-        }
-        load_q(qn, nb, nk);
-      }
-    }
-
+  int slot = 0, consumed = 0;
+  uint32_t phases = 0;
+  bool timed_out = false;
+  while (consumed < issued) {
     const uint32_t bar = bar0 + slot * 8;
     // all lanes take the same decision, so the warp never splits on a timeout
     if (!__all_sync(kFull, mbar_wait_bounded(bar, (phases >> slot) & 1u))) {
@@ -359,14 +382,46 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       break;
     }
     phases ^= 1u << slot;
-    ++consumed;
+    const StageMeta md = wmeta[slot];
+    const int b = md.b, kvh = md.kvh_flags >> 16, flags = md.kvh_flags & 0xffff;
 
-    const int ctx = ctx_s[cc.b];
-    const int tok0 = cc.j * bs + csub * kTok;
-    const int n_valid = ctx - tok0 < kTok ? ctx - tok0 : kTok;
+    if (flags & kSegStart) {
+      if (qn_b == b && qn_kvh == kvh) {
+#pragma unroll
+        for (int kc = 0; kc < KC; ++kc) {
+          qf[kc][0] = qn[kc][0];
+          qf[kc][1] = qn[kc][1];
+        }
+      } else {
+        load_q(qf, b, kvh);
+      }
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[kc][i] = 0.f;
+      }
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+      // start fetching the next pair's queries now; they are used only then
+      qn_b = -1;
+      if (flags & kMoreInRange) {
+        int nb = b, nk = kvh + 1;
+        if (nk == Hkv) {
+          nk = 0;
+          do {
+            ++nb;
+          } while (cum[nb + 1] == cum[nb]);
+        }
+        load_q(qn, nb, nk);
+        qn_b = nb;
+        qn_kvh = nk;
+      }
+    }
+
+    const int n_valid = ctx_s[b] - md.tok0 < kTok ? ctx_s[b] - md.tok0 : kTok;
     const uint32_t kt = ring + slot * G_::kStageBytes;
     const uint32_t vt = kt + G_::kTileBytes;
-    const bool have = ok[slot] != 0;
+    const bool have = (flags & kHasData) != 0;
     // Move the stage into registers first and hand the slot straight back to
     // TMA, so the ring keeps loading while this warp computes.
     uint32_t ka[KC][4], va[KC][4];
@@ -393,10 +448,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
     fence_proxy_async_smem();
     __syncwarp();
-    if (pc.u < u1) {
-      produce(slot);
-      ++issued;
-    }
+    if (produce(slot)) ++issued;
 
     if (have) {
       // S^T = K . Q^T  (two accumulators to halve the dependent chain)
@@ -449,63 +501,55 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
     }
 
-    const int nsub = stages_in_block(ctx, cc.j, bs);
-    if (csub + 1 == nsub) {
-      const bool seg_end = (cc.u + 1 == u1) || (cc.j + 1 == cc.nblk);
-      if (seg_end) {
-        float L0 = l0, L1 = l1;
+    if (flags & kSegEnd) {
+      float L0 = l0, L1 = l1;
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          L0 += __shfl_xor_sync(kFull, L0, off);
-          L1 += __shfl_xor_sync(kFull, L1, off);
-        }
-        const int h0 = 2 * cq, h1 = 2 * cq + 1;
-        const bool complete = seg_j0 == 0 && cc.j + 1 == cc.nblk;
-        if (complete) {
-          T* ob = static_cast<T*>(a.out) + (static_cast<int64_t>(cc.b) * Hq + cc.kvh * G) * D;
-          const float i0 = 1.f / L0, i1 = 1.f / L1;
-#pragma unroll
-          for (int mt = 0; mt < KC; ++mt) {
-            const int d = mt * 16 + g;
-            if (h0 < G) {
-              ob[h0 * D + d] = Num<T>::from_f(o[mt][0] * i0);
-              ob[h0 * D + d + 8] = Num<T>::from_f(o[mt][2] * i0);
-            }
-            if (h1 < G) {
-              ob[h1 * D + d] = Num<T>::from_f(o[mt][1] * i1);
-              ob[h1 * D + d + 8] = Num<T>::from_f(o[mt][3] * i1);
-            }
-          }
-        } else {
-          float* piece = a.ws_pieces + (w * 2 + (first_seg ? 0 : 1)) * (G * (D + 2));
-          if (g == 0) {
-            if (h0 < G) { piece[h0] = m0; piece[G + h0] = L0; }
-            if (h1 < G) { piece[h1] = m1; piece[G + h1] = L1; }
-          }
-          float* po = piece + 2 * G;
-#pragma unroll
-          for (int mt = 0; mt < KC; ++mt) {
-            const int d = mt * 16 + g;
-            if (h0 < G) {
-              po[h0 * D + d] = o[mt][0];
-              po[h0 * D + d + 8] = o[mt][2];
-            }
-            if (h1 < G) {
-              po[h1 * D + d] = o[mt][1];
-              po[h1 * D + d + 8] = o[mt][3];
-            }
-          }
-          piece_done<T, D>(a, cum, cc.b, cc.kvh, U, W, lane);
-        }
-        first_seg = false;
-        seg_start = true;
+      for (int off = 4; off < 32; off <<= 1) {
+        L0 += __shfl_xor_sync(kFull, L0, off);
+        L1 += __shfl_xor_sync(kFull, L1, off);
       }
-      csub = 0;
-      cursor_next(cc, cum, Hkv);
-    } else {
-      ++csub;
+      const int h0 = 2 * cq, h1 = 2 * cq + 1;
+      if (flags & kComplete) {
+        T* ob = static_cast<T*>(a.out) + (static_cast<int64_t>(b) * Hq + kvh * G) * D;
+        const float i0 = 1.f / L0, i1 = 1.f / L1;
+#pragma unroll
+        for (int mt = 0; mt < KC; ++mt) {
+          const int d = mt * 16 + g;
+          if (h0 < G) {
+            ob[h0 * D + d] = Num<T>::from_f(o[mt][0] * i0);
+            ob[h0 * D + d + 8] = Num<T>::from_f(o[mt][2] * i0);
+          }
+          if (h1 < G) {
+            ob[h1 * D + d] = Num<T>::from_f(o[mt][1] * i1);
+            ob[h1 * D + d + 8] = Num<T>::from_f(o[mt][3] * i1);
+          }
+        }
+      } else {
+        const int pslot = (flags & kFirstInRange) ? 0 : 1;
+        float* piece =
+            a.ws_pieces + (static_cast<int64_t>(md.range) * 2 + pslot) * (G * (D + 2));
+        if (g == 0) {
+          if (h0 < G) { piece[h0] = m0; piece[G + h0] = L0; }
+          if (h1 < G) { piece[h1] = m1; piece[G + h1] = L1; }
+        }
+        float* po = piece + 2 * G;
+#pragma unroll
+        for (int mt = 0; mt < KC; ++mt) {
+          const int d = mt * 16 + g;
+          if (h0 < G) {
+            po[h0 * D + d] = o[mt][0];
+            po[h0 * D + d + 8] = o[mt][2];
+          }
+          if (h1 < G) {
+            po[h1 * D + d] = o[mt][1];
+            po[h1 * D + d + 8] = o[mt][3];
+          }
+        }
+        piece_done<T, D>(a, cum, b, kvh, sp, lane);
+      }
     }
     slot = slot + 1 == kStages ? 0 : slot + 1;
+    ++consumed;
   }
 
   if (timed_out) {
@@ -516,6 +560,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       phases ^= 1u << s_;
     }
   }
+  worker_finished(a, sp.W, lane);
 }
 
 template <typename T, int D>
@@ -554,7 +599,8 @@ int decode_tc_workers_per_cta() { return tc::kWarps; }
 
 size_t decode_tc_smem_bytes(int head_dim, int batch) {
   const size_t ring = static_cast<size_t>(tc::kWarps) * tc::kStages * 2 * tc::kTok * head_dim * 2;
-  const size_t meta = tc::kWarps * tc::kStages * (8 + 4) + sizeof(int32_t) * (2 * batch + 1);
+  const size_t meta = tc::kWarps * tc::kStages * (8 + sizeof(tc::StageMeta)) +
+                      sizeof(int32_t) * (2 * batch + 1);
   return 1024 + ring + meta;
 }
 

@@ -30,7 +30,7 @@ class PagedKVCache:
             self.v_cache.view(view).fill_(fill_bits)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
         ws = pa_decode_workspace_size(max_batch, num_q_heads, num_kv_heads, head_dim)
-        self.workspace = torch.empty(ws, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
 
     # ---- pool ops (host) with their device side effects ----
     def alloc(self, seq_id, n, stream=None):
