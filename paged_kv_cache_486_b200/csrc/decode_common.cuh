@@ -153,6 +153,18 @@ __device__ inline void scan_context(const DecodeArgs& a, int32_t* cum, int32_t* 
   __syncthreads();
 }
 
+// Each CTA pulls a slice of the block table into L2, so that the first block
+// ids the workers read after the context scan are L2 hits.
+__device__ inline void prefetch_tables(const DecodeArgs& a) {
+  const int64_t bytes = static_cast<int64_t>(a.batch) * a.max_blocks * 4;
+  const int64_t lines = (bytes + 127) / 128;
+  const char* base = reinterpret_cast<const char*>(a.block_tables);
+  for (int64_t l = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; l < lines;
+       l += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + l * 128));
+  }
+}
+
 // Rows of sequences with an empty context are zero; CTA (b mod grid) writes them.
 template <typename T>
 __device__ inline void zero_empty_rows(const DecodeArgs& a, const int32_t* ctx_s) {

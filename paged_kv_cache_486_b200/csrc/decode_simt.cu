@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) decode_simt_kernel(DecodeArgs
   extern __shared__ int32_t simt_smem[];
   int32_t* cum = simt_smem;
   int32_t* ctx_s = simt_smem + a.batch + 1;
+  prefetch_tables(a);
   scan_context(a, cum, ctx_s);
   wait_prior_grid();  // the cache, the output and the workspace are touched only after this
   zero_empty_rows<T>(a, ctx_s);

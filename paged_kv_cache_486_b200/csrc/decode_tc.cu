@@ -246,6 +246,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
   }
+  prefetch_tables(a);
   scan_context(a, cum, ctx_s);  // ends with __syncthreads()
 
   // Until wait_prior_grid() below the kernel reads only its inputs
