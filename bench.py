@@ -372,6 +372,62 @@ def run_e2e(args, wl, eng, dist):
             "ms_per_step": total / args.steps}
 
 
+def run_swap(args, dist, rank, world):
+    """Eviction to host memory and back: swap every sequence of the workload out to a
+    pinned host cache and in again (pa_swap on the host pools, pa_swap_blocks on the
+    GPU), timed per direction; the reference is a plain pinned copy of the same bytes."""
+    import paged_kv_cache_486_b200 as pa
+    wl = workloads.make(args.config)
+    eng, st = _setup(wl)
+    hk = torch.empty(eng.k_cache.shape, dtype=eng.k_cache.dtype).pin_memory()
+    hv = torch.empty(eng.v_cache.shape, dtype=eng.v_cache.dtype).pin_memory()
+    host = pa.Pool(wl.num_blocks, wl.bs)
+    seqs = [int(x) for x in wl.batch]
+    out_pairs = np.concatenate([pa.pa_swap(eng.pool, host, s) for s in seqs])
+    in_pairs = np.concatenate([pa.pa_swap(host, eng.pool, s) for s in seqs])
+    nbytes = len(out_pairs) * 2 * eng.k_cache[0].numel() * eng.k_cache.element_size()
+    d_out = torch.from_numpy(out_pairs).cuda()
+    d_in = torch.from_numpy(in_pairs).cuda()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(args.steps):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return statistics.mean(ms)
+
+    t_out = timed(lambda: pa.pa_swap_blocks([hk], [hv], [eng.k_cache], [eng.v_cache], d_out,
+                                            eng.dev_error))
+    t_in = timed(lambda: pa.pa_swap_blocks([eng.k_cache], [eng.v_cache], [hk], [hv], d_in,
+                                           eng.dev_error))
+    # reference: one contiguous pinned copy of the same number of bytes each way
+    hbuf = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dbuf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    r_d2h = timed(lambda: hbuf.copy_(dbuf, non_blocking=True))
+    r_h2d = timed(lambda: dbuf.copy_(hbuf, non_blocking=True))
+    assert eng.device_errors() == 0
+    gbs = lambda ms: nbytes / (ms / 1e3) / 1e9
+    return {"metric": "swap_blocks GB/s (device <-> pinned host, whole batch)", "op": "swap",
+            "value": 2 * nbytes / ((t_out + t_in) / 1e3) / 1e9, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": wl.dtype, "data": "synthetic",
+            "config": {"workload": wl.name, "blocks": int(len(out_pairs)), "bytes_each_way": nbytes},
+            "swap_out_gbs": gbs(t_out), "swap_in_gbs": gbs(t_in),
+            "swap_out_ms": t_out, "swap_in_ms": t_in, "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "host link", "unit": "GB/s",
+                         "peak": {"d2h": gbs(r_d2h), "h2d": gbs(r_h2d)},
+                         "peak_source": "contiguous pinned torch copy of the same bytes, same run",
+                         "frac": {"out": r_d2h / t_out, "in": r_h2d / t_in}}}
+
+
 # ---------------------------------------------------------- oracle timings
 def cpu_baseline(wl, target_s=10.0):
     import oracle
@@ -456,6 +512,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="step", choices=["step", "swap"],
+                    help="step: the decode step (default); swap: eviction to host and back")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -474,7 +532,8 @@ def main():
     torch.cuda.set_device(local)
     dist, rank, world = _dist()
     try:
-        line = run_ours(args, dist, rank, world)
+        line = run_swap(args, dist, rank, world) if args.op == "swap" else \
+            run_ours(args, dist, rank, world)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

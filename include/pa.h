@@ -117,6 +117,20 @@ pa_status pa_free(pa_pool* pool, int64_t seq_id);
  * PA_ERR_NOT_FOUND: unknown parent; PA_ERR_INVALID: child exists. */
 pa_status pa_fork(pa_pool* pool, int64_t parent_id, int64_t child_id);
 
+/* Fine-grained eviction ([P2] "How PagedAttention solves this": under memory
+ * pressure small pages move to the CPU instead of whole sequences): move
+ * seq_id from pool `from` to pool `to` (e.g. a device pool and a host pool of
+ * the same block size).  The sequence gets one new block in `to` per block it
+ * held (logical order) and keeps its length; each old block loses one holder,
+ * so a block shared with other sequences stays in `from` for them.
+ * pairs_out_host[2 * max_pairs] receives the (from_block, to_block) pairs the
+ * caller copies with pa_swap_blocks; *n_pairs_out their count.
+ * PA_ERR_OOM: `to` has too few free blocks; PA_ERR_NOT_FOUND: unknown sequence;
+ * PA_ERR_INVALID: the sequence is already in `to`, block sizes differ, or
+ * max_pairs is too small.  On any error nothing changes. */
+pa_status pa_swap(pa_pool* from, pa_pool* to, int64_t seq_id, int32_t* pairs_out_host,
+                  int32_t max_pairs, int32_t* n_pairs_out);
+
 /* Block-table rows for n_seqs sequences: table_out_host[i * max_blocks + j] is
  * the physical block of logical block j of seq_ids_host[i], -1 past the end;
  * ctx_lens_out_host[i] is its token count.  PA_ERR_INVALID if a sequence holds
@@ -166,6 +180,21 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache
 pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
                          int32_t num_layers, const int32_t* pairs, int32_t n_pairs,
                          int32_t num_blocks, int64_t block_bytes, int32_t* dev_error,
+                         pa_stream stream);
+
+/* Copy blocks between two sets of pools, e.g. a device cache and a host cache:
+ * for each pair (from, to) and each layer, block `to` of dst_k / dst_v becomes a
+ * byte copy of block `from` of src_k / src_v.  The four pointer arrays are host
+ * arrays of num_layers (1..128) pool pointers; every pool and `pairs`
+ * ([n_pairs, 2] int32) must be device memory or pinned host memory (the kernel
+ * reads and writes host memory across the host link directly).
+ * block_bytes = num_kv_heads * block_size * head_dim * element size (a multiple
+ * of 16).  Ids outside [0, src_num_blocks) / [0, dst_num_blocks) are skipped
+ * with PA_DEVERR_BAD_BLOCK. */
+pa_status pa_swap_blocks(void* const* dst_k_host, void* const* dst_v_host,
+                         void* const* src_k_host, void* const* src_v_host, int32_t num_layers,
+                         const int32_t* pairs, int32_t n_pairs, int32_t src_num_blocks,
+                         int32_t dst_num_blocks, int64_t block_bytes, int32_t* dev_error,
                          pa_stream stream);
 
 /* ------------------------------------------------------------------------

@@ -67,6 +67,10 @@ def lib():
         L.orc_paged_decode_attention.argtypes = [P, P, P, P, P, C.c_int32, C.c_int32, C.c_int32,
                                                  C.c_int32, C.c_int32, C.c_int32, C.c_double,
                                                  C.c_int, P, P, C.c_int64, C.c_int32]
+        L.orc_swap.restype = C.c_int
+        L.orc_swap.argtypes = [P, P, C.c_int64, P, P]
+        L.orc_copy_between.restype = C.c_int
+        L.orc_copy_between.argtypes = [P, P, P, P, C.c_int32, P, C.c_int32, C.c_int64]
         L.orc_contiguous_attention.restype = C.c_int
         L.orc_contiguous_attention.argtypes = [P, P, P, C.c_int64, C.c_int32, C.c_int32,
                                                C.c_int32, C.c_double, C.c_int, P, P, C.c_int32]
@@ -161,6 +165,24 @@ class Pool:
         st = lib().orc_block_table(self.h, _ptr(seqs), len(seqs), max_blocks, _ptr(table),
                                    _ptr(ctx))
         return st, table, ctx
+
+
+def swap(from_pool, to_pool, seq):
+    """Move `seq` from one pool to the other; returns (status, pairs int32[n, 2] (from, to))."""
+    pairs = np.zeros((max(from_pool.num_blocks, 1), 2), dtype=np.int32)
+    n = np.zeros(1, dtype=np.int32)
+    st = lib().orc_swap(from_pool.h, to_pool.h, seq, _ptr(pairs), _ptr(n))
+    if st != OK:
+        return st, None
+    return st, pairs[: int(n[0])].copy()
+
+
+def copy_between(dst_k, dst_v, src_k, src_v, pairs):
+    pairs = _c(pairs, np.int32).reshape(-1, 2)
+    L = len(dst_k)
+    arr = lambda xs: (C.c_void_p * L)(*[x.ctypes.data for x in xs])
+    return lib().orc_copy_between(arr(dst_k), arr(dst_v), arr(src_k), arr(src_v), L, _ptr(pairs),
+                                  pairs.shape[0], src_k[0][0].nbytes)
 
 
 # ---------------------------------------------------------- data movement

@@ -317,6 +317,60 @@ int orc_block_table(const void* pool, const int64_t* seqs, int32_t n_seqs, int32
   return ORC_OK;
 }
 
+// ------------------------------- swapping ----------------------------------
+// [P2] "How PagedAttention solves this", fine-grained eviction: under memory
+// pressure small pages move to the CPU instead of whole sequences staying or
+// going.  Reading: a sequence is moved between a device pool and a host pool
+// block by block: every block of the sequence gets a block in the other pool
+// (in logical order), the sequence then lives in the other pool with the same
+// length, and its old blocks lose one holder (a block shared with other
+// sequences stays where it is for them).  All or nothing.  The (from, to)
+// block pairs are what the caller copies.
+int orc_swap(void* from_pool, void* to_pool, int64_t seq, int32_t* pairs_out, int32_t* n_out) {
+  Pool* from = static_cast<Pool*>(from_pool);
+  Pool* to = static_cast<Pool*>(to_pool);
+  auto it = from->seqs.find(seq);
+  if (it == from->seqs.end()) return ORC_NOT_FOUND;
+  if (to->seqs.count(seq) || from->block_size != to->block_size) return ORC_INVALID;
+  const Sequence old = it->second;
+  if (static_cast<int64_t>(old.blocks.size()) > static_cast<int64_t>(to->free_stack.size()))
+    return ORC_OOM;
+  Sequence moved;
+  moved.len = old.len;
+  int32_t k = 0;
+  for (int32_t b : old.blocks) {
+    const int32_t nb = take_block(to);
+    moved.blocks.push_back(nb);
+    pairs_out[2 * k] = b;
+    pairs_out[2 * k + 1] = nb;
+    ++k;
+  }
+  for (int32_t b : old.blocks) drop_block(from, b);
+  from->seqs.erase(seq);
+  to->seqs.emplace(seq, moved);
+  *n_out = k;
+  return ORC_OK;
+}
+
+// Block copy between two pools (e.g. device -> host): for each pair, in order,
+// block `to` of the destination caches becomes a byte copy of block `from` of
+// the source caches, for every layer.
+int orc_copy_between(void* const* dst_k, void* const* dst_v, void* const* src_k,
+                     void* const* src_v, int32_t num_layers, const int32_t* pairs,
+                     int32_t n_pairs, int64_t block_bytes) {
+  for (int32_t i = 0; i < n_pairs; ++i) {
+    const int64_t src = pairs[2 * i];
+    const int64_t dst = pairs[2 * i + 1];
+    for (int32_t l = 0; l < num_layers; ++l) {
+      std::memcpy(static_cast<char*>(dst_k[l]) + dst * block_bytes,
+                  static_cast<const char*>(src_k[l]) + src * block_bytes, block_bytes);
+      std::memcpy(static_cast<char*>(dst_v[l]) + dst * block_bytes,
+                  static_cast<const char*>(src_v[l]) + src * block_bytes, block_bytes);
+    }
+  }
+  return ORC_OK;
+}
+
 // ----------------------------- cache write ---------------------------------
 // Store each new token's key and value rows in the cache at its slot; slot -1
 // means "no token" and is skipped.  Cache layout: [num_blocks, kv_heads,

@@ -35,6 +35,8 @@ SIGNATURES = {
     "pa_pool_destroy": (None, [_P]),
     "pa_alloc": (_I32, [_P, _I64, _I32, _P, _P, _I32, _P]),
     "pa_alloc_batch": (_I32, [_P, _P, _I32, _I32, _P, _P, _I32, _P]),
+    "pa_swap": (_I32, [_P, _P, _I64, _P, _I32, _P]),
+    "pa_swap_blocks": (_I32, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I64, _P, _P]),
     "pa_free": (_I32, [_P, _I64]),
     "pa_fork": (_I32, [_P, _I64, _I64]),
     "pa_block_table": (_I32, [_P, _P, _I32, _I32, _P, _P]),
@@ -173,6 +175,40 @@ class Pool:
 
     def pa_seq_len(self, seq_id: int) -> int:
         return lib.pa_seq_len(self._h, seq_id)
+
+
+def pa_swap(from_pool, to_pool, seq_id):
+    """Move seq_id between pools -> (from_block, to_block) pairs int32[n, 2]."""
+    n_max = max(from_pool.num_blocks, 1)
+    pairs = np.empty((n_max, 2), dtype=np.int32)
+    n = _I32(0)
+    _check(lib.pa_swap(from_pool._h, to_pool._h, seq_id, _np_ptr(pairs), n_max, C.byref(n)),
+           "pa_swap")
+    return pairs[: n.value].copy()
+
+
+def _any_ptr(t, name):
+    if not isinstance(t, torch.Tensor) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor")
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    return _P(t.data_ptr())
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, dev_error=None, stream=None):
+    """Lists of per-layer pools (CUDA or pinned host tensors) [NB, Hkv, bs, D];
+    pairs int32 [n, 2] (from, to), CUDA or pinned host."""
+    L = len(dst_k)
+    arr = lambda xs, nm: (_P * L)(*[_any_ptr(x, nm).value for x in xs])
+    n = 0 if pairs is None else pairs.shape[0]
+    if n and pairs.dtype != torch.int32:
+        raise ValueError("pairs must be int32")
+    block_bytes = src_k[0][0].numel() * src_k[0].element_size()
+    st = lib.pa_swap_blocks(arr(dst_k, "dst_k"), arr(dst_v, "dst_v"), arr(src_k, "src_k"),
+                            arr(src_v, "src_v"), L, _any_ptr(pairs, "pairs") if n else None, n,
+                            src_k[0].shape[0], dst_k[0].shape[0], block_bytes,
+                            _dev_ptr(dev_error, "dev_error", torch.int32), _stream(stream))
+    _check(st, "pa_swap_blocks")
 
 
 def pa_kv_bytes(num_layers, num_tokens, num_kv_heads, head_dim, dtype_bytes) -> int:

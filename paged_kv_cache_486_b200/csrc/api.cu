@@ -179,6 +179,60 @@ pa_status pa_copy_blocks(void* const* k_caches_host, void* const* v_caches_host,
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_copy_blocks");
 }
 
+// A pointer the kernels can dereference: device memory, managed memory, or
+// pinned (page-locked, registered) host memory; returns the device address.
+static bool device_address(const void* p, const void** out) {
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) {
+    *out = p;
+    return true;
+  }
+  if (attr.type == cudaMemoryTypeHost && attr.devicePointer) {
+    *out = attr.devicePointer;
+    return true;
+  }
+  return false;
+}
+
+pa_status pa_swap_blocks(void* const* dst_k_host, void* const* dst_v_host,
+                         void* const* src_k_host, void* const* src_v_host, int32_t num_layers,
+                         const int32_t* pairs, int32_t n_pairs, int32_t src_num_blocks,
+                         int32_t dst_num_blocks, int64_t block_bytes, int32_t* dev_error,
+                         pa_stream stream) {
+  if (num_layers < 1 || num_layers > pa::kMaxLayers || n_pairs < 0 || src_num_blocks < 0 ||
+      dst_num_blocks < 0 || block_bytes <= 0 || block_bytes % 16)
+    return fail(PA_ERR_INVALID, "pa_swap_blocks: bad sizes (layers=%d pairs=%d block_bytes=%lld)",
+                num_layers, n_pairs, static_cast<long long>(block_bytes));
+  if (n_pairs == 0) return PA_OK;
+  if (!dst_k_host || !dst_v_host || !src_k_host || !src_v_host || !pairs)
+    return fail(PA_ERR_INVALID, "pa_swap_blocks: NULL pointer");
+  const void* pairs_dev = nullptr;
+  if (!device_address(pairs, &pairs_dev))
+    return fail(PA_ERR_INVALID, "pa_swap_blocks: pairs is neither device nor pinned host memory");
+  pa::LayerPtrs dst, src;
+  std::memset(&dst, 0, sizeof dst);
+  std::memset(&src, 0, sizeof src);
+  void* const* in[4] = {dst_k_host, dst_v_host, src_k_host, src_v_host};
+  void** outp[4] = {dst.k, dst.v, src.k, src.v};
+  for (int a = 0; a < 4; ++a) {
+    for (int i = 0; i < num_layers; ++i) {
+      const void* d = nullptr;
+      if (!in[a][i] || !aligned(in[a][i], 16) || !device_address(in[a][i], &d))
+        return fail(PA_ERR_INVALID, "pa_swap_blocks: layer %d pool pointer is NULL, misaligned "
+                    "or not device-accessible (use device or pinned host memory)", i);
+      outp[a][i] = const_cast<void*>(d);
+    }
+  }
+  const cudaError_t e = pa::launch_swap_blocks(
+      dst, src, num_layers, static_cast<const int32_t*>(pairs_dev), n_pairs, src_num_blocks,
+      dst_num_blocks, block_bytes, dev_error, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_swap_blocks");
+}
+
 size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                 int32_t head_dim) {
   if (batch < 0 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||

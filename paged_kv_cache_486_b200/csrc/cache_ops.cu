@@ -86,6 +86,56 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant_
   }
 }
 
+// Block copy between two pools (device <-> pinned host memory, or device <->
+// device): block pairs[i].to of the destination becomes a copy of block
+// pairs[i].from of the source, for every layer, key and value.  Several 16-byte
+// loads are kept in flight per thread so that reads across the host link
+// (which cannot be posted like writes) overlap.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const __grid_constant__ LayerPtrs dst,
+                                                          const __grid_constant__ LayerPtrs src,
+                                                          const int32_t* __restrict__ pairs,
+                                                          int32_t src_blocks, int32_t dst_blocks,
+                                                          int64_t block_chunks,
+                                                          int32_t* dev_error) {
+  const int32_t pair = blockIdx.x;
+  const int32_t layer = blockIdx.y >> 1;
+  const bool is_v = blockIdx.y & 1;
+  const int32_t from = pairs[2 * pair];
+  const int32_t to = pairs[2 * pair + 1];
+  if (from < 0 || from >= src_blocks || to < 0 || to >= dst_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) report(dev_error, PA_DEVERR_BAD_BLOCK);
+    return;
+  }
+  const uint4* s = static_cast<const uint4*>(is_v ? src.v[layer] : src.k[layer]) + from * block_chunks;
+  uint4* d = static_cast<uint4*>(is_v ? dst.v[layer] : dst.k[layer]) + to * block_chunks;
+  constexpr int kUnroll = 8;
+  const int64_t step = static_cast<int64_t>(blockDim.x) * kUnroll;
+  for (int64_t i0 = threadIdx.x; i0 < block_chunks; i0 += step) {
+    uint4 buf[kUnroll];
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      const int64_t i = i0 + static_cast<int64_t>(k) * blockDim.x;
+      if (i < block_chunks) buf[k] = s[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      const int64_t i = i0 + static_cast<int64_t>(k) * blockDim.x;
+      if (i < block_chunks) d[i] = buf[k];
+    }
+  }
+}
+
+cudaError_t launch_swap_blocks(const LayerPtrs& dst, const LayerPtrs& src, int32_t num_layers,
+                               const int32_t* pairs, int32_t n_pairs, int32_t src_blocks,
+                               int32_t dst_blocks, int64_t block_bytes, int32_t* dev_error,
+                               cudaStream_t stream) {
+  if (n_pairs == 0) return cudaSuccess;
+  dim3 grid(n_pairs, 2 * num_layers);
+  swap_blocks_kernel<<<grid, 256, 0, stream>>>(dst, src, pairs, src_blocks, dst_blocks,
+                                               block_bytes / 16, dev_error);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k_cache,
                                      void* v_cache, const int64_t* slots, int32_t n_tokens,
                                      int32_t num_kv_heads, int32_t row_bytes, int32_t block_size,

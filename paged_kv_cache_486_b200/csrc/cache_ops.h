@@ -23,4 +23,9 @@ cudaError_t launch_copy_blocks(const LayerPtrs& ptrs, int32_t num_layers, const 
                                int32_t n_pairs, int32_t num_blocks, int64_t block_bytes,
                                int32_t* dev_error, cudaStream_t stream);
 
+cudaError_t launch_swap_blocks(const LayerPtrs& dst, const LayerPtrs& src, int32_t num_layers,
+                               const int32_t* pairs, int32_t n_pairs, int32_t src_blocks,
+                               int32_t dst_blocks, int64_t block_bytes, int32_t* dev_error,
+                               cudaStream_t stream);
+
 }  // namespace pa

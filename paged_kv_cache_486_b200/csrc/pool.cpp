@@ -188,6 +188,49 @@ pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_s
   return PA_OK;
 }
 
+// "KV Cache and PagedAttention: Why Your LLM Server Slows Down" / "How
+// PagedAttention solves this": under memory pressure small pages move to the
+// CPU.  The sequence moves to `to` with one new block per old block (logical
+// order) and the same length; its old blocks each lose one holder.  Nothing
+// changes unless `to` has room for every block.
+pa_status pa_swap(pa_pool* from, pa_pool* to, int64_t seq_id, int32_t* pairs_out_host,
+                  int32_t max_pairs, int32_t* n_pairs_out) {
+  if (!from || !to || from == to || !n_pairs_out || max_pairs < 0 ||
+      (max_pairs > 0 && !pairs_out_host))
+    return pa::fail(PA_ERR_INVALID, "pa_swap: bad arguments");
+  if (from->block_size != to->block_size)
+    return pa::fail(PA_ERR_INVALID, "pa_swap: block sizes differ (%d vs %d)", from->block_size,
+                    to->block_size);
+  auto it = from->seqs.find(seq_id);
+  if (it == from->seqs.end())
+    return pa::fail(PA_ERR_NOT_FOUND, "pa_swap: unknown sequence %lld",
+                    static_cast<long long>(seq_id));
+  if (to->seqs.count(seq_id))
+    return pa::fail(PA_ERR_INVALID, "pa_swap: sequence %lld is already in the destination pool",
+                    static_cast<long long>(seq_id));
+  const std::vector<int32_t>& src = it->second.blocks;
+  const int32_t n = static_cast<int32_t>(src.size());
+  if (n > max_pairs)
+    return pa::fail(PA_ERR_INVALID, "pa_swap: %d pairs needed, room for %d", n, max_pairs);
+  if (n > static_cast<int32_t>(to->free_stack.size()))
+    return pa::fail(PA_ERR_OOM, "pa_swap: %d blocks needed, %zu free in the destination", n,
+                    to->free_stack.size());
+  pa_pool::Seq moved;
+  moved.len = it->second.len;
+  moved.blocks.reserve(n);
+  for (int32_t k = 0; k < n; ++k) {
+    const int32_t b = to->pop();
+    moved.blocks.push_back(b);
+    pairs_out_host[2 * k] = src[k];
+    pairs_out_host[2 * k + 1] = b;
+  }
+  for (int32_t b : src) from->unref(b);
+  from->seqs.erase(it);
+  to->seqs.emplace(seq_id, std::move(moved));
+  *n_pairs_out = n;
+  return PA_OK;
+}
+
 pa_status pa_free(pa_pool* pool, int64_t seq_id) {
   if (!pool) return pa::fail(PA_ERR_INVALID, "pa_free: NULL pool");
   auto it = pool->seqs.find(seq_id);

@@ -215,3 +215,39 @@ def test_random_long_scripts():
             else:
                 m.apply(("free", int(rng.choice(live))))
             m.check()
+
+
+def test_swap_moves_a_sequence_and_its_content():
+    """Swapping out and back in keeps every sequence's content (checked cell by cell)."""
+    dev, host = oracle.Pool(6, 2), oracle.Pool(4, 2)
+    mem = {"d": np.full(12, -1), "h": np.full(8, -1)}
+    dev.alloc(1, 5)            # 3 blocks
+    dev.fork(1, 2)             # shares them
+    _, s3, _ = dev.alloc(3, 2)
+    t, _ = _used_blocks(dev, [1, 3])
+    pos = np.arange(5)
+    mem["d"][t[0][pos // 2] * 2 + pos % 2] = [10, 11, 12, 13, 14]
+    mem["d"][s3] = [30, 31]
+    st, pairs = oracle.swap(dev, host, 1)
+    assert st == oracle.OK and len(pairs) == 3
+    for a, b in pairs:
+        mem["h"][b * 2:(b + 1) * 2] = mem["d"][a * 2:(a + 1) * 2]
+    assert dev.seq_len(1) == -1 and host.seq_len(1) == 5
+    assert dev.num_free() == 6 - 3 - 1     # seq 2 still holds the shared blocks
+    th, _ = _used_blocks(host, [1])
+    assert list(mem["h"][th[0][pos // 2] * 2 + pos % 2]) == [10, 11, 12, 13, 14]
+    assert oracle.swap(dev, host, 3)[0] == oracle.OK      # 1 more host block
+    assert oracle.swap(dev, host, 2)[0] == oracle.OOM     # 3 blocks, 0 free: nothing moves
+    assert dev.seq_len(2) == 5 and host.num_free() == 0
+    st, back = oracle.swap(host, dev, 1)
+    assert st == oracle.OK
+    for a, b in back:
+        mem["d"][b * 2:(b + 1) * 2] = mem["h"][a * 2:(a + 1) * 2]
+    td, _ = _used_blocks(dev, [1])
+    assert list(mem["d"][td[0][pos // 2] * 2 + pos % 2]) == [10, 11, 12, 13, 14]
+    assert host.num_free() == 3            # the swapped-in sequence's host blocks came back
+    assert oracle.swap(dev, host, 9)[0] == oracle.NOT_FOUND
+    assert oracle.swap(host, dev, 3)[0] == oracle.OOM      # seqs 1 and 2 fill the device pool
+    assert dev.free(2) == oracle.OK
+    assert oracle.swap(host, dev, 3)[0] == oracle.OK
+    assert oracle.swap(dev, dev, 3)[0] == oracle.INVALID   # already in the destination

@@ -173,3 +173,65 @@ def test_batched_alloc_equals_sequential_and_rolls_back():
             t1, c1 = a.pa_block_table(live, nb + 1)
             t2, c2 = b.pa_block_table(live, nb + 1)
             assert np.array_equal(t1, t2) and np.array_equal(c1, c2)
+
+
+def test_swap_matches_the_oracle():
+    rng = np.random.default_rng(13)
+    for trial in range(25):
+        bs = int(rng.choice([1, 4, 16]))
+        nd, nh = int(rng.integers(4, 40)), int(rng.integers(2, 30))
+        pd, ph = pa.Pool(nd, bs), pa.Pool(nh, bs)
+        od, oh = oracle.Pool(nd, bs), oracle.Pool(nh, bs)
+        where = {}  # seq -> "d" / "h"
+        for _ in range(120):
+            r = rng.random()
+            dev_seqs = [s for s, w in where.items() if w == "d"]
+            host_seqs = [s for s, w in where.items() if w == "h"]
+            if r < 0.45 or not where:
+                s = int(rng.integers(0, 10))
+                if where.get(s) == "h":
+                    continue
+                n = int(rng.integers(0, 2 * bs + 1))
+                st, sl2, cw2 = od.alloc(s, n)
+                try:
+                    sl, cw = pd.pa_alloc(s, n)
+                    assert st == oracle.OK and np.array_equal(sl, sl2) and np.array_equal(cw, cw2)
+                    where[s] = "d"
+                except pa.PagedAttnError as e:
+                    assert e.status == st
+            elif r < 0.55 and dev_seqs:
+                p, c = int(rng.choice(dev_seqs)), int(rng.integers(0, 10))
+                if c in where:
+                    continue
+                assert od.fork(p, c) == oracle.OK
+                pd.pa_fork(p, c)
+                where[c] = "d"
+            elif r < 0.75 and dev_seqs:
+                s = int(rng.choice(dev_seqs))
+                st, pr2 = oracle.swap(od, oh, s)
+                try:
+                    pr = pa.pa_swap(pd, ph, s)
+                    assert st == oracle.OK and np.array_equal(pr, pr2)
+                    where[s] = "h"
+                except pa.PagedAttnError as e:
+                    assert e.status == st == pa.PA_ERR_OOM
+            elif r < 0.95 and host_seqs:
+                s = int(rng.choice(host_seqs))
+                st, pr2 = oracle.swap(oh, od, s)
+                try:
+                    pr = pa.pa_swap(ph, pd, s)
+                    assert st == oracle.OK and np.array_equal(pr, pr2)
+                    where[s] = "d"
+                except pa.PagedAttnError as e:
+                    assert e.status == st == pa.PA_ERR_OOM
+            elif where:
+                s = int(rng.choice(sorted(where)))
+                if where[s] == "d":
+                    pd.pa_free(s)
+                    assert od.free(s) == oracle.OK
+                else:
+                    ph.pa_free(s)
+                    assert oh.free(s) == oracle.OK
+                del where[s]
+            _same_state(pd, od, nd, sorted(s for s, w in where.items() if w == "d"), nd + 1)
+            _same_state(ph, oh, nh, sorted(s for s, w in where.items() if w == "h"), nh + 1)
