@@ -71,6 +71,16 @@ def lib():
         L.orc_swap.argtypes = [P, P, C.c_int64, P, P]
         L.orc_copy_between.restype = C.c_int
         L.orc_copy_between.argtypes = [P, P, P, P, C.c_int32, P, C.c_int32, C.c_int64]
+        L.orc_reshape_and_cache_int8.restype = C.c_int
+        L.orc_reshape_and_cache_int8.argtypes = [P, P, P, P, P, P, P, C.c_int64, C.c_int32,
+                                                 C.c_int32, C.c_int32, C.c_int32, C.c_int]
+        L.orc_quantize_rows.restype = None
+        L.orc_quantize_rows.argtypes = [P, C.c_int64, C.c_int32, C.c_int, P, P]
+        L.orc_paged_decode_attention_int8.restype = C.c_int
+        L.orc_paged_decode_attention_int8.argtypes = [P, P, P, P, P, P, P, C.c_int32, C.c_int32,
+                                                      C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                                      C.c_double, C.c_int, P, P, C.c_int64,
+                                                      C.c_int32]
         L.orc_contiguous_attention.restype = C.c_int
         L.orc_contiguous_attention.argtypes = [P, P, P, C.c_int64, C.c_int32, C.c_int32,
                                                C.c_int32, C.c_double, C.c_int, P, P, C.c_int32]
@@ -243,4 +253,53 @@ def contiguous_attention(q, k, v, scale, dtype, heads=None):
                                         0 if hs is None else len(hs))
     if st != OK:
         raise ValueError(f"oracle attention rejected its arguments ({st})")
+    return out
+
+
+# ------------------------------------------------------------- INT8 cache
+class Int8Cache:
+    """Host INT8 cache: key codes [NB, Hkv, bs, D], value codes [NB, Hkv, D, bs],
+    fp32 scales [NB, Hkv, bs] for keys and values."""
+
+    def __init__(self, num_blocks, kv_heads, block_size, head_dim):
+        self.k = np.zeros((num_blocks, kv_heads, block_size, head_dim), np.int8)
+        self.v = np.zeros((num_blocks, kv_heads, head_dim, block_size), np.int8)
+        self.ks = np.zeros((num_blocks, kv_heads, block_size), np.float32)
+        self.vs = np.zeros((num_blocks, kv_heads, block_size), np.float32)
+
+
+def quantize_rows(x, dtype):
+    x = np.ascontiguousarray(x)
+    n, D = x.shape
+    codes = np.empty((n, D), np.int8)
+    scales = np.empty(n, np.float32)
+    lib().orc_quantize_rows(_ptr(x), n, D, DTYPE_CODE[dtype], _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def reshape_and_cache_int8(key, value, cache, slots, dtype):
+    key = np.ascontiguousarray(key)
+    value = np.ascontiguousarray(value)
+    T, Hkv, D = key.shape
+    slots = _c(slots, np.int64)
+    return lib().orc_reshape_and_cache_int8(_ptr(key), _ptr(value), _ptr(cache.k), _ptr(cache.v),
+                                            _ptr(cache.ks), _ptr(cache.vs), _ptr(slots), T, Hkv,
+                                            D, cache.k.shape[2], cache.k.shape[0],
+                                            DTYPE_CODE[dtype])
+
+
+def paged_decode_attention_int8(q, cache, tables, ctx, scale, dtype, rows=None, n_threads=None):
+    q = np.ascontiguousarray(q)
+    B, Hq, D = q.shape
+    NB, Hkv, bs, _ = cache.k.shape
+    tables = _c(tables, np.int32)
+    ctx = _c(ctx, np.int32)
+    out = np.full((B, Hq, D), np.nan)
+    r = None if rows is None else _c(rows, np.int64)
+    st = lib().orc_paged_decode_attention_int8(
+        _ptr(q), _ptr(cache.k), _ptr(cache.v), _ptr(cache.ks), _ptr(cache.vs), _ptr(tables),
+        _ptr(ctx), B, Hq, Hkv, D, bs, tables.shape[1], float(scale), DTYPE_CODE[dtype], _ptr(out),
+        _ptr(r), 0 if r is None else len(r), n_threads or (os.cpu_count() or 1))
+    if st != OK:
+        raise ValueError(f"oracle int8 attention rejected its arguments ({st})")
     return out

@@ -415,6 +415,67 @@ int orc_copy_blocks(void* const* k_caches, void* const* v_caches, int32_t num_la
   return ORC_OK;
 }
 
+// ------------------------------ INT8 cache ---------------------------------
+// "KV Cache for intermediates..." / "The four solutions", KV-cache quantisation:
+// keys and values stored in 8 bits (about half the memory of fp16).  The pages
+// fix no scheme; the reading taken here: per (token, kv head), symmetric over
+// head_dim, with every step in IEEE fp32 so that the integer decisions are
+// reproducible:  amax = max_d |x_d|,  scale = amax / 127,  code_d = round to
+// nearest even of (x_d / scale), clamped to [-127, 127]; a zero row has scale 0
+// and zero codes.  A value is read back as code * scale.
+static void quantize_row(const void* src, int64_t base, int32_t D, int dtype, int8_t* codes,
+                         float* scale_out) {
+  float amax = 0.f;
+  for (int32_t d = 0; d < D; ++d)
+    amax = std::max(amax, std::fabs(static_cast<float>(load_elem(src, base + d, dtype))));
+  const float scale = amax / 127.0f;
+  for (int32_t d = 0; d < D; ++d) {
+    int32_t c = 0;
+    if (scale > 0.f) {
+      const float x = static_cast<float>(load_elem(src, base + d, dtype));
+      c = static_cast<int32_t>(std::nearbyint(x / scale));
+      c = std::min(127, std::max(-127, c));
+    }
+    codes[d] = static_cast<int8_t>(c);
+  }
+  *scale_out = scale;
+}
+
+// Write new tokens into an INT8 cache.  Key codes [NB, Hkv, bs, D]; value codes
+// stored transposed [NB, Hkv, D, bs]; scales [NB, Hkv, bs] (fp32) for each.
+int orc_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
+                               int8_t* v_codes, float* k_scales, float* v_scales,
+                               const int64_t* slots, int64_t n_tokens, int32_t kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               int dtype) {
+  const int32_t D = head_dim;
+  std::vector<int8_t> row(D);
+  for (int64_t t = 0; t < n_tokens; ++t) {
+    const int64_t slot = slots[t];
+    if (slot < 0) continue;
+    if (slot >= static_cast<int64_t>(num_blocks) * block_size) return ORC_INVALID;
+    const int64_t blk = slot / block_size, off = slot % block_size;
+    for (int32_t h = 0; h < kv_heads; ++h) {
+      const int64_t src = (t * kv_heads + h) * D;
+      const int64_t tile = blk * kv_heads + h;
+      float sc;
+      quantize_row(key, src, D, dtype, row.data(), &sc);
+      for (int32_t d = 0; d < D; ++d) k_codes[(tile * block_size + off) * D + d] = row[d];
+      k_scales[tile * block_size + off] = sc;
+      quantize_row(value, src, D, dtype, row.data(), &sc);
+      for (int32_t d = 0; d < D; ++d) v_codes[(tile * D + d) * block_size + off] = row[d];
+      v_scales[tile * block_size + off] = sc;
+    }
+  }
+  return ORC_OK;
+}
+
+// Quantise rows [n, D] (tests): codes [n, D], scales [n].
+void orc_quantize_rows(const void* x, int64_t n, int32_t D, int dtype, int8_t* codes,
+                       float* scales) {
+  for (int64_t i = 0; i < n; ++i) quantize_row(x, i * D, D, dtype, codes + i * D, scales + i);
+}
+
 // ------------------------------ attention ----------------------------------
 // One new query per sequence attends to the cached keys and values of all of
 // the sequence's tokens ([P5] "The precise scientific definition": a new token
@@ -510,6 +571,46 @@ int orc_paged_decode_attention(const void* q, const void* k_cache, const void* v
       for (int64_t i = t; i < total; i += n_threads) paged_row(a, rows ? rows[i] : i);
     });
   }
+  for (auto& th : pool) th.join();
+  return ORC_OK;
+}
+
+// Paged attention over an INT8 cache: the gather reads code * scale (exact in
+// fp64), then the same definition as above.  q / out as in the paged form.
+int orc_paged_decode_attention_int8(const void* q, const int8_t* k_codes, const int8_t* v_codes,
+                                    const float* k_scales, const float* v_scales,
+                                    const int32_t* tables, const int32_t* ctx, int32_t batch,
+                                    int32_t q_heads, int32_t kv_heads, int32_t head_dim,
+                                    int32_t block_size, int32_t max_blocks, double scale,
+                                    int dtype, double* out, const int64_t* rows, int64_t n_rows,
+                                    int32_t n_threads) {
+  if (kv_heads <= 0 || q_heads % kv_heads != 0) return ORC_INVALID;
+  const int32_t group = q_heads / kv_heads, D = head_dim, bs = block_size;
+  const int64_t total = rows ? n_rows : static_cast<int64_t>(batch) * q_heads;
+  auto one = [&](int64_t row) {
+    const int64_t b = row / q_heads;
+    const int32_t h = static_cast<int32_t>(row % q_heads);
+    const int32_t g = h / group;
+    const int64_t n = ctx[b];
+    std::vector<double> qq(D), kk(n * D), vv(n * D);
+    for (int32_t d = 0; d < D; ++d) qq[d] = load_elem(q, (b * q_heads + h) * D + d, dtype);
+    for (int64_t j = 0; j < n; ++j) {
+      const int64_t tile = static_cast<int64_t>(tables[b * max_blocks + j / bs]) * kv_heads + g;
+      const int64_t off = j % bs;
+      const double ks = k_scales[tile * bs + off], vs = v_scales[tile * bs + off];
+      for (int32_t d = 0; d < D; ++d) {
+        kk[j * D + d] = ks * k_codes[(tile * bs + off) * D + d];
+        vv[j * D + d] = vs * v_codes[(tile * D + d) * bs + off];
+      }
+    }
+    attend_one(qq.data(), kk.data(), vv.data(), n, D, scale, out + row * D);
+  };
+  if (n_threads < 1) n_threads = 1;
+  std::vector<std::thread> pool;
+  for (int32_t t = 0; t < n_threads; ++t)
+    pool.emplace_back([&, t]() {
+      for (int64_t i = t; i < total; i += n_threads) one(rows ? rows[i] : i);
+    });
   for (auto& th : pool) th.join();
   return ORC_OK;
 }
