@@ -58,7 +58,7 @@ def _peak_hbm():
 def _kernel_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_486_b200", "csrc")
-    for name in ("decode_tc.cu", "decode_common.cuh", "decode_simt.cu"):
+    for name in ("decode_tc.cuh", "decode_tc.cu", "decode_common.cuh", "decode_simt.cu"):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -292,6 +292,57 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
                          int32_t* num_workers_out);
 
 /* ------------------------------------------------------------------------
+ * INT8 KV cache.  [P5] "The four solutions", KV-cache quantisation: keys and
+ * values stored in 8 bits take about half the memory (and read bandwidth) of
+ * fp16.  Scheme (reading; the pages fix none): per (token, kv head), symmetric
+ * over head_dim, every step in IEEE fp32:
+ *   amax = max_d |x_d|,  scale = amax / 127,
+ *   code_d = round-half-to-even(x_d / scale) clamped to [-127, 127]
+ * (a row of zeros has scale 0 and zero codes); an element reads back as
+ * code * scale.  Layout per layer:
+ *   k_codes  [num_blocks, num_kv_heads, block_size, head_dim] int8
+ *   v_codes  [num_blocks, num_kv_heads, head_dim, block_size] int8 (transposed:
+ *            one head_dim row holds the block's tokens)
+ *   k_scales, v_scales [num_blocks, num_kv_heads, block_size] float32.
+ * Block copies (copy-on-write, eviction) of an INT8 cache are pa_copy_blocks /
+ * pa_swap_blocks calls on the code pools (block_bytes = num_kv_heads *
+ * block_size * head_dim) and on the scale pools (num_kv_heads * block_size * 4).
+ * ---------------------------------------------------------------------- */
+
+/* Quantise new tokens into an INT8 cache: as pa_reshape_and_cache (same
+ * key / value / slot_mapping arguments, `dtype` is that of key and value: f32,
+ * f16 or bf16), but each (token, kv head) row is written as codes + scale by
+ * the scheme above; codes and scales are bit-exact to it.  head_dim 64 or 128;
+ * every pointer 16-byte aligned (slot_mapping 8).  Slots outside the pool set
+ * PA_DEVERR_BAD_SLOT and are skipped; -1 is skipped silently. */
+pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
+                                    int8_t* v_codes, float* k_scales, float* v_scales,
+                                    const int64_t* slot_mapping, int32_t n_tokens,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                                    pa_stream stream);
+
+/* Decode attention over an INT8 cache: the definition of pa_decode_attention
+ * with K_b[j, g, :] = k_code * k_scale and V_b[j, g, :] = v_code * v_scale of
+ * token j.  q and out in `dtype` (f16 or bf16); head_dim 128; group
+ * (num_q_heads / num_kv_heads) <= 8; block_size in {16, 32, 64, 128};
+ * num_blocks * num_kv_heads * max(block_size, 128) < 2^31; code pools and
+ * scale pools 16-byte aligned.  block_tables, context_lens, workspace (same
+ * size, zero-once contract and reuse as pa_decode_attention), dev_error, the
+ * work split and flags are those of pa_decode_attention_ex; num_workers = 0
+ * chooses automatically.  Runs on tensor cores: codes are converted exactly
+ * to fp16 / bf16, products accumulate in fp32, out is rounded once. */
+pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_codes,
+                                   const int8_t* v_codes, const float* k_scales,
+                                   const float* v_scales, const int32_t* block_tables,
+                                   const int32_t* context_lens, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t block_size, int32_t num_blocks, int32_t max_blocks,
+                                   float scale, pa_dtype dtype, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_error,
+                                   int32_t num_workers, int32_t flags, pa_stream stream);
+
+/* ------------------------------------------------------------------------
  * Host-side validators (no device work): PA_OK or PA_ERR_INVALID + message.
  * ---------------------------------------------------------------------- */
 /* Every slot is -1 or in [0, num_blocks * block_size), and no slot repeats. */

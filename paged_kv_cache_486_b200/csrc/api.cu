@@ -12,6 +12,7 @@
 #include "decode_common.cuh"
 #include "decode_launch.h"
 #include "host_common.h"
+#include "int8_launch.h"
 
 namespace {
 
@@ -99,6 +100,68 @@ bool tile_map(CUtensorMap* out, const void* base, int64_t rows, int head_dim, pa
   e.dtype = dt;
   g_maps_next = (g_maps_next + 1) % 8;
   *out = e.map;
+  return true;
+}
+
+// INT8 cache maps.  Keys [rows = NB * Hkv * bs, 128] bytes are seen as
+// [rows / 4][2][128] (groups of 4 tokens, 2 tokens, bytes) with strides 512 and
+// 128: a box {128, 2, 4} is tokens {4i, 4i + 1} of 4 consecutive groups.  k_hi
+// starts 256 bytes (2 tokens) later, so its boxes are tokens {4i + 2, 4i + 3}.
+// Values [NB * Hkv * 128 rows, bs] bytes: a box {16, 128} is 16 tokens of every
+// head_dim row of one (block, kv head).
+bool make_int8_maps(pa::Int8Maps* m, const void* k_codes, const void* v_codes, int64_t rows,
+                    int block_size) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const auto u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t kd[3] = {128, 2, static_cast<cuuint64_t>(rows / 4)};
+  cuuint64_t ks[2] = {128, 512};
+  cuuint32_t kb[3] = {128, 2, 4};
+  cuuint32_t e3[3] = {1, 1, 1};
+  const char* kbase = static_cast<const char*>(k_codes);
+  for (int half = 0; half < 2; ++half) {
+    CUtensorMap* out = half ? &m->k_hi : &m->k_lo;
+    const CUresult r = enc(out, u8, 3, const_cast<char*>(kbase + 256 * half), kd, ks, kb, e3,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+  }
+  cuuint64_t vd[2] = {static_cast<cuuint64_t>(block_size),
+                      static_cast<cuuint64_t>(rows / block_size * 128)};
+  cuuint64_t vs[1] = {static_cast<cuuint64_t>(block_size)};
+  cuuint32_t vb[2] = {16, 128};
+  cuuint32_t e2[2] = {1, 1};
+  return enc(&m->v, u8, 2, const_cast<void*>(v_codes), vd, vs, vb, e2,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+struct Int8MapEntry {
+  const void* k;
+  const void* v;
+  int64_t rows;
+  int block_size;
+  pa::Int8Maps maps;
+};
+thread_local Int8MapEntry g_int8_maps[4];
+thread_local int g_int8_next = 0;
+
+bool int8_maps(pa::Int8Maps* out, const void* k, const void* v, int64_t rows, int block_size) {
+  for (auto& e : g_int8_maps) {
+    if (e.k == k && e.v == v && e.rows == rows && e.block_size == block_size) {
+      *out = e.maps;
+      return true;
+    }
+  }
+  Int8MapEntry& e = g_int8_maps[g_int8_next];
+  if (!make_int8_maps(&e.maps, k, v, rows, block_size)) return false;
+  e.k = k;
+  e.v = v;
+  e.rows = rows;
+  e.block_size = block_size;
+  g_int8_next = (g_int8_next + 1) % 4;
+  *out = e.maps;
   return true;
 }
 
@@ -334,6 +397,8 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.q = q;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
+  a.k_scales = nullptr;
+  a.v_scales = nullptr;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.dev_error = dev_error;
@@ -378,6 +443,133 @@ pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, con
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, workspace, workspace_bytes, dev_error,
                                 PA_PATH_AUTO, 0, 0, stream);
+}
+
+pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
+                                    int8_t* v_codes, float* k_scales, float* v_scales,
+                                    const int64_t* slot_mapping, int32_t n_tokens,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
+                                    pa_stream stream) {
+  if (!valid_dtype(dtype) || n_tokens < 0 || num_kv_heads < 1 || block_size < 1 ||
+      num_blocks < 0 || (head_dim != 64 && head_dim != 128))
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: bad sizes (n_tokens=%d "
+                "kv_heads=%d head_dim=%d block_size=%d num_blocks=%d)", n_tokens, num_kv_heads,
+                head_dim, block_size, num_blocks);
+  if (n_tokens == 0) return PA_OK;
+  if (!key || !value || !k_codes || !v_codes || !k_scales || !v_scales || !slot_mapping)
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: NULL pointer");
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_codes, 16) ||
+      !aligned(v_codes, 16) || !aligned(k_scales, 16) || !aligned(v_scales, 16) ||
+      !aligned(slot_mapping, 8))
+    return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: misaligned pointer");
+  pa::Int8WriteArgs a;
+  a.key = key;
+  a.value = value;
+  a.k_codes = k_codes;
+  a.v_codes = v_codes;
+  a.k_scales = k_scales;
+  a.v_scales = v_scales;
+  a.slots = slot_mapping;
+  a.n_tokens = n_tokens;
+  a.num_kv_heads = num_kv_heads;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.dev_error = dev_error;
+  const cudaError_t e =
+      pa::launch_reshape_and_cache_int8(a, dtype, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_reshape_and_cache_int8");
+}
+
+pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_codes,
+                                   const int8_t* v_codes, const float* k_scales,
+                                   const float* v_scales, const int32_t* block_tables,
+                                   const int32_t* context_lens, int32_t batch,
+                                   int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                   int32_t block_size, int32_t num_blocks, int32_t max_blocks,
+                                   float scale, pa_dtype dtype, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_error,
+                                   int32_t num_workers, int32_t flags, pa_stream stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: queries must be fp16 or bf16");
+  if (batch < 0 || batch > pa::kMaxBatch)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: batch %d outside [0, %d]", batch,
+                pa::kMaxBatch);
+  if (num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads ||
+      num_q_heads / num_kv_heads > 8)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: num_q_heads %d must be 1..8 times "
+                "num_kv_heads %d", num_q_heads, num_kv_heads);
+  if (head_dim != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: head_dim %d is not 128", head_dim);
+  if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: block_size %d not in "
+                "{16, 32, 64, 128}", block_size);
+  if (num_blocks < 0 || max_blocks < 0)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: negative num_blocks or max_blocks");
+  const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * 128 >= (int64_t(1) << 31) ||
+      rows >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: num_blocks * num_kv_heads * "
+                "max(block_size, 128) >= 2^31");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention_int8: scale is NaN");
+  if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: batch * num_kv_heads > %d",
+                pa::kMaxArrivals);
+  if (flags & ~PA_DECODE_OVERLAP_PROLOGUE)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: unknown flags 0x%x", flags);
+  if (batch == 0) return PA_OK;
+  if (num_blocks == 0)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: empty pool");
+  if (!out || !q || !k_codes || !v_codes || !k_scales || !v_scales || !block_tables ||
+      !context_lens || !workspace)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: NULL pointer");
+  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_codes, 16) || !aligned(v_codes, 16) ||
+      !aligned(k_scales, 16) || !aligned(v_scales, 16) || !aligned(workspace, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: misaligned pointer");
+  const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim);
+  if (workspace_bytes < need)
+    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: workspace %zu bytes < %zu needed",
+                workspace_bytes, need);
+  const int group = num_q_heads / num_kv_heads;
+  int workers = (sm_count() ? sm_count() : 148) * pa::decode_int8_workers_per_cta();
+  if (num_workers > 0) workers = num_workers;
+  if (workers > max_workers(group)) workers = max_workers(group);
+
+  pa::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_cache = k_codes;
+  a.v_cache = v_codes;
+  a.k_scales = k_scales;
+  a.v_scales = v_scales;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.dev_error = dev_error;
+  a.ws_ctrl = static_cast<uint32_t*>(workspace);
+  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + 256);
+  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                         pieces_offset(batch, num_kv_heads));
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks = max_blocks;
+  a.workers = workers;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  pa::Int8Maps maps;
+  if (!int8_maps(&maps, k_codes, v_codes, rows, block_size))
+    return fail(PA_ERR_CUDA, "pa_decode_attention_int8: cuTensorMapEncodeTiled failed");
+  const int per = pa::decode_int8_workers_per_cta();
+  const cudaError_t e =
+      pa::launch_decode_int8(a, dtype, maps, (workers + per - 1) / per,
+                             (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0,
+                             static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_decode_attention_int8 (decode kernel)");
 }
 
 pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {

@@ -47,6 +47,8 @@ struct DecodeArgs {
   const void* q;
   const void* k_cache;
   const void* v_cache;
+  const float* k_scales;  // 8-bit caches: per-token scales [NB, Hkv, bs] (else unused)
+  const float* v_scales;
   const int32_t* block_tables;
   const int32_t* context_lens;
   int32_t* dev_error;

@@ -1,0 +1,250 @@
+// Paged decode attention on tensor cores over an INT8 cache.
+//
+// Cache ("KV Cache for intermediates..." / "The four solutions", KV-cache
+// quantisation): key codes [NB, Hkv, bs, 128] int8, value codes transposed
+// [NB, Hkv, 128, bs] int8, one fp32 scale per (block, kv head, token) for keys
+// and for values; a key or value element reads back as code * scale.
+//
+// Stage (16 tokens of one block and kv head, 4224 bytes):
+//  * keys: 16 rows of 128 bytes, loaded as two TMA boxes of 8 rows.  The box
+//    of tokens {4i, 4i+1} lands in lines 0..7 and the box of tokens
+//    {4i+2, 4i+3} in lines 8..15, 128-byte swizzled, so line r holds token
+//    tau(r) = 4 (r mod 8 >> 1) + (r & 1) + 2 (r >= 8);
+//  * values: 128 rows (one per head_dim index) of the stage's 16 token bytes;
+//  * the 16 key scales and 16 value scales (two bulk copies of 64 bytes).
+// Products.  The rows of S^T = K . Q^T follow the key lines, so S^T row r is
+// token tau(r).  The contraction index of the first product is reordered so
+// that a lane's four key bytes (one 32-bit ldmatrix element, d = 16kc + 4cq
+// .. +3) are its four A elements; the query fragment uses the same order.  In
+// O^T += V^T . P^T a lane's four value bytes are tokens 4cq .. 4cq+3, which is
+// exactly the token order that the register transpose of S^T rows tau(.)
+// gives the P^T fragment, so neither operand is shuffled.  Codes become 16-bit
+// values exactly (|code| <= 127) by integer bit tricks, then every product is
+// the same mma as in the 16-bit path.
+// Scales.  Key scales multiply the score rows (with scale * log2 e).  Value
+// scales are folded into P: p'_j = p_j * vs_j / sigma with sigma the running
+// maximum of the segment's value scales (p' in [0, 1] whatever the scales'
+// magnitude; O is rescaled when sigma grows, and the output is O * sigma).
+// The softmax sum l keeps the unscaled p.
+//
+// Roofline.  Per context token and KV head the kernel must read 128 + 128 bytes
+// of codes and 4 + 4 bytes of scales: 264 bytes against 512 for fp16.
+#include "decode_tc.cuh"
+#include "int8_launch.h"
+
+namespace pa {
+namespace tc {
+
+// Four int8 codes (bytes of w) as two pairs of 16-bit values: .x = bytes 0, 1,
+// .y = bytes 2, 3.  fp16: 0x64 in the high byte makes 1024 + u with u the
+// biased code c + 128, and 1152 is subtracted.  bf16 (7-bit significand) goes
+// through fp32 the same way: 0x4B0000uu is 2^23 + u, minus 2^23 + 128.
+template <typename T>
+__device__ __forceinline__ uint2 codes_to(uint32_t w);
+
+template <>
+__device__ __forceinline__ uint2 codes_to<__half>(uint32_t w) {
+  const uint32_t x = w ^ 0x80808080u;
+  uint32_t lo = __byte_perm(x, 0x64646464u, 0x5140);
+  uint32_t hi = __byte_perm(x, 0x64646464u, 0x7362);
+  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));
+  const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&l), *reinterpret_cast<const uint32_t*>(&h));
+}
+
+template <>
+__device__ __forceinline__ uint2 codes_to<__nv_bfloat16>(uint32_t w) {
+  const uint32_t x = w ^ 0x80808080u;
+  float f[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    f[i] = __uint_as_float(__byte_perm(x, 0x4Bu, 0x4650 + i)) - 8388736.0f;
+  return make_uint2(pack2<__nv_bfloat16>(f[0], f[1]), pack2<__nv_bfloat16>(f[2], f[3]));
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                       uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                       uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Token of S^T row g (g < 8); row g + 8 holds that token + 2.
+__device__ __forceinline__ int row_token(int g) { return 4 * (g >> 1) + (g & 1); }
+
+template <typename T>
+struct Tiles8 {
+  static constexpr int D = 128;
+  static constexpr int KC = D / 16;
+  static constexpr int kStages = 5;
+  static constexpr int kKBytes = kTok * D;
+  static constexpr int kVBytes = kTok * D;
+  static constexpr int kSBytes = 2 * kTok * 4;
+  static constexpr int kStageBytes = kKBytes + kVBytes + kSBytes;
+  static constexpr int kSlots = kWarps * kStages;
+  // all key tiles, then all value tiles, then all scales (key tiles stay
+  // 1024-byte aligned for the swizzle)
+  static constexpr int kRingBytes = kSlots * kStageBytes;
+  static_assert(kRingBytes % 1024 == 0, "ring size");
+  using Maps = Int8Maps;
+  struct Frag {
+    uint32_t k[KC][2];  // [kc][row g, row g + 8]: 4 codes, d = 16kc + 4cq .. +3
+    uint32_t v[KC][2];  // [mt][d = 16mt + g, +8]: 4 codes, tokens 4cq .. +3
+    float ks0, ks1, vs0, vs1;  // scales of the lane's tokens row_token(g), +2
+  };
+  struct Seg {
+    float sig, inv;
+    __device__ void reset() { sig = inv = 0.f; }
+    __device__ float out_scale() const { return sig; }
+  };
+
+  __device__ static void prefetch(const Maps& m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_lo)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_hi)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.v)) : "memory");
+  }
+  __device__ static uint32_t ktile(uint32_t ring0, int i) { return ring0 + i * kKBytes; }
+  __device__ static uint32_t vtile(uint32_t ring0, int i) {
+    return ring0 + kSlots * kKBytes + i * kVBytes;
+  }
+  __device__ static uint32_t stile(uint32_t ring0, int i) {
+    return ring0 + kSlots * (kKBytes + kVBytes) + i * kSBytes;
+  }
+
+  __device__ static void issue(const Maps& m, const DecodeArgs& a, uint32_t ring0, int warp,
+                               int slot, int tile, int tok, uint32_t bar) {
+    const int i = warp * kStages + slot;
+    const int row = tile * a.block_size + tok;  // a multiple of 16
+    const uint32_t kd = ktile(ring0, i);
+    tma_3d(kd, &m.k_lo, 0, 0, row >> 2, bar);
+    tma_3d(kd + 1024, &m.k_hi, 0, 0, row >> 2, bar);
+    tma_2d(vtile(ring0, i), &m.v, tok, tile * D, bar);
+    const uint32_t sd = stile(ring0, i);
+    bulk_copy(sd, a.k_scales + row, kTok * 4, bar);
+    bulk_copy(sd + kTok * 4, a.v_scales + row, kTok * 4, bar);
+  }
+  // lane (g, cq) holds q[g][16kc + 4cq, +1] and q[g][16kc + 4cq + 2, +3]
+  __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 4 * cq + 2 * half; }
+
+  __device__ static void load(const DecodeArgs&, uint32_t ring0, int warp, int slot, int,
+                              int lane, Frag& f) {
+    const int i = warp * kStages + slot;
+    const uint32_t kt = ktile(ring0, i), vt = vtile(ring0, i), st = stile(ring0, i);
+    const int mi = lane >> 3, r8 = lane & 7;
+    const int line = r8 + ((mi & 1) << 3);
+#pragma unroll
+    for (int kk = 0; kk < KC / 2; ++kk) {
+      uint32_t r[4];
+      ldsm_x4(kt + line * 128 + (((2 * kk + (mi >> 1)) ^ r8) << 4), r);
+      f.k[2 * kk][0] = r[0];
+      f.k[2 * kk][1] = r[1];
+      f.k[2 * kk + 1][0] = r[2];
+      f.k[2 * kk + 1][1] = r[3];
+      ldsm_x4(vt + (32 * kk + 16 * (mi >> 1) + line) * 16, r);
+      f.v[2 * kk][0] = r[0];
+      f.v[2 * kk][1] = r[1];
+      f.v[2 * kk + 1][0] = r[2];
+      f.v[2 * kk + 1][1] = r[3];
+    }
+    const int tk = row_token(lane >> 2);
+    f.ks0 = lds_f32(st + 4 * tk);
+    f.ks1 = lds_f32(st + 4 * (tk + 2));
+    f.vs0 = lds_f32(st + kTok * 4 + 4 * tk);
+    f.vs1 = lds_f32(st + kTok * 4 + 4 * (tk + 2));
+  }
+
+  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const DecodeArgs& a,
+                                int n_valid, int lane, float (&t)[4]) {
+    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+      const uint2 r0 = codes_to<T>(f.k[kc][0]);
+      const uint2 r1 = codes_to<T>(f.k[kc][1]);
+      const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
+      if (kc & 1) mma16816<T>(s2, A, qf[kc]); else mma16816<T>(s, A, qf[kc]);
+    }
+    const int tk = row_token(lane >> 2);
+    const float k0 = f.ks0 * a.scale_log2, k1 = f.ks1 * a.scale_log2;
+    t[0] = (s[0] + s2[0]) * k0;
+    t[1] = (s[1] + s2[1]) * k0;
+    t[2] = (s[2] + s2[2]) * k1;
+    t[3] = (s[3] + s2[3]) * k1;
+    if (tk >= n_valid) t[0] = t[1] = -INFINITY;
+    if (tk + 2 >= n_valid) t[2] = t[3] = -INFINITY;
+  }
+
+  __device__ static void pv(const Frag& f, const float (&p)[4], float (&o)[KC][4], Seg& seg,
+                            int n_valid, int lane) {
+    const int tk = row_token(lane >> 2);
+    const float w0 = tk < n_valid ? f.vs0 : 0.f;
+    const float w1 = tk + 2 < n_valid ? f.vs1 : 0.f;
+    // the stage's largest value scale: the same in every lane
+    float mx = fmaxf(w0, w1);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+    if (mx > seg.sig) {
+      const float r = seg.sig / mx;
+#pragma unroll
+      for (int mt = 0; mt < KC; ++mt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mt][e] *= r;
+      }
+      seg.sig = mx;
+      seg.inv = 1.f / mx;
+    }
+    const float u0 = w0 * seg.inv, u1 = w1 * seg.inv;
+    uint32_t h01, t01, h23, t23;
+    split2<T>(p[0] * u0, p[1] * u0, h01, t01);
+    split2<T>(p[2] * u1, p[3] * u1, h23, t23);
+    const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
+    const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
+#pragma unroll
+    for (int mt = 0; mt < KC; ++mt) {
+      const uint2 r0 = codes_to<T>(f.v[mt][0]);
+      const uint2 r1 = codes_to<T>(f.v[mt][1]);
+      const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
+      mma16816<T>(o[mt], A, pb);
+      mma16816<T>(o[mt], A, pt);
+    }
+  }
+};
+
+}  // namespace tc
+
+int decode_int8_workers_per_cta() { return tc::kWarps; }
+
+cudaError_t launch_decode_int8(const DecodeArgs& a, pa_dtype dtype, const Int8Maps& maps,
+                               int num_ctas, bool overlap, cudaStream_t stream) {
+  if (dtype == PA_F16)
+    return tc::launch_tc<__half, 128, tc::Tiles8<__half>>(a, maps, num_ctas, overlap, stream);
+  return tc::launch_tc<__nv_bfloat16, 128, tc::Tiles8<__nv_bfloat16>>(a, maps, num_ctas, overlap,
+                                                                      stream);
+}
+
+}  // namespace pa

@@ -1,621 +1,139 @@
-// Paged decode attention on B200 tensor cores, K/V tiles staged by TMA.
+// Paged decode attention on tensor cores over an fp16 / bf16 cache.
 //
-// Shape of the work.  For one (sequence b, kv head) the G query heads that
-// share the KV head ("KV Cache for intermediates..." / "The four solutions",
-// GQA) form an 8-column operand, so each 16-token tile of keys and values is
-// read from HBM once per KV head and used by all G heads:
-//   S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]          (mma m16n8k16)
-//   O^T[D x 8 heads]     += V^T[D x 16] . P^T[16 x 8]       (mma m16n8k16)
-// Heads beyond G (G < 8) are zero query rows whose results are not stored.
-// Scores are kept in base-2 units (scale * log2 e) with an online softmax in
-// fp32 registers.  The exchange of P^T between the two products is a register
-// transpose (movmatrix), so P never goes through shared memory.
-//
-// Data movement.  Every warp is an independent worker (see decode_common.cuh)
-// with its own ring of kStages stage buffers.  Lane 0 issues, kStages stages
-// ahead of the consumer, the TMA loads of a stage: 16 rows x D of the key pool
-// and of the value pool, rows (block * Hkv + kv_head) * block_size + 16s, each
-// as D/64 boxes of 16 rows x 64 columns.  A box lands 128-byte-swizzled with
-// one row per 128-byte line, so the eight rows an ldmatrix reads sit in eight
-// different bank groups (with whole 256-byte rows in one box, rows t and t+4
-// would share banks).
-// Block ids come from the block table through a per-warp window of 32 ids
-// held one per lane and loaded one window ahead.  Each stage signals an
-// mbarrier with its byte count; every wait on it is bounded in time.
+// Stage: 16 rows x D of the key pool and of the value pool, rows
+// (block * Hkv + kv_head) * block_size + 16 s, each loaded as D/64 TMA boxes of
+// 16 rows x 64 columns.  A box lands 128-byte-swizzled with one row per
+// 128-byte line, so the eight rows an ldmatrix reads sit in eight different
+// bank groups (with whole 256-byte rows in one box, rows t and t+4 would share
+// banks).  Keys enter S^T = K . Q^T as the A operand straight from ldmatrix;
+// values enter O^T += V^T . P^T through ldmatrix.trans.
 //
 // Roofline.  Per context token and KV head the kernel must read D*2 bytes of
 // key and D*2 of value; tensor-core work is ~4*8*D flops per token and KV head
 // (8 padded heads), far below the tensor rate, so HBM bandwidth bounds it.
-#include <cuda.h>
-#include <cuda_runtime.h>
-
-#include <cstdint>
-
-#include "decode_common.cuh"
-#include "decode_launch.h"
+#include "decode_tc.cuh"
 
 namespace pa {
 namespace tc {
 
-constexpr int kTok = 16;     // tokens per stage (one mma tile of keys)
-constexpr int kWarps = 8;    // workers per CTA
-constexpr int kStages = 3;   // ring depth per worker
-constexpr unsigned kFull = 0xffffffffu;
-
-template <int D>
-struct Geo {
+template <typename T, int D>
+struct Tiles16 {
+  static constexpr int KC = D / 16;
+  static constexpr int kStages = 3;
   static constexpr int kTileBytes = kTok * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
-};
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase with `parity` to complete; false after ~2^31 clock
-// cycles (about a second) or 2^24 polls, whichever comes first.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t i = 0; i < (1u << 24); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > (1ll << 31)) break;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-constexpr int kBoxBytes = kTok * 64 * 2;  // one 16 x 64 box of 16-bit elements
-
-// The tile of 16 rows x D: D/64 boxes, box h holding columns [64h, 64h + 64).
-template <int D>
-__device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row,
-                                         uint32_t bar) {
-#pragma unroll
-  for (int h = 0; h < D / 64; ++h) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst + h * kBoxBytes),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(64 * h), "r"(row), "r"(bar)
-        : "memory");
-  }
-}
-
-// Byte address of 16-byte chunk `chunk` (0 .. D/8-1) of token row `tok`: box
-// chunk / 8, line tok, position (chunk mod 8) ^ (tok mod 8) (128-byte swizzle).
-__device__ __forceinline__ uint32_t swz(uint32_t tile, int tok, int chunk) {
-  return tile + (chunk >> 3) * kBoxBytes + tok * 128 + (((chunk & 7) ^ (tok & 7)) << 4);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
-}
-
-template <typename T>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4],
-                                         const uint32_t (&b)[2]);
-
-template <>
-__device__ __forceinline__ void mma16816<__half>(float (&c)[4], const uint32_t (&a)[4],
-                                                 const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-template <>
-__device__ __forceinline__ void mma16816<__nv_bfloat16>(float (&c)[4], const uint32_t (&a)[4],
-                                                        const uint32_t (&b)[2]) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
-template <typename T>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi);
-template <>
-__device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-template <>
-__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-template <typename T>
-__device__ __forceinline__ float2 unpack2(uint32_t x);
-template <>
-__device__ __forceinline__ float2 unpack2<__half>(uint32_t x) {
-  return __half22float2(*reinterpret_cast<const __half2*>(&x));
-}
-template <>
-__device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t x) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x));
-}
-
-// Softmax weights as a head + tail pair of 16-bit values (p = head + tail up to
-// ~16 significant bits), so that P . V keeps fp32-like accuracy even for bf16,
-// whose 8-bit significand alone would cost ~2^-9 |v| wherever outputs cancel.
-template <typename T>
-__device__ __forceinline__ void split2(float a, float b, uint32_t& head, uint32_t& tail) {
-  head = pack2<T>(a, b);
-  const float2 h = unpack2<T>(head);
-  tail = pack2<T>(a - h.x, b - h.y);
-}
-
-// Block id of unit u (or -1 past the worker's range), for the id window.
-__device__ __forceinline__ int32_t unit_block_id(const DecodeArgs& a, const int32_t* cum,
-                                                 int64_t u, int64_t u1) {
-  if (u >= u1) return -1;
-  const int b = find_seq(cum, a.batch, u, a.num_kv_heads);
-  const int nblk = cum[b + 1] - cum[b];
-  const int64_t rem = u - static_cast<int64_t>(a.num_kv_heads) * cum[b];
-  const int j = static_cast<int>(rem % nblk);
-  return __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j]);
-}
-
-__device__ __forceinline__ int stages_in_block(int ctx, int j, int bs) {
-  const int rem = ctx - j * bs;
-  const int n = rem < bs ? rem : bs;
-  return (n + kTok - 1) / kTok;
-}
-
-// What the producer lane tells the consumer about a stage it issued.
-constexpr int kHasData = 1;       // the tile was loaded (its block id was in range)
-constexpr int kSegStart = 2;      // first stage of a segment
-constexpr int kSegEnd = 4;        // last stage of a segment
-constexpr int kComplete = 8;      // the segment is a whole (sequence, kv head)
-constexpr int kFirstInRange = 16; // the segment holds its range's first unit (piece slot 0)
-constexpr int kMoreInRange = 32;  // the range continues after this (sequence, kv head)
-
-struct StageMeta {
-  int32_t b;
-  int32_t kvh_flags;  // kv head << 16 | flags
-  int32_t tok0;       // first token of the stage in the sequence
-  int32_t range;      // range the stage belongs to (piece slots)
-};
-
-template <typename T, int D>
-__global__ void __launch_bounds__(kWarps * 32, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
-                     const __grid_constant__ CUtensorMap vmap, DecodeArgs a) {
-  using G_ = Geo<D>;
-  constexpr int KC = D / 16;  // 16-wide chunks of head_dim
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t ring0 = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (ring0 - raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + G_::kRingBytes);
-  StageMeta* meta = reinterpret_cast<StageMeta*>(bars + kWarps * kStages);
-  int32_t* cum = reinterpret_cast<int32_t*>(meta + kWarps * kStages);
-  int32_t* ctx_s = cum + a.batch + 1;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(smem_u32(&bars[i]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
-  }
-  prefetch_tables(a);
-  scan_context(a, cum, ctx_s);  // ends with __syncthreads()
-
-  // Until wait_prior_grid() below the kernel reads only its inputs
-  // (context_lens, block_tables, q): with overlap enabled this prologue runs
-  // while the preceding kernel (typically the cache write) is still finishing.
-  const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
-  const int bs = a.block_size;
-  const Split sp = make_split(static_cast<int64_t>(Hkv) * cum[B], a.workers);
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const bool active = w < sp.W;  // false for every warp when there is no work
-
-  const uint32_t ring = ring0 + warp * kStages * G_::kStageBytes;
-  const uint32_t bar0 = smem_u32(&bars[warp * kStages]);
-  StageMeta* wmeta = meta + warp * kStages;
-
-  // ---------------- producer state (uniform across the warp) ----------------
-  int64_t prange = w;
-  int64_t pend = active ? sp.end(w) : 0;
-  UnitCursor pc;
-  cursor_seek(pc, active ? sp.start(w) : 0, pend, cum, B, Hkv);
-  int psub = 0;
-  int pnsub = active ? stages_in_block(ctx_s[pc.b], pc.j, bs) : 0;
-  bool pdone = !active, pnew_seg = true, pfirst = true;
-  int pseg_j0 = 0;
-  int64_t win = active ? sp.start(w) : 0;
-  int32_t ids_cur = unit_block_id(a, cum, win + lane, pend);
-  int32_t ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
-
-  // Issues the next stage into `slot` (claiming a tail chunk when the current
-  // range is used up); false when there is nothing left to issue.
-  auto produce = [&](int slot) -> bool {
-    if (pdone) return false;
-    if (pc.u >= pend) {
-      const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
-      if (chunk >= sp.NC) {
-        pdone = true;
-        return false;
-      }
-      prange = sp.W + chunk;
-      win = sp.start(prange);
-      pend = sp.end(prange);
-      cursor_seek(pc, win, pend, cum, B, Hkv);
-      psub = 0;
-      pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
-      pnew_seg = pfirst = true;
-      ids_cur = unit_block_id(a, cum, win + lane, pend);
-      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
-    }
-    if (pc.u >= win + 32) {
-      win += 32;
-      ids_cur = ids_next;
-      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
-    }
-    const int32_t id = __shfl_sync(kFull, ids_cur, static_cast<int>(pc.u - win));
-    if (pnew_seg) pseg_j0 = pc.j;
-    const int64_t pair_end = pc.u - pc.j + pc.nblk;  // one past the pair's last unit
-    const bool last_sub = psub + 1 == pnsub;
-    const bool seg_end = last_sub && (pc.u + 1 == pend || pc.j + 1 == pc.nblk);
-    const bool ok = id >= 0 && id < a.num_blocks;
-    const int flags = (ok ? kHasData : 0) | (pnew_seg ? kSegStart : 0) | (seg_end ? kSegEnd : 0) |
-                      (pseg_j0 == 0 && pair_end <= pend ? kComplete : 0) |
-                      (pfirst ? kFirstInRange : 0) | (pair_end < pend ? kMoreInRange : 0);
-    if (lane == 0) {
-      wmeta[slot] = StageMeta{pc.b, (pc.kvh << 16) | flags, pc.j * bs + psub * kTok,
-                              static_cast<int32_t>(prange)};
-      const uint32_t bar = bar0 + slot * 8;
-      if (ok) {
-        mbar_arrive_expect_tx(bar, G_::kStageBytes);
-        const int row = (id * Hkv + pc.kvh) * bs + psub * kTok;
-        const uint32_t dst = ring + slot * G_::kStageBytes;
-        tma_tile<D>(dst, &kmap, row, bar);
-        tma_tile<D>(dst + G_::kTileBytes, &vmap, row, bar);
-      } else {
-        report(a.dev_error, PA_DEVERR_BAD_BLOCK);
-        mbar_arrive(bar);
-      }
-    }
-    if (seg_end) pfirst = false;
-    if (last_sub) {
-      psub = 0;
-      cursor_next(pc, cum, Hkv);
-      if (pc.u < pend) pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
-      pnew_seg = pc.j == 0;
-    } else {
-      ++psub;
-      pnew_seg = false;
-    }
-    return true;
+  struct Maps {
+    CUtensorMap k, v;
+  };
+  struct Frag {
+    uint32_t k[KC][4], v[KC][4];
+  };
+  struct Seg {
+    __device__ void reset() {}
+    __device__ float out_scale() const { return 1.f; }
   };
 
-  // ---------------- consumer state ----------------
-  const int g = lane >> 2, cq = lane & 3;
-  uint32_t qf[KC][2], qn[KC][2];
-  int qn_b = -1, qn_kvh = -1;
-  float o[KC][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  __device__ static void prefetch(const Maps& m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.v)) : "memory");
+  }
+  __device__ static uint32_t stage(uint32_t ring0, int warp, int slot) {
+    return ring0 + (warp * kStages + slot) * kStageBytes;
+  }
+  __device__ static void issue(const Maps& m, const DecodeArgs& a, uint32_t ring0, int warp,
+                               int slot, int tile, int tok, uint32_t bar) {
+    const int row = tile * a.block_size + tok;
+    const uint32_t dst = stage(ring0, warp, slot);
+    tma_tile<D>(dst, &m.k, row, bar);
+    tma_tile<D>(dst + kTileBytes, &m.v, row, bar);
+  }
+  // lane (g, cq) holds q[g][16kc + 2cq, +1] and q[g][16kc + 8 + 2cq, +1]
+  __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 8 * half + 2 * cq; }
 
-  // Query fragments (B operand, k = head_dim, n = head) of pair (b, kvh):
-  // lane (g, cq) holds q[g][16kc + 2cq, +1] and q[g][16kc + 8 + 2cq, +1].
-  auto load_q = [&](uint32_t (&dst)[KC][2], int b, int kvh) {
-    const T* qb = static_cast<const T*>(a.q) + (static_cast<int64_t>(b) * Hq + kvh * G) * D;
+  __device__ static void load(const DecodeArgs&, uint32_t ring0, int warp, int slot,
+                              int n_valid, int lane, Frag& f) {
+    const uint32_t kt = stage(ring0, warp, slot);
+    const uint32_t vt = kt + kTileBytes;
+    if (n_valid < kTok) {
+      // rows past the context may hold anything (even NaN): clear them in V
+      const int per_box = (kTok - n_valid) * 8;  // 16-byte chunks past the context
+      for (int i = lane; i < per_box * (D / 64); i += 32) {
+        const int h = i / per_box, r = i - h * per_box;
+        const uint32_t addr = vt + h * kBoxBytes + n_valid * 128 + r * 16;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+      }
+      __syncwarp();
+    }
+    const int mi = lane >> 3;
+    const int ktok = ((mi & 1) << 3) + (lane & 7);
+    const int vtok = ((mi >> 1) << 3) + (lane & 7);
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      ldsm_x4(swz(kt, ktok, 2 * c + (mi >> 1)), f.k[c]);
+      ldsm_x4_trans(swz(vt, vtok, 2 * c + (mi & 1)), f.v[c]);
+    }
+  }
+
+  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const DecodeArgs& a,
+                                int n_valid, int lane, float (&t)[4]) {
+    // two accumulators halve the dependent chain
+    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-      if (g < G) {
-        dst[kc][0] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 2 * cq));
-        dst[kc][1] = __ldg(reinterpret_cast<const uint32_t*>(qb + g * D + kc * 16 + 8 + 2 * cq));
-      } else {
-        dst[kc][0] = dst[kc][1] = 0u;
-      }
+      if (kc & 1) mma16816<T>(s2, f.k[kc], qf[kc]); else mma16816<T>(s, f.k[kc], qf[kc]);
     }
-  };
-  if (active) {
-    load_q(qn, pc.b, pc.kvh);
-    qn_b = pc.b;
-    qn_kvh = pc.kvh;
+    const int g = lane >> 2;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) t[i] = (s[i] + s2[i]) * a.scale_log2;
+    if (g >= n_valid) t[0] = t[1] = -INFINITY;
+    if (g + 8 >= n_valid) t[2] = t[3] = -INFINITY;
   }
 
-  wait_prior_grid();  // from here on the cache, the output and the workspace are used
-  zero_empty_rows<T>(a, ctx_s);
-  if (!active) return;
-
-  int issued = 0;
-  while (issued < kStages && produce(issued)) ++issued;
-
-  int slot = 0, consumed = 0;
-  uint32_t phases = 0;
-  bool timed_out = false;
-  while (consumed < issued) {
-    const uint32_t bar = bar0 + slot * 8;
-    // all lanes take the same decision, so the warp never splits on a timeout
-    if (!__all_sync(kFull, mbar_wait_bounded(bar, (phases >> slot) & 1u))) {
-      if (lane == 0) report(a.dev_error, PA_DEVERR_TIMEOUT);
-      timed_out = true;
-      break;
-    }
-    phases ^= 1u << slot;
-    const StageMeta md = wmeta[slot];
-    const int b = md.b, kvh = md.kvh_flags >> 16, flags = md.kvh_flags & 0xffff;
-
-    if (flags & kSegStart) {
-      if (qn_b == b && qn_kvh == kvh) {
+  __device__ static void pv(const Frag& f, const float (&p)[4], float (&o)[KC][4], Seg&, int,
+                            int) {
+    uint32_t h01, t01, h23, t23;
+    split2<T>(p[0], p[1], h01, t01);
+    split2<T>(p[2], p[3], h23, t23);
+    const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
+    const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
+    // O^T += V^T . (P_head + P_tail)^T
 #pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
-          qf[kc][0] = qn[kc][0];
-          qf[kc][1] = qn[kc][1];
-        }
-      } else {
-        load_q(qf, b, kvh);
-      }
-#pragma unroll
-      for (int kc = 0; kc < KC; ++kc) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) o[kc][i] = 0.f;
-      }
-      m0 = m1 = -INFINITY;
-      l0 = l1 = 0.f;
-      // start fetching the next pair's queries now; they are used only then
-      qn_b = -1;
-      if (flags & kMoreInRange) {
-        int nb = b, nk = kvh + 1;
-        if (nk == Hkv) {
-          nk = 0;
-          do {
-            ++nb;
-          } while (cum[nb + 1] == cum[nb]);
-        }
-        load_q(qn, nb, nk);
-        qn_b = nb;
-        qn_kvh = nk;
-      }
-    }
-
-    const int n_valid = ctx_s[b] - md.tok0 < kTok ? ctx_s[b] - md.tok0 : kTok;
-    const uint32_t kt = ring + slot * G_::kStageBytes;
-    const uint32_t vt = kt + G_::kTileBytes;
-    const bool have = (flags & kHasData) != 0;
-    // Move the stage into registers first and hand the slot straight back to
-    // TMA, so the ring keeps loading while this warp computes.
-    uint32_t ka[KC][4], va[KC][4];
-    if (have) {
-      if (n_valid < kTok) {
-        // rows past the context may hold anything (even NaN): clear them in V
-        const int per_box = (kTok - n_valid) * 8;  // 16-byte chunks past the context
-        for (int i = lane; i < per_box * (D / 64); i += 32) {
-          const int h = i / per_box, r = i - h * per_box;
-          const uint32_t addr = vt + h * kBoxBytes + n_valid * 128 + r * 16;
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
-                       : "memory");
-        }
-        __syncwarp();
-      }
-      const int mi = lane >> 3;
-      const int ktok = ((mi & 1) << 3) + (lane & 7);
-      const int vtok = ((mi >> 1) << 3) + (lane & 7);
-#pragma unroll
-      for (int c = 0; c < KC; ++c) {
-        ldsm_x4(swz(kt, ktok, 2 * c + (mi >> 1)), ka[c]);
-        ldsm_x4_trans(swz(vt, vtok, 2 * c + (mi & 1)), va[c]);
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (produce(slot)) ++issued;
-
-    if (have) {
-      // S^T = K . Q^T  (two accumulators to halve the dependent chain)
-      float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kc = 0; kc < KC; ++kc) {
-        if (kc & 1) mma16816<T>(s2, ka[kc], qf[kc]); else mma16816<T>(s, ka[kc], qf[kc]);
-      }
-      // scores of (tok g, head 2cq), (g, 2cq+1), (g+8, 2cq), (g+8, 2cq+1)
-      float t0 = (s[0] + s2[0]) * a.scale_log2, t1 = (s[1] + s2[1]) * a.scale_log2;
-      float t2 = (s[2] + s2[2]) * a.scale_log2, t3 = (s[3] + s2[3]) * a.scale_log2;
-      if (g >= n_valid) t0 = t1 = -INFINITY;
-      if (g + 8 >= n_valid) t2 = t3 = -INFINITY;
-      float x0 = fmaxf(t0, t2), x1 = fmaxf(t1, t3);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, off));
-        x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, off));
-      }
-      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      const float p0 = exp2f(t0 - n0), p1 = exp2f(t1 - n1);
-      const float p2 = exp2f(t2 - n0), p3 = exp2f(t3 - n1);
-      // rescale the running sums only when some head's maximum moved
-      if (__any_sync(kFull, n0 > m0 || n1 > m1)) {
-        const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
-        l0 *= a0;
-        l1 *= a1;
-#pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
-          o[kc][0] *= a0;
-          o[kc][1] *= a1;
-          o[kc][2] *= a0;
-          o[kc][3] *= a1;
-        }
-        m0 = n0;
-        m1 = n1;
-      }
-      l0 += p0 + p2;
-      l1 += p1 + p3;
-      uint32_t h01, t01, h23, t23;
-      split2<T>(p0, p1, h01, t01);
-      split2<T>(p2, p3, h23, t23);
-      const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
-      const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
-      // O^T += V^T . (P_head + P_tail)^T
-#pragma unroll
-      for (int mt = 0; mt < KC; ++mt) {
-        mma16816<T>(o[mt], va[mt], pb);
-        mma16816<T>(o[mt], va[mt], pt);
-      }
-    }
-
-    if (flags & kSegEnd) {
-      float L0 = l0, L1 = l1;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        L0 += __shfl_xor_sync(kFull, L0, off);
-        L1 += __shfl_xor_sync(kFull, L1, off);
-      }
-      const int h0 = 2 * cq, h1 = 2 * cq + 1;
-      if (flags & kComplete) {
-        T* ob = static_cast<T*>(a.out) + (static_cast<int64_t>(b) * Hq + kvh * G) * D;
-        const float i0 = 1.f / L0, i1 = 1.f / L1;
-#pragma unroll
-        for (int mt = 0; mt < KC; ++mt) {
-          const int d = mt * 16 + g;
-          if (h0 < G) {
-            ob[h0 * D + d] = Num<T>::from_f(o[mt][0] * i0);
-            ob[h0 * D + d + 8] = Num<T>::from_f(o[mt][2] * i0);
-          }
-          if (h1 < G) {
-            ob[h1 * D + d] = Num<T>::from_f(o[mt][1] * i1);
-            ob[h1 * D + d + 8] = Num<T>::from_f(o[mt][3] * i1);
-          }
-        }
-      } else {
-        const int pslot = (flags & kFirstInRange) ? 0 : 1;
-        float* piece =
-            a.ws_pieces + (static_cast<int64_t>(md.range) * 2 + pslot) * (G * (D + 2));
-        if (g == 0) {
-          if (h0 < G) { piece[h0] = m0; piece[G + h0] = L0; }
-          if (h1 < G) { piece[h1] = m1; piece[G + h1] = L1; }
-        }
-        float* po = piece + 2 * G;
-#pragma unroll
-        for (int mt = 0; mt < KC; ++mt) {
-          const int d = mt * 16 + g;
-          if (h0 < G) {
-            po[h0 * D + d] = o[mt][0];
-            po[h0 * D + d + 8] = o[mt][2];
-          }
-          if (h1 < G) {
-            po[h1 * D + d] = o[mt][1];
-            po[h1 * D + d + 8] = o[mt][3];
-          }
-        }
-        piece_done<T, D>(a, cum, b, kvh, sp, lane);
-      }
-    }
-    slot = slot + 1 == kStages ? 0 : slot + 1;
-    ++consumed;
-  }
-
-  if (timed_out) {
-    // let copies already in flight land before the CTA's shared memory goes away
-    for (int k = consumed; k < issued; ++k) {
-      const int s_ = k % kStages;
-      mbar_wait_bounded(bar0 + s_ * 8, (phases >> s_) & 1u);
-      phases ^= 1u << s_;
+    for (int mt = 0; mt < KC; ++mt) {
+      mma16816<T>(o[mt], f.v[mt], pb);
+      mma16816<T>(o[mt], f.v[mt], pt);
     }
   }
-  worker_finished(a, sp.W, lane);
-}
-
-template <typename T, int D>
-static cudaError_t launch_t(const DecodeArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                            int num_ctas, bool overlap, cudaStream_t stream) {
-  const size_t smem = decode_tc_smem_bytes(D, a.batch);
-  auto kern = decode_tc_kernel<T, D>;
-  // the opt-in shared-memory limit is per device; raise it once to the most any
-  // batch can ask for
-  static bool raised[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || !raised[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(decode_tc_smem_bytes(D, kMaxBatch)));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) raised[dev] = true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_ctas);
-  cfg.blockDim = dim3(kWarps * 32);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, a);
-}
+};
 
 }  // namespace tc
 
 int decode_tc_workers_per_cta() { return tc::kWarps; }
 
 size_t decode_tc_smem_bytes(int head_dim, int batch) {
-  const size_t ring = static_cast<size_t>(tc::kWarps) * tc::kStages * 2 * tc::kTok * head_dim * 2;
-  const size_t meta = tc::kWarps * tc::kStages * (8 + sizeof(tc::StageMeta)) +
-                      sizeof(int32_t) * (2 * batch + 1);
-  return 1024 + ring + meta;
+  return head_dim == 128 ? tc::tc_smem_bytes<tc::Tiles16<__half, 128>>(batch)
+                         : tc::tc_smem_bytes<tc::Tiles16<__half, 64>>(batch);
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
                              const CUtensorMap& vmap, int num_ctas, bool overlap,
                              cudaStream_t stream) {
+  using tc::Tiles16;
   if (a.head_dim == 128) {
-    return dtype == PA_F16
-               ? tc::launch_t<__half, 128>(a, kmap, vmap, num_ctas, overlap, stream)
-               : tc::launch_t<__nv_bfloat16, 128>(a, kmap, vmap, num_ctas, overlap, stream);
+    if (dtype == PA_F16) {
+      using P = Tiles16<__half, 128>;
+      return tc::launch_tc<__half, 128, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
+    }
+    using P = Tiles16<__nv_bfloat16, 128>;
+    return tc::launch_tc<__nv_bfloat16, 128, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap,
+                                                stream);
   }
-  return dtype == PA_F16
-             ? tc::launch_t<__half, 64>(a, kmap, vmap, num_ctas, overlap, stream)
-             : tc::launch_t<__nv_bfloat16, 64>(a, kmap, vmap, num_ctas, overlap, stream);
+  if (dtype == PA_F16) {
+    using P = Tiles16<__half, 64>;
+    return tc::launch_tc<__half, 64, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
+  }
+  using P = Tiles16<__nv_bfloat16, 64>;
+  return tc::launch_tc<__nv_bfloat16, 64, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
 }
 
 }  // namespace pa

@@ -66,3 +66,35 @@ def gathered(eng, bt, ctx, b, kind, heads=None):
 def bits(t):
     t = t.contiguous()
     return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)
+
+
+def build_int8(wl, poison=True, workers=0, stream=None):
+    """As build(), over an INT8 cache (PagedKVCacheInt8)."""
+    from paged_kv_cache_486_b200.engine import PagedKVCacheInt8
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCacheInt8(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda",
+                           fill_bits=0x5A if poison else None)
+
+    def tokens(seq, pos0, n):
+        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
+
+    eng.apply_ops(wl.ops, tokens, stream)
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    q = wl.q("cuda")
+    out = eng.decode(q, bt, ctx, wl.scale, num_workers=workers, stream=stream)
+    torch.cuda.synchronize()
+    return dict(eng=eng, bt=bt, ctx=ctx, q=q, out=out)
+
+
+def gathered_int8(eng, bt, ctx, b, kvh):
+    """(k codes [n, D], v codes [n, D], k scales [n], v scales [n]) of batch row b and
+    kv head kvh in logical order, read through its table (torch indexing)."""
+    n = int(ctx[b])
+    bs = eng.block_size
+    pos = torch.arange(n, device=eng.k_codes.device)
+    blk = bt[b].long()[pos // bs]
+    off = pos % bs
+    # per-head views first, so each gather has one advanced-index pattern
+    kc, vc = eng.k_codes[:, kvh], eng.v_codes[:, kvh]  # [NB, bs, D], [NB, D, bs]
+    return (kc[blk, off, :], vc[blk, :, off], eng.k_scales[:, kvh][blk, off],
+            eng.v_scales[:, kvh][blk, off])

@@ -76,3 +76,50 @@ def contiguous_row(wl, b, heads=None):
                                         wl.dtype)
         out[h] = o[0]
     return out
+
+
+def run_script_int8(wl):
+    """The op script through the oracle pool with an INT8 cache (copy-on-write
+    copies move codes and scales).  Returns dict(pool, table, ctx, cache)."""
+    pool = oracle.Pool(wl.num_blocks, wl.bs)
+    cache = oracle.Int8Cache(wl.num_blocks, wl.Hkv, wl.bs, wl.D)
+    for op in wl.ops:
+        if op[0] == "alloc":
+            _, seq, n, pos0, write = op
+            st, slots, cow = pool.alloc(seq, n)
+            assert st == oracle.OK, (op, st)
+            if len(cow):
+                oracle.copy_blocks([cache.k], [cache.v], cow)      # codes
+                oracle.copy_blocks([cache.ks], [cache.vs], cow)    # scales
+            if write and n > 0:
+                k = raw(wl.tokens(seq, pos0, n, 0))
+                v = raw(wl.tokens(seq, pos0, n, 1))
+                assert oracle.reshape_and_cache_int8(k, v, cache, slots, wl.dtype) == oracle.OK
+        elif op[0] == "fork":
+            assert pool.fork(op[1], op[2]) == oracle.OK
+        else:
+            assert pool.free(op[1]) == oracle.OK
+    st, table, ctx = pool.block_table(wl.batch, wl.max_blocks)
+    assert st == oracle.OK
+    return dict(pool=pool, table=table, ctx=ctx, cache=cache)
+
+
+def int8_contiguous_row(wl, b, heads):
+    """Oracle INT8 attention of batch row b for the listed query heads, from the
+    sequence's logical rows quantised into a fresh one-sequence oracle cache (the
+    scheme is per (token, kv head), so each kv head is quantised on its own)."""
+    seq = int(wl.batch[b])
+    q = raw(wl.q()[b])
+    out = np.full((wl.Hq, wl.D), np.nan)
+    for h in heads:
+        g = h // wl.G
+        k = raw(wl.contiguous_kv(seq, 0, heads=[g]))
+        v = raw(wl.contiguous_kv(seq, 1, heads=[g]))
+        n = k.shape[0]
+        nb = max(1, -(-n // wl.bs))
+        cache = oracle.Int8Cache(nb, 1, wl.bs, wl.D)
+        assert oracle.reshape_and_cache_int8(k, v, cache, np.arange(n), wl.dtype) == oracle.OK
+        o = oracle.paged_decode_attention_int8(q[h:h + 1][None], cache, np.arange(nb)[None],
+                                               [n], wl.scale, wl.dtype)
+        out[h] = o[0, 0]
+    return out
