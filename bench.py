@@ -428,6 +428,118 @@ def run_swap(args, dist, rank, world):
                          "frac": {"out": r_d2h / t_out, "in": r_h2d / t_in}}}
 
 
+def run_int8(args, dist, rank, world):
+    """The decode step over an INT8 cache (PagedKVCacheInt8): quantising cache write of
+    the step's tokens, then decode attention over codes + per-token scales."""
+    import paged_kv_cache_486_b200 as pa
+    from paged_kv_cache_486_b200.engine import PagedKVCacheInt8
+    wl = workloads.make(args.config)
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCacheInt8(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda")
+
+    def tokens(seq, pos0, n):
+        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
+
+    eng.apply_ops(wl.ops[:wl.n_prefill_ops], tokens)
+    slots, keys, vals, copies = [], [], [], []
+    for op in wl.decode_ops():
+        _, seq, n, pos0, _w = op
+        sl, cow = eng.alloc(seq, n)
+        slots.append(sl)
+        copies.extend(cow.tolist())
+        k, v = tokens(seq, pos0, n)
+        keys.append(k)
+        vals.append(v)
+    slots = torch.from_numpy(np.concatenate(slots)).cuda()
+    key, value = torch.cat(keys), torch.cat(vals)
+    pairs = torch.tensor(copies, dtype=torch.int32, device="cuda").reshape(-1, 2)
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    q = wl.q("cuda")
+    out = torch.empty_like(q)
+    flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    n_pairs = pairs.shape[0]
+
+    def decode(flags=0):
+        eng.decode(q, bt, ctx, wl.scale, out=out, flags=flags)
+
+    def step():
+        if n_pairs:
+            pa.pa_copy_blocks([eng.k_codes], [eng.v_codes], pairs, eng.dev_error)
+            pa.pa_copy_blocks([eng.k_scales], [eng.v_scales], pairs, eng.dev_error)
+        eng.write(key, value, slots)
+        decode(pa.PA_DECODE_OVERLAP_PROLOGUE)
+
+    step()
+    torch.cuda.synchronize()
+    g_step, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step()
+    with torch.cuda.graph(g_dec):
+        decode()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(graph, n):
+        ms = []
+        for _ in range(n):
+            _flush_l2(flush)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return ms
+
+    timed(g_step, args.warmup)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    step_ms = timed(g_step, args.steps)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    timed(g_dec, args.warmup)
+    decode_ms = timed(g_dec, args.steps)
+    torch.cuda.synchronize()
+    assert eng.device_errors() == 0, "device guards fired"
+    del g_step, g_dec
+
+    total_ms, _, value = aggregate(dist, sum(step_ms), wl.B * args.steps)
+    c = wl.context_lens().astype(np.int64)
+    kv = int(c.sum()) * wl.Hkv * (2 * wl.D + 8)        # codes + fp32 scales, keys and values
+    qo = 2 * wl.B * wl.Hq * wl.D * wl.elem_bytes
+    tables = int(((c + wl.bs - 1) // wl.bs).sum()) * 4 + 4 * wl.B
+    alg = kv + qo + tables
+    dec_ms = statistics.mean(decode_ms)
+    achieved = alg / (dec_ms / 1e3) / 1e9
+    peak, peak_kind = _peak_hbm()
+    launches = 2 + (2 if n_pairs else 0)
+    return {
+        "metric": METRIC + " (INT8 KV cache)", "op": "int8", "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": f"{wl.dtype} queries, int8 cache (fp32 scales)",
+        "data": "synthetic (seeded counter-based N(0,1) stand-in values, shuffled block pool)",
+        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+                   "head_dim": wl.D, "block_size": wl.bs, "layers_per_step": 1,
+                   "context_tokens": int(c.sum()), "kv_read_bytes_per_step": alg,
+                   "parallelism": f"replicas x{world}",
+                   "timing": "CUDA-graph replay of the step (INT8 cache write + INT8 decode), "
+                             "CUDA events per step",
+                   "l2": "flushed between timed steps (256 MiB read outside the events)"},
+        "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3, "decode_us_min": min(decode_ms) * 1e3,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
+                     "traffic": None,
+                     "timed": "pa_decode_attention_int8 call (one kernel), graph replay"},
+        "gpu_launches": launches * args.steps, "clocks": clocks,
+    }
+
+
 # ---------------------------------------------------------- oracle timings
 def cpu_baseline(wl, target_s=10.0):
     import oracle
@@ -512,8 +624,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="step", choices=["step", "swap"],
-                    help="step: the decode step (default); swap: eviction to host and back")
+    ap.add_argument("--op", default="step", choices=["step", "swap", "int8"],
+                    help="step: the decode step (default); swap: eviction to host and back; "
+                         "int8: the decode step over an INT8 cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -532,8 +645,8 @@ def main():
     torch.cuda.set_device(local)
     dist, rank, world = _dist()
     try:
-        line = run_swap(args, dist, rank, world) if args.op == "swap" else \
-            run_ours(args, dist, rank, world)
+        run = {"swap": run_swap, "int8": run_int8}.get(args.op, run_ours)
+        line = run(args, dist, rank, world)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -301,8 +301,9 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  * (a row of zeros has scale 0 and zero codes); an element reads back as
  * code * scale.  Layout per layer:
  *   k_codes  [num_blocks, num_kv_heads, block_size, head_dim] int8
- *   v_codes  [num_blocks, num_kv_heads, head_dim, block_size] int8 (transposed:
- *            one head_dim row holds the block's tokens)
+ *   v_codes  [num_blocks, num_kv_heads, block_size / 16, head_dim, 16] int8
+ *            (transposed in groups of 16 tokens: one group's values form a
+ *            contiguous head_dim x 16 tile, one row per head_dim index)
  *   k_scales, v_scales [num_blocks, num_kv_heads, block_size] float32.
  * Block copies (copy-on-write, eviction) of an INT8 cache are pa_copy_blocks /
  * pa_swap_blocks calls on the code pools (block_bytes = num_kv_heads *
@@ -313,7 +314,7 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  * key / value / slot_mapping arguments, `dtype` is that of key and value: f32,
  * f16 or bf16), but each (token, kv head) row is written as codes + scale by
  * the scheme above; codes and scales are bit-exact to it.  head_dim 64 or 128;
- * every pointer 16-byte aligned (slot_mapping 8).  Slots outside the pool set
+ * block_size a multiple of 16; every pointer 16-byte aligned (slot_mapping 8).  Slots outside the pool set
  * PA_DEVERR_BAD_SLOT and are skipped; -1 is skipped silently. */
 pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
                                     int8_t* v_codes, float* k_scales, float* v_scales,

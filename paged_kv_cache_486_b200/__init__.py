@@ -307,11 +307,12 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, contex
 def pa_reshape_and_cache_int8(key, value, k_codes, v_codes, k_scales, v_scales, slot_mapping,
                               dev_error=None, stream=None):
     """Quantise key/value [T, Hkv, D] into an INT8 cache: k_codes int8 [NB, Hkv, bs, D],
-    v_codes int8 [NB, Hkv, D, bs], k_scales / v_scales float32 [NB, Hkv, bs] (all CUDA)."""
+    v_codes int8 [NB, Hkv, bs/16, D, 16], k_scales / v_scales float32 [NB, Hkv, bs]
+    (all CUDA)."""
     T, Hkv, D = key.shape
     NB, Hkv2, bs, D2 = k_codes.shape
     if ((Hkv, D) != (Hkv2, D2) or value.shape != key.shape
-            or tuple(v_codes.shape) != (NB, Hkv, D, bs)
+            or tuple(v_codes.shape) != (NB, Hkv, bs // 16, D, 16)
             or tuple(k_scales.shape) != (NB, Hkv, bs) or v_scales.shape != k_scales.shape):
         raise ValueError("shape mismatch between key/value and the INT8 cache")
     st = lib.pa_reshape_and_cache_int8(

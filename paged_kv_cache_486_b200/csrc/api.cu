@@ -107,13 +107,9 @@ bool tile_map(CUtensorMap* out, const void* base, int64_t rows, int head_dim, pa
 // [rows / 4][2][128] (groups of 4 tokens, 2 tokens, bytes) with strides 512 and
 // 128: a box {128, 2, 4} is tokens {4i, 4i + 1} of 4 consecutive groups.  k_hi
 // starts 256 bytes (2 tokens) later, so its boxes are tokens {4i + 2, 4i + 3}.
-// Values [NB * Hkv * 128 rows, bs] bytes: a box {16, 128} is 16 tokens of every
-// head_dim row of one (block, kv head).
-bool make_int8_maps(pa::Int8Maps* m, const void* k_codes, const void* v_codes, int64_t rows,
-                    int block_size) {
+bool make_int8_maps(pa::Int8Maps* m, const void* k_codes, int64_t rows) {
   auto enc = encode_fn();
   if (!enc) return false;
-  const auto u8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   cuuint64_t kd[3] = {128, 2, static_cast<cuuint64_t>(rows / 4)};
   cuuint64_t ks[2] = {128, 512};
   cuuint32_t kb[3] = {128, 2, 4};
@@ -121,45 +117,34 @@ bool make_int8_maps(pa::Int8Maps* m, const void* k_codes, const void* v_codes, i
   const char* kbase = static_cast<const char*>(k_codes);
   for (int half = 0; half < 2; ++half) {
     CUtensorMap* out = half ? &m->k_hi : &m->k_lo;
-    const CUresult r = enc(out, u8, 3, const_cast<char*>(kbase + 256 * half), kd, ks, kb, e3,
+    const CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                           const_cast<char*>(kbase + 256 * half), kd, ks, kb, e3,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
   }
-  cuuint64_t vd[2] = {static_cast<cuuint64_t>(block_size),
-                      static_cast<cuuint64_t>(rows / block_size * 128)};
-  cuuint64_t vs[1] = {static_cast<cuuint64_t>(block_size)};
-  cuuint32_t vb[2] = {16, 128};
-  cuuint32_t e2[2] = {1, 1};
-  return enc(&m->v, u8, 2, const_cast<void*>(v_codes), vd, vs, vb, e2,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return true;
 }
 
 struct Int8MapEntry {
   const void* k;
-  const void* v;
   int64_t rows;
-  int block_size;
   pa::Int8Maps maps;
 };
 thread_local Int8MapEntry g_int8_maps[4];
 thread_local int g_int8_next = 0;
 
-bool int8_maps(pa::Int8Maps* out, const void* k, const void* v, int64_t rows, int block_size) {
+bool int8_maps(pa::Int8Maps* out, const void* k, int64_t rows) {
   for (auto& e : g_int8_maps) {
-    if (e.k == k && e.v == v && e.rows == rows && e.block_size == block_size) {
+    if (e.k == k && e.rows == rows) {
       *out = e.maps;
       return true;
     }
   }
   Int8MapEntry& e = g_int8_maps[g_int8_next];
-  if (!make_int8_maps(&e.maps, k, v, rows, block_size)) return false;
+  if (!make_int8_maps(&e.maps, k, rows)) return false;
   e.k = k;
-  e.v = v;
   e.rows = rows;
-  e.block_size = block_size;
   g_int8_next = (g_int8_next + 1) % 4;
   *out = e.maps;
   return true;
@@ -451,8 +436,8 @@ pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* 
                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                     int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
                                     pa_stream stream) {
-  if (!valid_dtype(dtype) || n_tokens < 0 || num_kv_heads < 1 || block_size < 1 ||
-      num_blocks < 0 || (head_dim != 64 && head_dim != 128))
+  if (!valid_dtype(dtype) || n_tokens < 0 || num_kv_heads < 1 || block_size < 16 ||
+      block_size % 16 || num_blocks < 0 || (head_dim != 64 && head_dim != 128))
     return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: bad sizes (n_tokens=%d "
                 "kv_heads=%d head_dim=%d block_size=%d num_blocks=%d)", n_tokens, num_kv_heads,
                 head_dim, block_size, num_blocks);
@@ -562,7 +547,7 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_cod
   a.workers = workers;
   a.scale_log2 = scale * 1.4426950408889634f;
   pa::Int8Maps maps;
-  if (!int8_maps(&maps, k_codes, v_codes, rows, block_size))
+  if (!int8_maps(&maps, k_codes, rows))
     return fail(PA_ERR_CUDA, "pa_decode_attention_int8: cuTensorMapEncodeTiled failed");
   const int per = pa::decode_int8_workers_per_cta();
   const cudaError_t e =

@@ -1,16 +1,19 @@
 // Paged decode attention on tensor cores over an INT8 cache.
 //
 // Cache ("KV Cache for intermediates..." / "The four solutions", KV-cache
-// quantisation): key codes [NB, Hkv, bs, 128] int8, value codes transposed
-// [NB, Hkv, 128, bs] int8, one fp32 scale per (block, kv head, token) for keys
-// and for values; a key or value element reads back as code * scale.
+// quantisation): key codes [NB, Hkv, bs, 128] int8, value codes transposed in
+// 16-token groups [NB, Hkv, bs / 16, 128, 16] int8, one fp32 scale per (block,
+// kv head, token) for keys and for values; an element reads back as
+// code * scale.
 //
 // Stage (16 tokens of one block and kv head, 4224 bytes):
 //  * keys: 16 rows of 128 bytes, loaded as two TMA boxes of 8 rows.  The box
 //    of tokens {4i, 4i+1} lands in lines 0..7 and the box of tokens
 //    {4i+2, 4i+3} in lines 8..15, 128-byte swizzled, so line r holds token
 //    tau(r) = 4 (r mod 8 >> 1) + (r & 1) + 2 (r >= 8);
-//  * values: 128 rows (one per head_dim index) of the stage's 16 token bytes;
+//  * values: the group's contiguous 128 x 16-byte tile (one row per head_dim
+//    index), one bulk copy of 2 KB (as 128 TMA rows of 16 bytes it would cost
+//    the copy engine far more requests per byte);
 //  * the 16 key scales and 16 value scales (two bulk copies of 64 bytes).
 // Products.  The rows of S^T = K . Q^T follow the key lines, so S^T row r is
 // token tau(r).  The contraction index of the first product is reordered so
@@ -78,15 +81,6 @@ __device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int
       : "memory");
 }
 
-__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                       uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
   asm volatile(
@@ -127,7 +121,6 @@ struct Tiles8 {
   __device__ static void prefetch(const Maps& m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_lo)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_hi)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.v)) : "memory");
   }
   __device__ static uint32_t ktile(uint32_t ring0, int i) { return ring0 + i * kKBytes; }
   __device__ static uint32_t vtile(uint32_t ring0, int i) {
@@ -144,7 +137,9 @@ struct Tiles8 {
     const uint32_t kd = ktile(ring0, i);
     tma_3d(kd, &m.k_lo, 0, 0, row >> 2, bar);
     tma_3d(kd + 1024, &m.k_hi, 0, 0, row >> 2, bar);
-    tma_2d(vtile(ring0, i), &m.v, tok, tile * D, bar);
+    const int8_t* vsrc = static_cast<const int8_t*>(a.v_cache) +
+                         (static_cast<int64_t>(tile) * (a.block_size / kTok) + tok / kTok) * kVBytes;
+    bulk_copy(vtile(ring0, i), vsrc, kVBytes, bar);
     const uint32_t sd = stile(ring0, i);
     bulk_copy(sd, a.k_scales + row, kTok * 4, bar);
     bulk_copy(sd + kTok * 4, a.v_scales + row, kTok * 4, bar);

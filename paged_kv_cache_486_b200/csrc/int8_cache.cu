@@ -7,7 +7,8 @@
 //   amax = max_d |x_d|,  scale = amax / 127,
 //   code_d = round-to-nearest-even(x_d / scale) clamped to [-127, 127]
 // (a zero row has scale 0 and zero codes).  Key codes [NB, Hkv, bs, D], value
-// codes transposed [NB, Hkv, D, bs] (so a decode lane's 4 value bytes are 4
+// codes transposed in groups of 16 tokens [NB, Hkv, bs / 16, D, 16] (one group
+// is a contiguous D x 16 tile, and a decode lane's 4 value bytes are 4
 // consecutive tokens), fp32 scales [NB, Hkv, bs] for each.
 #include <cuda_runtime.h>
 
@@ -70,7 +71,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_int8_kernel(
       if (lane == 0) k_scales[tile * block_size + off] = scale;
     } else {
 #pragma unroll
-      for (int i = 0; i < PER; ++i) v_codes[(tile * D + lane * PER + i) * block_size + off] = c[i];
+      for (int i = 0; i < PER; ++i)
+        v_codes[((tile * (block_size / 16) + off / 16) * D + lane * PER + i) * 16 + off % 16] = c[i];
       if (lane == 0) v_scales[tile * block_size + off] = scale;
     }
   }

@@ -21,15 +21,15 @@ struct Int8WriteArgs {
   int32_t* dev_error;
 };
 
-// head_dim 64 or 128; key / value in `dtype` (f32, f16, bf16).
+// head_dim 64 or 128, block_size a multiple of 16; key / value in `dtype`.
 cudaError_t launch_reshape_and_cache_int8(const Int8WriteArgs& a, pa_dtype dtype,
                                           cudaStream_t stream);
 
 // Tensor maps of an INT8 cache (see decode_int8.cu): k_lo / k_hi view the key
-// codes as rows of 128 bytes grouped by 4 tokens (k_hi starts 2 rows later);
-// v views the transposed value codes as rows of block_size bytes.
+// codes as rows of 128 bytes grouped by 4 tokens (k_hi starts 2 rows later).
+// Value tiles are contiguous and need no map.
 struct Int8Maps {
-  CUtensorMap k_lo, k_hi, v;
+  CUtensorMap k_lo, k_hi;
 };
 
 // fp16 / bf16 queries, head_dim 128, group <= 8, block_size a multiple of 16.

@@ -93,8 +93,9 @@ class PagedKVCache:
 
 class PagedKVCacheInt8(PagedKVCache):
     """The same pool and call order over an INT8 cache: codes + per-token fp32 scales
-    (key codes [NB, Hkv, bs, D], value codes transposed [NB, Hkv, D, bs], scales
-    [NB, Hkv, bs]).  key / value / q stay in `dtype`; head_dim 128 for decode."""
+    (key codes [NB, Hkv, bs, D], value codes transposed in 16-token groups
+    [NB, Hkv, bs/16, D, 16], scales [NB, Hkv, bs]).  key / value / q stay in `dtype`;
+    block_size a multiple of 16; head_dim 128 for decode."""
 
     def __init__(self, num_blocks, block_size, num_kv_heads, head_dim, dtype, num_q_heads,
                  max_batch, device="cuda", fill_bits=None):
@@ -105,7 +106,9 @@ class PagedKVCacheInt8(PagedKVCache):
         dev = self.device
         self.k_codes = torch.empty((num_blocks, num_kv_heads, block_size, head_dim),
                                    dtype=torch.int8, device=dev)
-        self.v_codes = torch.empty((num_blocks, num_kv_heads, head_dim, block_size),
+        if block_size % 16:
+            raise ValueError("an INT8 cache needs block_size a multiple of 16")
+        self.v_codes = torch.empty((num_blocks, num_kv_heads, block_size // 16, head_dim, 16),
                                    dtype=torch.int8, device=dev)
         self.k_scales = torch.empty((num_blocks, num_kv_heads, block_size), dtype=torch.float32,
                                     device=dev)

@@ -95,6 +95,6 @@ def gathered_int8(eng, bt, ctx, b, kvh):
     blk = bt[b].long()[pos // bs]
     off = pos % bs
     # per-head views first, so each gather has one advanced-index pattern
-    kc, vc = eng.k_codes[:, kvh], eng.v_codes[:, kvh]  # [NB, bs, D], [NB, D, bs]
-    return (kc[blk, off, :], vc[blk, :, off], eng.k_scales[:, kvh][blk, off],
+    kc, vc = eng.k_codes[:, kvh], eng.v_codes[:, kvh]  # [NB, bs, D], [NB, bs/16, D, 16]
+    return (kc[blk, off, :], vc[blk, off // 16, :, off % 16], eng.k_scales[:, kvh][blk, off],
             eng.v_scales[:, kvh][blk, off])

@@ -51,7 +51,7 @@ def _check_cache(wl, g, o):
             kc, vc, ks, vs = (t.cpu().numpy() for t in gathered_int8(g["eng"], g["bt"],
                                                                      g["ctx"], b, h))
             assert np.array_equal(kc, cache.k[blk, h, off, :])
-            assert np.array_equal(vc, cache.v[:, h][blk, :, off])
+            assert np.array_equal(vc, cache.v[:, h][blk, off // 16, :, off % 16])
             assert np.array_equal(ks.view(np.uint32), cache.ks[blk, h, off].view(np.uint32))
             assert np.array_equal(vs.view(np.uint32), cache.vs[blk, h, off].view(np.uint32))
 
