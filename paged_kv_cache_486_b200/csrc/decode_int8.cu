@@ -25,10 +25,10 @@
 // values exactly (|code| <= 127) by integer bit tricks, then every product is
 // the same mma as in the 16-bit path.
 // Scales.  Key scales multiply the score rows (with scale * log2 e).  Value
-// scales are folded into P: p'_j = p_j * vs_j / sigma with sigma the running
-// maximum of the segment's value scales (p' in [0, 1] whatever the scales'
-// magnitude; O is rescaled when sigma grows, and the output is O * sigma).
-// The softmax sum l keeps the unscaled p.
+// scales are folded into P: p'_j = p_j * vs_j / sigma with sigma a lazily
+// updated running maximum of the segment's value scales (p' stays within a
+// fixed range whatever the scales' magnitude; O is rescaled when sigma moves,
+// and the output is O * sigma).  The softmax sum l keeps the unscaled p.
 //
 // Roofline.  Per context token and KV head the kernel must read 128 + 128 bytes
 // of codes and 4 + 4 bytes of scales: 264 bytes against 512 for fp16.
@@ -199,11 +199,13 @@ struct Tiles8 {
     const int tk = row_token(lane >> 2);
     const float w0 = tk < n_valid ? f.vs0 : 0.f;
     const float w1 = tk + 2 < n_valid ? f.vs1 : 0.f;
-    // the stage's largest value scale: the same in every lane
-    float mx = fmaxf(w0, w1);
+    // Lazy normaliser: sigma moves only when a value scale exceeds 16 sigma
+    // (then to the stage's largest scale, the same in every lane), so
+    // vs / sigma <= 16 and p' = p vs / sigma <= 2^12, well inside fp16.
+    if (__any_sync(kFull, fmaxf(w0, w1) > seg.sig * 16.f)) {
+      float mx = fmaxf(w0, w1);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-    if (mx > seg.sig) {
+      for (int off = 4; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
       const float r = seg.sig / mx;
 #pragma unroll
       for (int mt = 0; mt < KC; ++mt) {

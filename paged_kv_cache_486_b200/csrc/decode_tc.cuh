@@ -48,6 +48,7 @@ namespace tc {
 constexpr int kTok = 16;     // tokens per stage (one mma tile of keys)
 constexpr int kWarps = 8;    // workers per CTA
 constexpr unsigned kFull = 0xffffffffu;
+constexpr float kSlack = 8.f;  // base-2 units a score may exceed the softmax reference
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -430,17 +431,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       // units, -inf past the context
       float t[4];
       P::scores(fr, qf, a, n_valid, lane, t);
+      // Lazy running maximum: weights are taken against the current reference m
+      // unless some score of the stage is more than kSlack above it (then the
+      // stage's maximum is reduced across the warp and the sums are rescaled).
+      // Weights stay <= 2^kSlack; l and o share m, so the result is unchanged.
       float x0 = fmaxf(t[0], t[2]), x1 = fmaxf(t[1], t[3]);
+      if (__any_sync(kFull, x0 > m0 + kSlack || x1 > m1 + kSlack)) {
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, off));
-        x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, off));
-      }
-      const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-      const float p[4] = {exp2f(t[0] - n0), exp2f(t[1] - n1), exp2f(t[2] - n0),
-                          exp2f(t[3] - n1)};
-      // rescale the running sums only when some head's maximum moved
-      if (__any_sync(kFull, n0 > m0 || n1 > m1)) {
+        for (int off = 4; off < 32; off <<= 1) {
+          x0 = fmaxf(x0, __shfl_xor_sync(kFull, x0, off));
+          x1 = fmaxf(x1, __shfl_xor_sync(kFull, x1, off));
+        }
+        const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
         const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
         l0 *= a0;
         l1 *= a1;
@@ -454,6 +456,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         m0 = n0;
         m1 = n1;
       }
+      const float p[4] = {exp2f(t[0] - m0), exp2f(t[1] - m1), exp2f(t[2] - m0),
+                          exp2f(t[3] - m1)};
       l0 += p[0] + p[2];
       l1 += p[1] + p[3];
       P::pv(fr, p, o, seg, n_valid, lane);
