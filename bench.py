@@ -464,8 +464,7 @@ def run_int8(args, dist, rank, world):
 
     def step():
         if n_pairs:
-            pa.pa_copy_blocks([eng.k_codes], [eng.v_codes], pairs, eng.dev_error)
-            pa.pa_copy_blocks([eng.k_scales], [eng.v_scales], pairs, eng.dev_error)
+            pa.pa_copy_blocks([eng.k_pool], [eng.v_pool], pairs, eng.dev_error)
         eng.write(key, value, slots)
         decode(pa.PA_DECODE_OVERLAP_PROLOGUE)
 
@@ -517,7 +516,7 @@ def run_int8(args, dist, rank, world):
     dec_ms = statistics.mean(decode_ms)
     achieved = alg / (dec_ms / 1e3) / 1e9
     peak, peak_kind = _peak_hbm()
-    launches = 2 + (2 if n_pairs else 0)
+    launches = 2 + (1 if n_pairs else 0)
     return {
         "metric": METRIC + " (INT8 KV cache)", "op": "int8", "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -212,7 +212,8 @@ pa_status pa_swap_blocks(void* const* dst_k_host, void* const* dst_v_host,
  *   nearest even, from fp32 accumulators.
  * block_tables: [batch, max_blocks] int32, device; context_lens: [batch] int32.
  * head_dim in {64, 128}; block_size in {8, 16, 32, 64, 128}; batch <= 4096;
- * batch * num_kv_heads <= 262144; num_blocks * num_kv_heads * block_size < 2^31.
+ * num_kv_heads <= 4096; batch * num_kv_heads <= 262144;
+ * num_blocks * num_kv_heads * block_size < 2^31; num_kv_heads * max_blocks < 2^31.
  * workspace: device scratch of at least pa_decode_workspace_size(...) bytes,
  *   16-byte aligned, zero-filled once before its first use (e.g. cudaMemset);
  *   every call that completes leaves it zero-filled again, so it is reused
@@ -299,26 +300,35 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  *   amax = max_d |x_d|,  scale = amax / 127,
  *   code_d = round-half-to-even(x_d / scale) clamped to [-127, 127]
  * (a row of zeros has scale 0 and zero codes); an element reads back as
- * code * scale.  Layout per layer:
- *   k_codes  [num_blocks, num_kv_heads, block_size, head_dim] int8
- *   v_codes  [num_blocks, num_kv_heads, block_size / 16, head_dim, 16] int8
- *            (transposed in groups of 16 tokens: one group's values form a
- *            contiguous head_dim x 16 tile, one row per head_dim index)
- *   k_scales, v_scales [num_blocks, num_kv_heads, block_size] float32.
- * Block copies (copy-on-write, eviction) of an INT8 cache are pa_copy_blocks /
- * pa_swap_blocks calls on the code pools (block_bytes = num_kv_heads *
- * block_size * head_dim) and on the scale pools (num_kv_heads * block_size * 4).
+ * code * scale.  head_dim is 128 and block_size a multiple of 16.
+ *
+ * Layout: per layer a key pool and a value pool, each
+ * [num_blocks, num_kv_heads, block_size / 16] records of 2112 bytes, one record
+ * per 16-token group of a (block, kv head) (so a pool is
+ * pa_int8_block_bytes(...) bytes per block):
+ *   key record:   16 lines of 128 signed code bytes, then 16 fp32 key scales
+ *                 (token order).  Group token t = 4i + 2h + e is on line
+ *                 L = 2i + e + 8h; the codes of head_dim 16c .. 16c + 15 sit at
+ *                 bytes L * 128 + 16 (c xor (L mod 8)) .. + 15.
+ *   value record: 128 rows of 16 signed code bytes (row d: head_dim d of
+ *                 tokens 0 .. 15 in token order), then 16 fp32 value scales.
+ * Each record is what the decode kernel keeps in shared memory for one stage,
+ * so one bulk copy moves it.  Block copies (copy-on-write, eviction) of an
+ * INT8 cache are pa_copy_blocks / pa_swap_blocks on the two pools with
+ * block_bytes = pa_int8_block_bytes(...).
  * ---------------------------------------------------------------------- */
+
+/* Bytes of one block of one INT8 pool (0 if the shape is not supported). */
+size_t pa_int8_block_bytes(int32_t num_kv_heads, int32_t head_dim, int32_t block_size);
 
 /* Quantise new tokens into an INT8 cache: as pa_reshape_and_cache (same
  * key / value / slot_mapping arguments, `dtype` is that of key and value: f32,
  * f16 or bf16), but each (token, kv head) row is written as codes + scale by
- * the scheme above; codes and scales are bit-exact to it.  head_dim 64 or 128;
- * block_size a multiple of 16; every pointer 16-byte aligned (slot_mapping 8).  Slots outside the pool set
+ * the scheme above; codes and scales are bit-exact to it.  Pools and key /
+ * value 16-byte aligned, slot_mapping 8.  Slots outside the pool set
  * PA_DEVERR_BAD_SLOT and are skipped; -1 is skipped silently. */
-pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
-                                    int8_t* v_codes, float* k_scales, float* v_scales,
-                                    const int64_t* slot_mapping, int32_t n_tokens,
+pa_status pa_reshape_and_cache_int8(const void* key, const void* value, void* k_pool,
+                                    void* v_pool, const int64_t* slot_mapping, int32_t n_tokens,
                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                     int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
                                     pa_stream stream);
@@ -326,16 +336,14 @@ pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* 
 /* Decode attention over an INT8 cache: the definition of pa_decode_attention
  * with K_b[j, g, :] = k_code * k_scale and V_b[j, g, :] = v_code * v_scale of
  * token j.  q and out in `dtype` (f16 or bf16); head_dim 128; group
- * (num_q_heads / num_kv_heads) <= 8; block_size in {16, 32, 64, 128};
- * num_blocks * num_kv_heads * max(block_size, 128) < 2^31; code pools and
- * scale pools 16-byte aligned.  block_tables, context_lens, workspace (same
- * size, zero-once contract and reuse as pa_decode_attention), dev_error, the
- * work split and flags are those of pa_decode_attention_ex; num_workers = 0
- * chooses automatically.  Runs on tensor cores: codes are converted exactly
- * to fp16 / bf16, products accumulate in fp32, out is rounded once. */
-pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_codes,
-                                   const int8_t* v_codes, const float* k_scales,
-                                   const float* v_scales, const int32_t* block_tables,
+ * (num_q_heads / num_kv_heads) <= 8; block_size in {16, 32, 64, 128}; pools
+ * 16-byte aligned.  block_tables, context_lens, workspace (same size, zero-once
+ * contract and reuse as pa_decode_attention), dev_error, the work split and
+ * flags are those of pa_decode_attention_ex; num_workers = 0 chooses
+ * automatically.  Runs on tensor cores: codes are converted exactly to fp16 /
+ * bf16, products accumulate in fp32, out is rounded once. */
+pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* block_tables,
                                    const int32_t* context_lens, int32_t batch,
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                    int32_t block_size, int32_t num_blocks, int32_t max_blocks,

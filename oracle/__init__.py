@@ -258,13 +258,12 @@ def contiguous_attention(q, k, v, scale, dtype, heads=None):
 
 # ------------------------------------------------------------- INT8 cache
 class Int8Cache:
-    """Host INT8 cache: key codes [NB, Hkv, bs, D], value codes transposed in
-    groups of 16 tokens [NB, Hkv, bs/16, D, 16], fp32 scales [NB, Hkv, bs] for keys
-    and values (bs a multiple of 16)."""
+    """Host INT8 cache in its logical layout: key codes and value codes
+    [NB, Hkv, bs, D], fp32 scales [NB, Hkv, bs] for keys and values."""
 
     def __init__(self, num_blocks, kv_heads, block_size, head_dim):
         self.k = np.zeros((num_blocks, kv_heads, block_size, head_dim), np.int8)
-        self.v = np.zeros((num_blocks, kv_heads, block_size // 16, head_dim, 16), np.int8)
+        self.v = np.zeros((num_blocks, kv_heads, block_size, head_dim), np.int8)
         self.ks = np.zeros((num_blocks, kv_heads, block_size), np.float32)
         self.vs = np.zeros((num_blocks, kv_heads, block_size), np.float32)
 

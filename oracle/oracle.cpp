@@ -441,17 +441,14 @@ static void quantize_row(const void* src, int64_t base, int32_t D, int dtype, in
   *scale_out = scale;
 }
 
-// Write new tokens into an INT8 cache.  Key codes [NB, Hkv, bs, D]; value codes
-// transposed in groups of 16 tokens, [NB, Hkv, bs / 16, D, 16] (so one group's
-// values for every head_dim index are one contiguous tile); scales
-// [NB, Hkv, bs] (fp32) for each.  block_size must be a multiple of 16.
+// Write new tokens into an INT8 cache, kept here in its logical layout: key
+// codes and value codes [NB, Hkv, bs, D], scales [NB, Hkv, bs] (fp32) for each.
 int orc_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
                                int8_t* v_codes, float* k_scales, float* v_scales,
                                const int64_t* slots, int64_t n_tokens, int32_t kv_heads,
                                int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                int dtype) {
   const int32_t D = head_dim;
-  if (block_size % 16 != 0) return ORC_INVALID;
   std::vector<int8_t> row(D);
   for (int64_t t = 0; t < n_tokens; ++t) {
     const int64_t slot = slots[t];
@@ -466,8 +463,7 @@ int orc_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_cod
       for (int32_t d = 0; d < D; ++d) k_codes[(tile * block_size + off) * D + d] = row[d];
       k_scales[tile * block_size + off] = sc;
       quantize_row(value, src, D, dtype, row.data(), &sc);
-      const int64_t group = tile * (block_size / 16) + off / 16;
-      for (int32_t d = 0; d < D; ++d) v_codes[(group * D + d) * 16 + off % 16] = row[d];
+      for (int32_t d = 0; d < D; ++d) v_codes[(tile * block_size + off) * D + d] = row[d];
       v_scales[tile * block_size + off] = sc;
     }
   }
@@ -588,7 +584,7 @@ int orc_paged_decode_attention_int8(const void* q, const int8_t* k_codes, const 
                                     int32_t block_size, int32_t max_blocks, double scale,
                                     int dtype, double* out, const int64_t* rows, int64_t n_rows,
                                     int32_t n_threads) {
-  if (kv_heads <= 0 || q_heads % kv_heads != 0 || block_size % 16 != 0) return ORC_INVALID;
+  if (kv_heads <= 0 || q_heads % kv_heads != 0) return ORC_INVALID;
   const int32_t group = q_heads / kv_heads, D = head_dim, bs = block_size;
   const int64_t total = rows ? n_rows : static_cast<int64_t>(batch) * q_heads;
   auto one = [&](int64_t row) {
@@ -604,7 +600,7 @@ int orc_paged_decode_attention_int8(const void* q, const int8_t* k_codes, const 
       const double ks = k_scales[tile * bs + off], vs = v_scales[tile * bs + off];
       for (int32_t d = 0; d < D; ++d) {
         kk[j * D + d] = ks * k_codes[(tile * bs + off) * D + d];
-        vv[j * D + d] = vs * v_codes[((tile * (bs / 16) + off / 16) * D + d) * 16 + off % 16];
+        vv[j * D + d] = vs * v_codes[(tile * bs + off) * D + d];
       }
     }
     attend_one(qq.data(), kk.data(), vv.data(), n, D, scale, out + row * D);

@@ -55,11 +55,12 @@ SIGNATURES = {
                                       _I32, _I32, _P]),
     "pa_decode_attention_static_ws": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                              _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
-    "pa_reshape_and_cache_int8": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
-                                         _I32, C.c_int, _P, _P]),
-    "pa_decode_attention_int8": (_I32, [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
-                                        _I32, _I32, _I32, C.c_float, C.c_int, _P, C.c_size_t, _P,
-                                        _I32, _I32, _P]),
+    "pa_int8_block_bytes": (C.c_size_t, [_I32, _I32, _I32]),
+    "pa_reshape_and_cache_int8": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                         C.c_int, _P, _P]),
+    "pa_decode_attention_int8": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                        _I32, _I32, C.c_float, C.c_int, _P, C.c_size_t, _P, _I32,
+                                        _I32, _P]),
     "pa_decode_plan": (_I32, [_I32, _I32, _I32, _I32, _I32, C.c_int, _P, _P]),
     "pa_validate_slot_mapping": (_I32, [_P, _I32, _I32, _I32]),
     "pa_validate_block_table": (_I32, [_P, _P, _I32, _I32, _I32, _I32]),
@@ -304,42 +305,44 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, contex
     _check(st, "pa_decode_attention_static_ws")
 
 
-def pa_reshape_and_cache_int8(key, value, k_codes, v_codes, k_scales, v_scales, slot_mapping,
-                              dev_error=None, stream=None):
-    """Quantise key/value [T, Hkv, D] into an INT8 cache: k_codes int8 [NB, Hkv, bs, D],
-    v_codes int8 [NB, Hkv, bs/16, D, 16], k_scales / v_scales float32 [NB, Hkv, bs]
-    (all CUDA)."""
+INT8_RECORD_BYTES = 2112  # one 16-token group of one (block, kv head): codes + fp32 scales
+
+
+def pa_int8_block_bytes(num_kv_heads, head_dim, block_size) -> int:
+    return int(lib.pa_int8_block_bytes(num_kv_heads, head_dim, block_size))
+
+
+def pa_reshape_and_cache_int8(key, value, k_pool, v_pool, slot_mapping, dev_error=None,
+                              stream=None):
+    """Quantise key/value [T, Hkv, 128] into an INT8 cache: k_pool / v_pool uint8
+    [NB, Hkv, bs/16, 2112] records (layout in include/pa.h)."""
     T, Hkv, D = key.shape
-    NB, Hkv2, bs, D2 = k_codes.shape
-    if ((Hkv, D) != (Hkv2, D2) or value.shape != key.shape
-            or tuple(v_codes.shape) != (NB, Hkv, bs // 16, D, 16)
-            or tuple(k_scales.shape) != (NB, Hkv, bs) or v_scales.shape != k_scales.shape):
-        raise ValueError("shape mismatch between key/value and the INT8 cache")
+    NB, Hkv2, G16, R = k_pool.shape
+    if (Hkv != Hkv2 or value.shape != key.shape or v_pool.shape != k_pool.shape
+            or R != INT8_RECORD_BYTES):
+        raise ValueError("shape mismatch between key/value and the INT8 pools")
     st = lib.pa_reshape_and_cache_int8(
         _dev_ptr(key, "key"), _dev_ptr(value, "value", key.dtype),
-        _dev_ptr(k_codes, "k_codes", torch.int8), _dev_ptr(v_codes, "v_codes", torch.int8),
-        _dev_ptr(k_scales, "k_scales", torch.float32), _dev_ptr(v_scales, "v_scales", torch.float32),
-        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, bs, NB,
+        _dev_ptr(k_pool, "k_pool", torch.uint8), _dev_ptr(v_pool, "v_pool", torch.uint8),
+        _dev_ptr(slot_mapping, "slot_mapping", torch.int64), T, Hkv, D, 16 * G16, NB,
         DTYPE_CODE[key.dtype], _dev_ptr(dev_error, "dev_error", torch.int32), _stream(stream))
     _check(st, "pa_reshape_and_cache_int8")
 
 
-def pa_decode_attention_int8(out, q, k_codes, v_codes, k_scales, v_scales, block_tables,
-                             context_lens, scale, workspace, dev_error=None, num_workers=0,
-                             flags=0, stream=None):
-    """Decode attention over an INT8 cache (layout as pa_reshape_and_cache_int8); q/out
+def pa_decode_attention_int8(out, q, k_pool, v_pool, block_tables, context_lens, scale,
+                             workspace, dev_error=None, num_workers=0, flags=0, stream=None):
+    """Decode attention over an INT8 cache (pools as pa_reshape_and_cache_int8); q/out
     [B, Hq, 128] fp16 or bf16; the other arguments as pa_decode_attention."""
     B, Hq, D = q.shape
-    NB, Hkv, bs, _ = k_codes.shape
+    NB, Hkv, G16, _ = k_pool.shape
     MB = block_tables.shape[1]
     if out.shape != q.shape:
         raise ValueError("out must have q's shape")
     st = lib.pa_decode_attention_int8(
-        _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_codes, "k_codes", torch.int8),
-        _dev_ptr(v_codes, "v_codes", torch.int8), _dev_ptr(k_scales, "k_scales", torch.float32),
-        _dev_ptr(v_scales, "v_scales", torch.float32),
+        _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_pool, "k_pool", torch.uint8),
+        _dev_ptr(v_pool, "v_pool", torch.uint8),
         _dev_ptr(block_tables, "block_tables", torch.int32),
-        _dev_ptr(context_lens, "context_lens", torch.int32), B, Hq, Hkv, D, bs, NB, MB,
+        _dev_ptr(context_lens, "context_lens", torch.int32), B, Hq, Hkv, D, 16 * G16, NB, MB,
         float(scale), DTYPE_CODE[q.dtype], _dev_ptr(workspace, "workspace"),
         workspace.numel() * workspace.element_size(),
         _dev_ptr(dev_error, "dev_error", torch.int32), num_workers, flags, _stream(stream))

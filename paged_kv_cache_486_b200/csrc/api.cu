@@ -56,21 +56,40 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// A pool [num_blocks, Hkv, bs, D] seen as `rows` rows of D elements; one box is
-// 16 rows x 64 columns (128 bytes, the 128-byte swizzle span).
-bool make_tile_map(CUtensorMap* map, const void* base, int64_t rows, int head_dim, pa_dtype dt) {
+// A pool [num_blocks, Hkv, bs, D] seen as `rows` rows of D elements.  Preferred
+// form (three_d): {64 columns, rows, D / 64 column blocks} with strides D * 2
+// (row) and 128 bytes (column block), box {64, 16, D / 64}: one copy lands a
+// whole 16-row tile as D / 64 column blocks of 16 lines x 128 bytes.  If the
+// driver declines that map, {D, rows} with box {64, 16}, one copy per block.
+bool make_tile_map(CUtensorMap* map, bool* three_d, const void* base, int64_t rows,
+                   int head_dim, pa_dtype dt) {
   auto enc = encode_fn();
   if (!enc) return false;
   const CUtensorMapDataType t =
       dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (head_dim > 64) {
+    cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(head_dim / 64)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, 128};
+    cuuint32_t box[3] = {64, 16, static_cast<cuuint32_t>(head_dim / 64)};
+    cuuint32_t es[3] = {1, 1, 1};
+    if (enc(map, t, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+        CUDA_SUCCESS) {
+      *three_d = true;
+      return true;
+    }
+  }
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
   cuuint32_t box[2] = {64, 16};
   cuuint32_t es[2] = {1, 1};
-  const CUresult r = enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  *three_d = false;
+  return enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 // Small per-thread cache: encoding is cheap but not free, and decode is called
@@ -80,73 +99,30 @@ struct MapEntry {
   int64_t rows;
   int head_dim;
   int dtype;
+  bool three_d;
   CUtensorMap map;
 };
 thread_local MapEntry g_maps[8];
 thread_local int g_maps_next = 0;
 
-bool tile_map(CUtensorMap* out, const void* base, int64_t rows, int head_dim, pa_dtype dt) {
+bool tile_map(CUtensorMap* out, bool* three_d, const void* base, int64_t rows, int head_dim,
+              pa_dtype dt) {
   for (auto& e : g_maps) {
     if (e.base == base && e.rows == rows && e.head_dim == head_dim && e.dtype == dt) {
       *out = e.map;
+      *three_d = e.three_d;
       return true;
     }
   }
   MapEntry& e = g_maps[g_maps_next];
-  if (!make_tile_map(&e.map, base, rows, head_dim, dt)) return false;
+  if (!make_tile_map(&e.map, &e.three_d, base, rows, head_dim, dt)) return false;
   e.base = base;
   e.rows = rows;
   e.head_dim = head_dim;
   e.dtype = dt;
   g_maps_next = (g_maps_next + 1) % 8;
   *out = e.map;
-  return true;
-}
-
-// INT8 cache maps.  Keys [rows = NB * Hkv * bs, 128] bytes are seen as
-// [rows / 4][2][128] (groups of 4 tokens, 2 tokens, bytes) with strides 512 and
-// 128: a box {128, 2, 4} is tokens {4i, 4i + 1} of 4 consecutive groups.  k_hi
-// starts 256 bytes (2 tokens) later, so its boxes are tokens {4i + 2, 4i + 3}.
-bool make_int8_maps(pa::Int8Maps* m, const void* k_codes, int64_t rows) {
-  auto enc = encode_fn();
-  if (!enc) return false;
-  cuuint64_t kd[3] = {128, 2, static_cast<cuuint64_t>(rows / 4)};
-  cuuint64_t ks[2] = {128, 512};
-  cuuint32_t kb[3] = {128, 2, 4};
-  cuuint32_t e3[3] = {1, 1, 1};
-  const char* kbase = static_cast<const char*>(k_codes);
-  for (int half = 0; half < 2; ++half) {
-    CUtensorMap* out = half ? &m->k_hi : &m->k_lo;
-    const CUresult r = enc(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
-                           const_cast<char*>(kbase + 256 * half), kd, ks, kb, e3,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return false;
-  }
-  return true;
-}
-
-struct Int8MapEntry {
-  const void* k;
-  int64_t rows;
-  pa::Int8Maps maps;
-};
-thread_local Int8MapEntry g_int8_maps[4];
-thread_local int g_int8_next = 0;
-
-bool int8_maps(pa::Int8Maps* out, const void* k, int64_t rows) {
-  for (auto& e : g_int8_maps) {
-    if (e.k == k && e.rows == rows) {
-      *out = e.maps;
-      return true;
-    }
-  }
-  Int8MapEntry& e = g_int8_maps[g_int8_next];
-  if (!make_int8_maps(&e.maps, k, rows)) return false;
-  e.k = k;
-  e.rows = rows;
-  g_int8_next = (g_int8_next + 1) % 4;
-  *out = e.maps;
+  *three_d = e.three_d;
   return true;
 }
 
@@ -328,9 +304,10 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   if (batch < 0 || batch > pa::kMaxBatch)
     return fail(PA_ERR_INVALID, "pa_decode_attention: batch %d outside [0, %d]", batch,
                 pa::kMaxBatch);
-  if (num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads)
+  if (num_kv_heads < 1 || num_kv_heads > pa::kMaxKvHeads || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads)
     return fail(PA_ERR_INVALID, "pa_decode_attention: num_q_heads %d not a multiple of "
-                "num_kv_heads %d", num_q_heads, num_kv_heads);
+                "num_kv_heads %d (at most %d)", num_q_heads, num_kv_heads, pa::kMaxKvHeads);
   if (head_dim != 64 && head_dim != 128)
     return fail(PA_ERR_INVALID, "pa_decode_attention: head_dim %d not in {64, 128}", head_dim);
   if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
@@ -343,6 +320,8 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   if (rows >= (int64_t(1) << 31))
     return fail(PA_ERR_INVALID, "pa_decode_attention: num_blocks * num_kv_heads * block_size "
                 "= %lld >= 2^31", static_cast<long long>(rows));
+  if (static_cast<int64_t>(num_kv_heads) * max_blocks >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_kv_heads * max_blocks >= 2^31");
   if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention: scale is NaN");
   if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
     return fail(PA_ERR_INVALID, "pa_decode_attention: batch * num_kv_heads = %lld > %d",
@@ -382,8 +361,6 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.q = q;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
-  a.k_scales = nullptr;
-  a.v_scales = nullptr;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.dev_error = dev_error;
@@ -405,11 +382,13 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   cudaError_t e;
   if (use_tc) {
     CUtensorMap kmap, vmap;
-    if (!tile_map(&kmap, k_cache, rows, head_dim, dtype) ||
-        !tile_map(&vmap, v_cache, rows, head_dim, dtype))
+    bool k3 = false, v3 = false;
+    if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
+        !tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype))
       return fail(PA_ERR_CUDA, "pa_decode_attention: cuTensorMapEncodeTiled failed");
+    if (k3 != v3) return fail(PA_ERR_CUDA, "pa_decode_attention: inconsistent tensor maps");
     const int per = pa::decode_tc_workers_per_cta();
-    e = pa::launch_decode_tc(a, dtype, kmap, vmap, (workers + per - 1) / per, overlap,
+    e = pa::launch_decode_tc(a, dtype, kmap, vmap, k3, (workers + per - 1) / per, overlap,
                              static_cast<cudaStream_t>(stream));
   } else {
     e = pa::launch_decode_simt(a, dtype, overlap, static_cast<cudaStream_t>(stream));
@@ -430,35 +409,31 @@ pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, con
                                 PA_PATH_AUTO, 0, 0, stream);
 }
 
-pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* k_codes,
-                                    int8_t* v_codes, float* k_scales, float* v_scales,
-                                    const int64_t* slot_mapping, int32_t n_tokens,
+pa_status pa_reshape_and_cache_int8(const void* key, const void* value, void* k_pool,
+                                    void* v_pool, const int64_t* slot_mapping, int32_t n_tokens,
                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                     int32_t num_blocks, pa_dtype dtype, int32_t* dev_error,
                                     pa_stream stream) {
   if (!valid_dtype(dtype) || n_tokens < 0 || num_kv_heads < 1 || block_size < 16 ||
-      block_size % 16 || num_blocks < 0 || (head_dim != 64 && head_dim != 128))
+      block_size % 16 || num_blocks < 0 || head_dim != pa::i8::kDim)
     return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: bad sizes (n_tokens=%d "
-                "kv_heads=%d head_dim=%d block_size=%d num_blocks=%d)", n_tokens, num_kv_heads,
-                head_dim, block_size, num_blocks);
+                "kv_heads=%d head_dim=%d block_size=%d num_blocks=%d; head_dim must be 128 and "
+                "block_size a multiple of 16)", n_tokens, num_kv_heads, head_dim, block_size,
+                num_blocks);
   if (n_tokens == 0) return PA_OK;
-  if (!key || !value || !k_codes || !v_codes || !k_scales || !v_scales || !slot_mapping)
+  if (!key || !value || !k_pool || !v_pool || !slot_mapping)
     return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: NULL pointer");
-  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_codes, 16) ||
-      !aligned(v_codes, 16) || !aligned(k_scales, 16) || !aligned(v_scales, 16) ||
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
       !aligned(slot_mapping, 8))
     return fail(PA_ERR_INVALID, "pa_reshape_and_cache_int8: misaligned pointer");
   pa::Int8WriteArgs a;
   a.key = key;
   a.value = value;
-  a.k_codes = k_codes;
-  a.v_codes = v_codes;
-  a.k_scales = k_scales;
-  a.v_scales = v_scales;
+  a.k_pool = static_cast<uint8_t*>(k_pool);
+  a.v_pool = static_cast<uint8_t*>(v_pool);
   a.slots = slot_mapping;
   a.n_tokens = n_tokens;
   a.num_kv_heads = num_kv_heads;
-  a.head_dim = head_dim;
   a.block_size = block_size;
   a.num_blocks = num_blocks;
   a.dev_error = dev_error;
@@ -467,9 +442,15 @@ pa_status pa_reshape_and_cache_int8(const void* key, const void* value, int8_t* 
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_reshape_and_cache_int8");
 }
 
-pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_codes,
-                                   const int8_t* v_codes, const float* k_scales,
-                                   const float* v_scales, const int32_t* block_tables,
+size_t pa_int8_block_bytes(int32_t num_kv_heads, int32_t head_dim, int32_t block_size) {
+  if (num_kv_heads < 1 || head_dim != pa::i8::kDim || block_size < 16 || block_size % 16)
+    return 0;
+  return static_cast<size_t>(num_kv_heads) * (block_size / pa::i8::kGroup) *
+         pa::i8::kRecordBytes;
+}
+
+pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* block_tables,
                                    const int32_t* context_lens, int32_t batch,
                                    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                    int32_t block_size, int32_t num_blocks, int32_t max_blocks,
@@ -481,22 +462,21 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_cod
   if (batch < 0 || batch > pa::kMaxBatch)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: batch %d outside [0, %d]", batch,
                 pa::kMaxBatch);
-  if (num_kv_heads < 1 || num_q_heads < num_kv_heads || num_q_heads % num_kv_heads ||
-      num_q_heads / num_kv_heads > 8)
+  if (num_kv_heads < 1 || num_kv_heads > pa::kMaxKvHeads || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads || num_q_heads / num_kv_heads > 8)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: num_q_heads %d must be 1..8 times "
-                "num_kv_heads %d", num_q_heads, num_kv_heads);
-  if (head_dim != 128)
+                "num_kv_heads %d (at most %d)", num_q_heads, num_kv_heads, pa::kMaxKvHeads);
+  if (head_dim != pa::i8::kDim)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: head_dim %d is not 128", head_dim);
   if (block_size != 16 && block_size != 32 && block_size != 64 && block_size != 128)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: block_size %d not in "
                 "{16, 32, 64, 128}", block_size);
   if (num_blocks < 0 || max_blocks < 0)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: negative num_blocks or max_blocks");
-  const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
-  if (static_cast<int64_t>(num_blocks) * num_kv_heads * 128 >= (int64_t(1) << 31) ||
-      rows >= (int64_t(1) << 31))
+  if (static_cast<int64_t>(num_blocks) * num_kv_heads * block_size >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(num_kv_heads) * max_blocks >= (int64_t(1) << 31))
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: num_blocks * num_kv_heads * "
-                "max(block_size, 128) >= 2^31");
+                "block_size or num_kv_heads * max_blocks >= 2^31");
   if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention_int8: scale is NaN");
   if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: batch * num_kv_heads > %d",
@@ -504,14 +484,10 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_cod
   if (flags & ~PA_DECODE_OVERLAP_PROLOGUE)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: unknown flags 0x%x", flags);
   if (batch == 0) return PA_OK;
-  if (num_blocks == 0)
-    return fail(PA_ERR_INVALID, "pa_decode_attention_int8: empty pool");
-  if (!out || !q || !k_codes || !v_codes || !k_scales || !v_scales || !block_tables ||
-      !context_lens || !workspace)
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !workspace)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: NULL pointer");
-  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_codes, 16) || !aligned(v_codes, 16) ||
-      !aligned(k_scales, 16) || !aligned(v_scales, 16) || !aligned(workspace, 16) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4))
+  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_pool, 16) || !aligned(v_pool, 16) ||
+      !aligned(workspace, 16) || !aligned(block_tables, 4) || !aligned(context_lens, 4))
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: misaligned pointer");
   const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim);
   if (workspace_bytes < need)
@@ -525,10 +501,8 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_cod
   pa::DecodeArgs a;
   a.out = out;
   a.q = q;
-  a.k_cache = k_codes;
-  a.v_cache = v_codes;
-  a.k_scales = k_scales;
-  a.v_scales = v_scales;
+  a.k_cache = k_pool;
+  a.v_cache = v_pool;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.dev_error = dev_error;
@@ -546,14 +520,10 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const int8_t* k_cod
   a.max_blocks = max_blocks;
   a.workers = workers;
   a.scale_log2 = scale * 1.4426950408889634f;
-  pa::Int8Maps maps;
-  if (!int8_maps(&maps, k_codes, rows))
-    return fail(PA_ERR_CUDA, "pa_decode_attention_int8: cuTensorMapEncodeTiled failed");
   const int per = pa::decode_int8_workers_per_cta();
-  const cudaError_t e =
-      pa::launch_decode_int8(a, dtype, maps, (workers + per - 1) / per,
-                             (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0,
-                             static_cast<cudaStream_t>(stream));
+  const cudaError_t e = pa::launch_decode_int8(a, dtype, (workers + per - 1) / per,
+                                               (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0,
+                                               static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_decode_attention_int8 (decode kernel)");
 }
 

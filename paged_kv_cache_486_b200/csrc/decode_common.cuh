@@ -41,14 +41,13 @@ constexpr int kMaxBatch = 4096;
 constexpr int kMaxWorkers = 2048;
 constexpr int kPieceHeadBudget = 16384;  // workers x G kept in the workspace
 constexpr int kMaxArrivals = 262144;     // batch x kv heads (arrival words)
+constexpr int kMaxKvHeads = 4096;        // kv heads per layer
 
 struct DecodeArgs {
   void* out;
   const void* q;
   const void* k_cache;
   const void* v_cache;
-  const float* k_scales;  // 8-bit caches: per-token scales [NB, Hkv, bs] (else unused)
-  const float* v_scales;
   const int32_t* block_tables;
   const int32_t* context_lens;
   int32_t* dev_error;

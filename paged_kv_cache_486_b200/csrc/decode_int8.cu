@@ -1,29 +1,20 @@
 // Paged decode attention on tensor cores over an INT8 cache.
 //
 // Cache ("KV Cache for intermediates..." / "The four solutions", KV-cache
-// quantisation): key codes [NB, Hkv, bs, 128] int8, value codes transposed in
-// 16-token groups [NB, Hkv, bs / 16, 128, 16] int8, one fp32 scale per (block,
-// kv head, token) for keys and for values; an element reads back as
-// code * scale.
+// quantisation): per (token, kv head) 128 signed 8-bit codes and one fp32
+// scale, for keys and for values; an element reads back as code * scale.  The
+// pools hold one record per 16-token group of a (block, kv head) (layout in
+// int8_launch.h), so a stage is two bulk copies of kRecordBytes.
 //
-// Stage (16 tokens of one block and kv head, 4224 bytes):
-//  * keys: 16 rows of 128 bytes, loaded as two TMA boxes of 8 rows.  The box
-//    of tokens {4i, 4i+1} lands in lines 0..7 and the box of tokens
-//    {4i+2, 4i+3} in lines 8..15, 128-byte swizzled, so line r holds token
-//    tau(r) = 4 (r mod 8 >> 1) + (r & 1) + 2 (r >= 8);
-//  * values: the group's contiguous 128 x 16-byte tile (one row per head_dim
-//    index), one bulk copy of 2 KB (as 128 TMA rows of 16 bytes it would cost
-//    the copy engine far more requests per byte);
-//  * the 16 key scales and 16 value scales (two bulk copies of 64 bytes).
-// Products.  The rows of S^T = K . Q^T follow the key lines, so S^T row r is
-// token tau(r).  The contraction index of the first product is reordered so
-// that a lane's four key bytes (one 32-bit ldmatrix element, d = 16kc + 4cq
-// .. +3) are its four A elements; the query fragment uses the same order.  In
-// O^T += V^T . P^T a lane's four value bytes are tokens 4cq .. 4cq+3, which is
-// exactly the token order that the register transpose of S^T rows tau(.)
-// gives the P^T fragment, so neither operand is shuffled.  Codes become 16-bit
-// values exactly (|code| <= 127) by integer bit tricks, then every product is
-// the same mma as in the 16-bit path.
+// Products.  Key record line r holds token tau(r) = key_token(r), so row r of
+// S^T = K . Q^T is token tau(r).  The contraction index of the first product
+// is reordered so that a lane's four key bytes (one 32-bit ldmatrix element,
+// d = 16kc + 4cq .. +3) are its four A elements; the query fragment uses the
+// same order.  In O^T += V^T . P^T a lane's four value bytes are tokens
+// 4cq .. 4cq+3, which is exactly the token order that the register transpose
+// of S^T rows tau(.) gives the P^T fragment, so neither operand is shuffled.
+// Codes become 16-bit values exactly (|code| <= 127) by integer bit tricks,
+// then every product is the same mma as in the 16-bit path.
 // Scales.  Key scales multiply the score rows (with scale * log2 e).  Value
 // scales are folded into P: p'_j = p_j * vs_j / sigma with sigma a lazily
 // updated running maximum of the segment's value scales (p' stays within a
@@ -72,15 +63,6 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                       uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
   asm volatile(
@@ -90,23 +72,19 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
 }
 
 // Token of S^T row g (g < 8); row g + 8 holds that token + 2.
-__device__ __forceinline__ int row_token(int g) { return 4 * (g >> 1) + (g & 1); }
+__device__ __forceinline__ int row_token(int g) { return i8::key_token(g); }
 
 template <typename T>
 struct Tiles8 {
-  static constexpr int D = 128;
+  static constexpr int D = i8::kDim;
   static constexpr int KC = D / 16;
   static constexpr int kStages = 5;
-  static constexpr int kKBytes = kTok * D;
-  static constexpr int kVBytes = kTok * D;
-  static constexpr int kSBytes = 2 * kTok * 4;
-  static constexpr int kStageBytes = kKBytes + kVBytes + kSBytes;
-  static constexpr int kSlots = kWarps * kStages;
-  // all key tiles, then all value tiles, then all scales (key tiles stay
-  // 1024-byte aligned for the swizzle)
-  static constexpr int kRingBytes = kSlots * kStageBytes;
-  static_assert(kRingBytes % 1024 == 0, "ring size");
-  using Maps = Int8Maps;
+  static constexpr int kRec = i8::kRecordBytes;
+  static constexpr int kStageBytes = 2 * kRec;  // key record + value record
+  static constexpr int kRingBytes = (kWarps * kStages * kStageBytes + 1023) / 1024 * 1024;
+  struct Maps {
+    int unused;
+  };
   struct Frag {
     uint32_t k[KC][2];  // [kc][row g, row g + 8]: 4 codes, d = 16kc + 4cq .. +3
     uint32_t v[KC][2];  // [mt][d = 16mt + g, +8]: 4 codes, tokens 4cq .. +3
@@ -118,39 +96,23 @@ struct Tiles8 {
     __device__ float out_scale() const { return sig; }
   };
 
-  __device__ static void prefetch(const Maps& m) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_lo)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k_hi)) : "memory");
+  __device__ static void prefetch(const Maps&) {}
+  __device__ static uint32_t stage(uint32_t ring0, int warp, int slot) {
+    return ring0 + (warp * kStages + slot) * kStageBytes;
   }
-  __device__ static uint32_t ktile(uint32_t ring0, int i) { return ring0 + i * kKBytes; }
-  __device__ static uint32_t vtile(uint32_t ring0, int i) {
-    return ring0 + kSlots * kKBytes + i * kVBytes;
-  }
-  __device__ static uint32_t stile(uint32_t ring0, int i) {
-    return ring0 + kSlots * (kKBytes + kVBytes) + i * kSBytes;
-  }
-
-  __device__ static void issue(const Maps& m, const DecodeArgs& a, uint32_t ring0, int warp,
+  __device__ static void issue(const Maps&, const DecodeArgs& a, uint32_t ring0, int warp,
                                int slot, int tile, int tok, uint32_t bar) {
-    const int i = warp * kStages + slot;
-    const int row = tile * a.block_size + tok;  // a multiple of 16
-    const uint32_t kd = ktile(ring0, i);
-    tma_3d(kd, &m.k_lo, 0, 0, row >> 2, bar);
-    tma_3d(kd + 1024, &m.k_hi, 0, 0, row >> 2, bar);
-    const int8_t* vsrc = static_cast<const int8_t*>(a.v_cache) +
-                         (static_cast<int64_t>(tile) * (a.block_size / kTok) + tok / kTok) * kVBytes;
-    bulk_copy(vtile(ring0, i), vsrc, kVBytes, bar);
-    const uint32_t sd = stile(ring0, i);
-    bulk_copy(sd, a.k_scales + row, kTok * 4, bar);
-    bulk_copy(sd + kTok * 4, a.v_scales + row, kTok * 4, bar);
+    const int64_t rec = static_cast<int64_t>(tile) * (a.block_size / i8::kGroup) + tok / i8::kGroup;
+    const uint32_t dst = stage(ring0, warp, slot);
+    bulk_copy(dst, static_cast<const uint8_t*>(a.k_cache) + rec * kRec, kRec, bar);
+    bulk_copy(dst + kRec, static_cast<const uint8_t*>(a.v_cache) + rec * kRec, kRec, bar);
   }
   // lane (g, cq) holds q[g][16kc + 4cq, +1] and q[g][16kc + 4cq + 2, +3]
   __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 4 * cq + 2 * half; }
 
   __device__ static void load(const DecodeArgs&, uint32_t ring0, int warp, int slot, int,
                               int lane, Frag& f) {
-    const int i = warp * kStages + slot;
-    const uint32_t kt = ktile(ring0, i), vt = vtile(ring0, i), st = stile(ring0, i);
+    const uint32_t kt = stage(ring0, warp, slot), vt = kt + kRec;
     const int mi = lane >> 3, r8 = lane & 7;
     const int line = r8 + ((mi & 1) << 3);
 #pragma unroll
@@ -168,10 +130,10 @@ struct Tiles8 {
       f.v[2 * kk + 1][1] = r[3];
     }
     const int tk = row_token(lane >> 2);
-    f.ks0 = lds_f32(st + 4 * tk);
-    f.ks1 = lds_f32(st + 4 * (tk + 2));
-    f.vs0 = lds_f32(st + kTok * 4 + 4 * tk);
-    f.vs1 = lds_f32(st + kTok * 4 + 4 * (tk + 2));
+    f.ks0 = lds_f32(kt + i8::kCodeBytes + 4 * tk);
+    f.ks1 = lds_f32(kt + i8::kCodeBytes + 4 * (tk + 2));
+    f.vs0 = lds_f32(vt + i8::kCodeBytes + 4 * tk);
+    f.vs1 = lds_f32(vt + i8::kCodeBytes + 4 * (tk + 2));
   }
 
   __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const DecodeArgs& a,
@@ -236,11 +198,11 @@ struct Tiles8 {
 
 int decode_int8_workers_per_cta() { return tc::kWarps; }
 
-cudaError_t launch_decode_int8(const DecodeArgs& a, pa_dtype dtype, const Int8Maps& maps,
-                               int num_ctas, bool overlap, cudaStream_t stream) {
+cudaError_t launch_decode_int8(const DecodeArgs& a, pa_dtype dtype, int num_ctas, bool overlap,
+                               cudaStream_t stream) {
   if (dtype == PA_F16)
-    return tc::launch_tc<__half, 128, tc::Tiles8<__half>>(a, maps, num_ctas, overlap, stream);
-  return tc::launch_tc<__nv_bfloat16, 128, tc::Tiles8<__nv_bfloat16>>(a, maps, num_ctas, overlap,
+    return tc::launch_tc<__half, 128, tc::Tiles8<__half>>(a, {0}, num_ctas, overlap, stream);
+  return tc::launch_tc<__nv_bfloat16, 128, tc::Tiles8<__nv_bfloat16>>(a, {0}, num_ctas, overlap,
                                                                       stream);
 }
 

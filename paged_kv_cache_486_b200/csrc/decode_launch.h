@@ -15,10 +15,11 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, pa_dtype dtype, bool overlap
                                cudaStream_t stream);
 
 // Tensor-core path: fp16 / bf16, head_dim 64 or 128, group <= 8, block_size a
-// multiple of 16.  kmap / vmap describe the key / value pools as rows of
-// head_dim elements (see make_tile_maps in api.cu).
+// multiple of 16.  kmap / vmap describe the key / value pools (see
+// make_tile_map in api.cu): three_d = maps {64, rows, head_dim / 64}, else
+// {head_dim, rows}.
 cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
-                             const CUtensorMap& vmap, int num_ctas, bool overlap,
+                             const CUtensorMap& vmap, bool three_d, int num_ctas, bool overlap,
                              cudaStream_t stream);
 int decode_tc_workers_per_cta();
 size_t decode_tc_smem_bytes(int head_dim, int batch);

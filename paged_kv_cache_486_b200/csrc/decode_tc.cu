@@ -1,11 +1,12 @@
 // Paged decode attention on tensor cores over an fp16 / bf16 cache.
 //
 // Stage: 16 rows x D of the key pool and of the value pool, rows
-// (block * Hkv + kv_head) * block_size + 16 s, each loaded as D/64 TMA boxes of
-// 16 rows x 64 columns.  A box lands 128-byte-swizzled with one row per
-// 128-byte line, so the eight rows an ldmatrix reads sit in eight different
-// bank groups (with whole 256-byte rows in one box, rows t and t+4 would share
-// banks).  Keys enter S^T = K . Q^T as the A operand straight from ldmatrix;
+// (block * Hkv + kv_head) * block_size + 16 s, each loaded by one TMA copy as
+// D/64 column blocks of 16 rows x 64 columns (a 3-D box; two 2-D boxes if the
+// driver declines the 3-D map).  A column block lands 128-byte-swizzled with
+// one row per 128-byte line, so the eight rows an ldmatrix reads sit in eight
+// different bank groups (with whole 256-byte rows per line, rows t and t+4
+// would share banks).  Keys enter S^T = K . Q^T as the A operand straight from ldmatrix;
 // values enter O^T += V^T . P^T through ldmatrix.trans.
 //
 // Roofline.  Per context token and KV head the kernel must read D*2 bytes of
@@ -25,6 +26,7 @@ struct Tiles16 {
   static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
   struct Maps {
     CUtensorMap k, v;
+    int three_d;  // maps are {64, rows, D/64} (one copy per tile), else {D, rows}
   };
   struct Frag {
     uint32_t k[KC][4], v[KC][4];
@@ -45,8 +47,8 @@ struct Tiles16 {
                                int slot, int tile, int tok, uint32_t bar) {
     const int row = tile * a.block_size + tok;
     const uint32_t dst = stage(ring0, warp, slot);
-    tma_tile<D>(dst, &m.k, row, bar);
-    tma_tile<D>(dst + kTileBytes, &m.v, row, bar);
+    tma_tile<D>(dst, &m.k, row, m.three_d != 0, bar);
+    tma_tile<D>(dst + kTileBytes, &m.v, row, m.three_d != 0, bar);
   }
   // lane (g, cq) holds q[g][16kc + 2cq, +1] and q[g][16kc + 8 + 2cq, +1]
   __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 8 * half + 2 * cq; }
@@ -116,24 +118,26 @@ size_t decode_tc_smem_bytes(int head_dim, int batch) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
-                             const CUtensorMap& vmap, int num_ctas, bool overlap,
+                             const CUtensorMap& vmap, bool three_d, int num_ctas, bool overlap,
                              cudaStream_t stream) {
   using tc::Tiles16;
+  const int td = three_d ? 1 : 0;
   if (a.head_dim == 128) {
     if (dtype == PA_F16) {
       using P = Tiles16<__half, 128>;
-      return tc::launch_tc<__half, 128, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
+      return tc::launch_tc<__half, 128, P>(a, P::Maps{kmap, vmap, td}, num_ctas, overlap, stream);
     }
     using P = Tiles16<__nv_bfloat16, 128>;
-    return tc::launch_tc<__nv_bfloat16, 128, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap,
+    return tc::launch_tc<__nv_bfloat16, 128, P>(a, P::Maps{kmap, vmap, td}, num_ctas, overlap,
                                                 stream);
   }
   if (dtype == PA_F16) {
     using P = Tiles16<__half, 64>;
-    return tc::launch_tc<__half, 64, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
+    return tc::launch_tc<__half, 64, P>(a, P::Maps{kmap, vmap, td}, num_ctas, overlap, stream);
   }
   using P = Tiles16<__nv_bfloat16, 64>;
-  return tc::launch_tc<__nv_bfloat16, 64, P>(a, P::Maps{kmap, vmap}, num_ctas, overlap, stream);
+  return tc::launch_tc<__nv_bfloat16, 64, P>(a, P::Maps{kmap, vmap, td}, num_ctas, overlap,
+                                             stream);
 }
 
 }  // namespace pa

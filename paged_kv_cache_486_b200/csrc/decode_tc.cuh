@@ -97,10 +97,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 constexpr int kBoxBytes = kTok * 64 * 2;  // one 16 x 64 box of 16-bit elements
 
-// The tile of 16 rows x D: D/64 boxes, box h holding columns [64h, 64h + 64).
+// The tile of 16 rows x D lands as D/64 column blocks of 16 rows x 64 columns
+// (block h = columns [64h, 64h + 64)).  With a 3-D map {64 columns, rows, D/64
+// column blocks} it is one copy; with a 2-D map {D, rows} it is one copy per
+// column block.
 template <int D>
 __device__ __forceinline__ void tma_tile(uint32_t dst, const CUtensorMap* map, int row,
-                                         uint32_t bar) {
+                                         bool three_d, uint32_t bar) {
+  if (three_d) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(0), "r"(bar)
+        : "memory");
+    return;
+  }
 #pragma unroll
   for (int h = 0; h < D / 64; ++h) {
     asm volatile(
@@ -193,23 +204,6 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& head, uint32_
   tail = pack2<T>(a - h.x, b - h.y);
 }
 
-// Block id of unit u (or -1 past the worker's range), for the id window.
-__device__ __forceinline__ int32_t unit_block_id(const DecodeArgs& a, const int32_t* cum,
-                                                 int64_t u, int64_t u1) {
-  if (u >= u1) return -1;
-  const int b = find_seq(cum, a.batch, u, a.num_kv_heads);
-  const int nblk = cum[b + 1] - cum[b];
-  const int64_t rem = u - static_cast<int64_t>(a.num_kv_heads) * cum[b];
-  const int j = static_cast<int>(rem % nblk);
-  return __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j]);
-}
-
-__device__ __forceinline__ int stages_in_block(int ctx, int j, int bs) {
-  const int rem = ctx - j * bs;
-  const int n = rem < bs ? rem : bs;
-  return (n + kTok - 1) / kTok;
-}
-
 // What the producer lane tells the consumer about a stage it issued.
 constexpr int kHasData = 1;       // the tile was loaded (its block id was in range)
 constexpr int kSegStart = 2;      // first stage of a segment
@@ -221,9 +215,51 @@ constexpr int kMoreInRange = 32;  // the range continues after this (sequence, k
 struct StageMeta {
   int32_t b;
   int32_t kvh_flags;  // kv head << 16 | flags
-  int32_t tok0;       // first token of the stage in the sequence
+  int32_t n_valid;    // tokens of the stage inside the context (1 .. kTok)
   int32_t range;      // range the stage belongs to (piece slots)
 };
+
+// What the producer needs about one unit (one KV block of one (sequence, kv
+// head) pair inside a range [r0, r1)), packed in four words.  Each lane of a
+// warp computes the descriptor of one unit of a 32-unit window, a window
+// ahead of its use, so the producer's per-stage work is four shuffles.
+struct UnitDesc {
+  int32_t id;   // physical block id (-1 past the range)
+  int32_t bk;   // b << 16 | kv head
+  int32_t j;    // logical block index in the sequence
+  int32_t nf;   // tokens of the block inside the context | unit flags << 8
+};
+
+__device__ __forceinline__ UnitDesc unit_desc(const DecodeArgs& a, const int32_t* cum,
+                                              const int32_t* ctx_s, int64_t u, int64_t r0,
+                                              int64_t r1) {
+  UnitDesc d{-1, 0, 0, 0};
+  if (u >= r1) return d;
+  const int Hkv = a.num_kv_heads, bs = a.block_size;
+  const int b = find_seq(cum, a.batch, u, Hkv);
+  const int nblk = cum[b + 1] - cum[b];
+  const int rem = static_cast<int>(u - static_cast<int64_t>(Hkv) * cum[b]);  // < Hkv * nblk
+  const int kvh = rem / nblk;
+  const int j = rem - kvh * nblk;
+  const int64_t pair0 = u - j, pair1 = pair0 + nblk;
+  const int left = ctx_s[b] - j * bs;
+  const int ntok = left < bs ? left : bs;
+  const int flags = ((j == 0 || u == r0) ? kSegStart : 0) |
+                    ((u + 1 == r1 || j + 1 == nblk) ? kSegEnd : 0) |
+                    ((pair0 >= r0 && pair1 <= r1) ? kComplete : 0) |
+                    (pair0 <= r0 ? kFirstInRange : 0) | (pair1 < r1 ? kMoreInRange : 0);
+  d.id = __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + j]);
+  d.bk = (b << 16) | kvh;
+  d.j = j;
+  d.nf = ntok | (flags << 8);
+  return d;
+}
+
+__device__ __forceinline__ UnitDesc shfl_desc(const UnitDesc& d, int k) {
+  return UnitDesc{__shfl_sync(kFull, d.id, k), __shfl_sync(kFull, d.bk, k),
+                  __shfl_sync(kFull, d.j, k), __shfl_sync(kFull, d.nf, k)};
+}
+
 
 template <typename T, int D, class P>
 __global__ void __launch_bounds__(kWarps * 32, 1)
@@ -261,73 +297,65 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   StageMeta* wmeta = meta + warp * kStages;
 
   // ---------------- producer state (uniform across the warp) ----------------
+  // The warp walks its range(s) unit by unit; `cur` is the unit being issued.
   int64_t prange = w;
+  int64_t pr0 = active ? sp.start(w) : 0;
   int64_t pend = active ? sp.end(w) : 0;
-  UnitCursor pc;
-  cursor_seek(pc, active ? sp.start(w) : 0, pend, cum, B, Hkv);
-  int psub = 0;
-  int pnsub = active ? stages_in_block(ctx_s[pc.b], pc.j, bs) : 0;
-  bool pdone = !active, pnew_seg = true, pfirst = true;
-  int pseg_j0 = 0;
-  int64_t win = active ? sp.start(w) : 0;
-  int32_t ids_cur = unit_block_id(a, cum, win + lane, pend);
-  int32_t ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
+  int64_t pu = pr0;     // next unit to enter
+  int64_t win = pr0;    // first unit of the descriptor window
+  UnitDesc dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
+  UnitDesc dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+  UnitDesc cur{-1, 0, 0, 0};
+  int psub = 0, pnsub = 0;
+  bool pdone = !active;
 
   // Issues the next stage into `slot` (claiming a tail chunk when the current
   // range is used up); false when there is nothing left to issue.
   auto produce = [&](int slot) -> bool {
     if (pdone) return false;
-    if (pc.u >= pend) {
-      const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
-      if (chunk >= sp.NC) {
-        pdone = true;
-        return false;
+    if (psub == 0) {
+      if (pu >= pend) {
+        const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
+        if (chunk >= sp.NC) {
+          pdone = true;
+          return false;
+        }
+        prange = sp.W + chunk;
+        pr0 = pu = win = sp.start(prange);
+        pend = sp.end(prange);
+        dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
+        dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
       }
-      prange = sp.W + chunk;
-      win = sp.start(prange);
-      pend = sp.end(prange);
-      cursor_seek(pc, win, pend, cum, B, Hkv);
-      psub = 0;
-      pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
-      pnew_seg = pfirst = true;
-      ids_cur = unit_block_id(a, cum, win + lane, pend);
-      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
+      if (pu >= win + 32) {
+        win += 32;
+        dcur = dnext;
+        dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+      }
+      cur = shfl_desc(dcur, static_cast<int>(pu - win));
+      pnsub = ((cur.nf & 0xff) + kTok - 1) / kTok;
     }
-    if (pc.u >= win + 32) {
-      win += 32;
-      ids_cur = ids_next;
-      ids_next = unit_block_id(a, cum, win + 32 + lane, pend);
-    }
-    const int32_t id = __shfl_sync(kFull, ids_cur, static_cast<int>(pc.u - win));
-    if (pnew_seg) pseg_j0 = pc.j;
-    const int64_t pair_end = pc.u - pc.j + pc.nblk;  // one past the pair's last unit
-    const bool last_sub = psub + 1 == pnsub;
-    const bool seg_end = last_sub && (pc.u + 1 == pend || pc.j + 1 == pc.nblk);
-    const bool ok = id >= 0 && id < a.num_blocks;
-    const int flags = (ok ? kHasData : 0) | (pnew_seg ? kSegStart : 0) | (seg_end ? kSegEnd : 0) |
-                      (pseg_j0 == 0 && pair_end <= pend ? kComplete : 0) |
-                      (pfirst ? kFirstInRange : 0) | (pair_end < pend ? kMoreInRange : 0);
+    const int uflags = cur.nf >> 8;
+    const int left = (cur.nf & 0xff) - psub * kTok;
+    const bool ok = cur.id >= 0 && cur.id < a.num_blocks;
+    const int flags = (ok ? kHasData : 0) | (psub == 0 ? uflags & kSegStart : 0) |
+                      (psub + 1 == pnsub ? uflags & kSegEnd : 0) |
+                      (uflags & (kComplete | kFirstInRange | kMoreInRange));
     if (lane == 0) {
-      wmeta[slot] = StageMeta{pc.b, (pc.kvh << 16) | flags, pc.j * bs + psub * kTok,
+      const int kvh = cur.bk & 0xffff;
+      wmeta[slot] = StageMeta{cur.bk >> 16, (kvh << 16) | flags, left < kTok ? left : kTok,
                               static_cast<int32_t>(prange)};
       const uint32_t bar = bar0 + slot * 8;
       if (ok) {
         mbar_arrive_expect_tx(bar, P::kStageBytes);
-        P::issue(maps, a, ring0, warp, slot, id * Hkv + pc.kvh, psub * kTok, bar);
+        P::issue(maps, a, ring0, warp, slot, cur.id * Hkv + kvh, psub * kTok, bar);
       } else {
         report(a.dev_error, PA_DEVERR_BAD_BLOCK);
         mbar_arrive(bar);
       }
     }
-    if (seg_end) pfirst = false;
-    if (last_sub) {
+    if (++psub == pnsub) {
       psub = 0;
-      cursor_next(pc, cum, Hkv);
-      if (pc.u < pend) pnsub = stages_in_block(ctx_s[pc.b], pc.j, bs);
-      pnew_seg = pc.j == 0;
-    } else {
-      ++psub;
-      pnew_seg = false;
+      ++pu;
     }
     return true;
   };
@@ -355,9 +383,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
     }
   };
   if (active) {
-    load_q(qn, pc.b, pc.kvh);
-    qn_b = pc.b;
-    qn_kvh = pc.kvh;
+    const UnitDesc d0 = shfl_desc(dcur, 0);
+    qn_b = d0.bk >> 16;
+    qn_kvh = d0.bk & 0xffff;
+    load_q(qn, qn_b, qn_kvh);
   }
 
   wait_prior_grid();  // from here on the cache, the output and the workspace are used
@@ -416,7 +445,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
     }
 
-    const int n_valid = ctx_s[b] - md.tok0 < kTok ? ctx_s[b] - md.tok0 : kTok;
+    const int n_valid = md.n_valid;
     const bool have = (flags & kHasData) != 0;
     // Move the stage into registers first and hand the slot straight back to
     // TMA, so the ring keeps loading while this warp computes.

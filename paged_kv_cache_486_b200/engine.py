@@ -10,9 +10,9 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (PA_PATH_AUTO, Pool, pa_check_device_error, pa_copy_blocks, pa_decode_attention,
-               pa_decode_attention_int8, pa_decode_workspace_size, pa_reshape_and_cache,
-               pa_reshape_and_cache_int8)
+from . import (INT8_RECORD_BYTES, PA_PATH_AUTO, Pool, pa_check_device_error, pa_copy_blocks,
+               pa_decode_attention, pa_decode_attention_int8, pa_decode_workspace_size,
+               pa_reshape_and_cache, pa_reshape_and_cache_int8)
 
 
 class PagedKVCache:
@@ -92,55 +92,48 @@ class PagedKVCache:
 
 
 class PagedKVCacheInt8(PagedKVCache):
-    """The same pool and call order over an INT8 cache: codes + per-token fp32 scales
-    (key codes [NB, Hkv, bs, D], value codes transposed in 16-token groups
-    [NB, Hkv, bs/16, D, 16], scales [NB, Hkv, bs]).  key / value / q stay in `dtype`;
-    block_size a multiple of 16; head_dim 128 for decode."""
+    """The same pool and call order over an INT8 cache: a key pool and a value pool of
+    records [NB, Hkv, bs/16, 2112] (codes + per-token fp32 scales, layout in
+    include/pa.h).  key / value / q stay in `dtype`; head_dim 128, block_size a
+    multiple of 16."""
 
     def __init__(self, num_blocks, block_size, num_kv_heads, head_dim, dtype, num_q_heads,
                  max_batch, device="cuda", fill_bits=None):
+        if head_dim != 128 or block_size % 16:
+            raise ValueError("an INT8 cache needs head_dim 128 and block_size a multiple of 16")
         self.pool = Pool(num_blocks, block_size)
         self.num_blocks, self.block_size = num_blocks, block_size
         self.num_kv_heads, self.head_dim = num_kv_heads, head_dim
         self.num_q_heads, self.dtype, self.device = num_q_heads, dtype, torch.device(device)
-        dev = self.device
-        self.k_codes = torch.empty((num_blocks, num_kv_heads, block_size, head_dim),
-                                   dtype=torch.int8, device=dev)
-        if block_size % 16:
-            raise ValueError("an INT8 cache needs block_size a multiple of 16")
-        self.v_codes = torch.empty((num_blocks, num_kv_heads, block_size // 16, head_dim, 16),
-                                   dtype=torch.int8, device=dev)
-        self.k_scales = torch.empty((num_blocks, num_kv_heads, block_size), dtype=torch.float32,
-                                    device=dev)
-        self.v_scales = torch.empty_like(self.k_scales)
+        shape = (num_blocks, num_kv_heads, block_size // 16, INT8_RECORD_BYTES)
+        self.k_pool = torch.empty(shape, dtype=torch.uint8, device=self.device)
+        self.v_pool = torch.empty(shape, dtype=torch.uint8, device=self.device)
         if fill_bits is not None:  # poison unwritten slots: codes with a pattern, scales NaN
-            self.k_codes.view(torch.uint8).fill_(fill_bits & 0xFF)
-            self.v_codes.view(torch.uint8).fill_(fill_bits & 0xFF)
-            self.k_scales.fill_(float("nan"))
-            self.v_scales.fill_(float("nan"))
-        self.dev_error = torch.zeros(1, dtype=torch.int32, device=dev)
+            for p in (self.k_pool, self.v_pool):
+                p[..., :2048].fill_(fill_bits & 0xFF)
+                p[..., 2048:].view(torch.float32).fill_(float("nan"))
+        self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
         ws = pa_decode_workspace_size(max_batch, num_q_heads, num_kv_heads, head_dim)
-        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=dev)
+        self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
 
     def alloc(self, seq_id, n, stream=None):
         slots, cow = self.pool.pa_alloc(seq_id, n)
         if len(cow):
             pairs = torch.from_numpy(cow).to(self.device, non_blocking=False)
-            pa_copy_blocks([self.k_codes], [self.v_codes], pairs, self.dev_error, stream)
-            pa_copy_blocks([self.k_scales], [self.v_scales], pairs, self.dev_error, stream)
+            pa_copy_blocks([self.k_pool], [self.v_pool], pairs, self.dev_error, stream)
         return slots, cow
 
     def write(self, key, value, slots, stream=None):
         if not isinstance(slots, torch.Tensor):
             slots = torch.from_numpy(np.ascontiguousarray(slots, dtype=np.int64)).to(self.device)
-        pa_reshape_and_cache_int8(key, value, self.k_codes, self.v_codes, self.k_scales,
-                                  self.v_scales, slots, self.dev_error, stream)
+        pa_reshape_and_cache_int8(key, value, self.k_pool, self.v_pool, slots, self.dev_error,
+                                  stream)
 
     def decode(self, q, block_tables, context_lens, scale, out=None, num_workers=0, flags=0,
                stream=None, **_):
         if out is None:
             out = torch.empty_like(q)
-        pa_decode_attention_int8(out, q, self.k_codes, self.v_codes, self.k_scales, self.v_scales,
-                                 block_tables, context_lens, scale, self.workspace,
-                                 self.dev_error, num_workers, flags, stream)
+        pa_decode_attention_int8(out, q, self.k_pool, self.v_pool, block_tables, context_lens,
+                                 scale, self.workspace, self.dev_error, num_workers, flags,
+                                 stream)
         return out

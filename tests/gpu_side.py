@@ -86,15 +86,36 @@ def build_int8(wl, poison=True, workers=0, stream=None):
     return dict(eng=eng, bt=bt, ctx=ctx, q=q, out=out)
 
 
+def _key_record_offsets():
+    """[16, 128] byte offsets of code d of group token t in a key record (the layout
+    stated in include/pa.h, written out here from that statement)."""
+    off = np.zeros((16, 128), np.int64)
+    for t in range(16):
+        i, h, e = t >> 2, (t >> 1) & 1, t & 1
+        line = 2 * i + e + 8 * h
+        for d in range(128):
+            off[t, d] = line * 128 + 16 * ((d // 16) ^ (line % 8)) + d % 16
+    return torch.from_numpy(off)
+
+
+_KEY_OFF = _key_record_offsets()
+
+
 def gathered_int8(eng, bt, ctx, b, kvh):
-    """(k codes [n, D], v codes [n, D], k scales [n], v scales [n]) of batch row b and
-    kv head kvh in logical order, read through its table (torch indexing)."""
+    """(k codes [n, 128], v codes [n, 128], k scales [n], v scales [n]) of batch row b and
+    kv head kvh in logical order, decoded from the INT8 records through its table."""
     n = int(ctx[b])
     bs = eng.block_size
-    pos = torch.arange(n, device=eng.k_codes.device)
+    dev = eng.k_pool.device
+    pos = torch.arange(n, device=dev)
     blk = bt[b].long()[pos // bs]
-    off = pos % bs
-    # per-head views first, so each gather has one advanced-index pattern
-    kc, vc = eng.k_codes[:, kvh], eng.v_codes[:, kvh]  # [NB, bs, D], [NB, bs/16, D, 16]
-    return (kc[blk, off, :], vc[blk, off // 16, :, off % 16], eng.k_scales[:, kvh][blk, off],
-            eng.v_scales[:, kvh][blk, off])
+    grp = (pos % bs) // 16
+    t = pos % 16
+    krec = eng.k_pool[:, kvh][blk, grp]           # [n, 2112] uint8
+    vrec = eng.v_pool[:, kvh][blk, grp]
+    kc = torch.gather(krec, 1, _KEY_OFF.to(dev)[t]).view(torch.int8)
+    d = torch.arange(128, device=dev)
+    vc = torch.gather(vrec, 1, d[None, :] * 16 + t[:, None]).view(torch.int8)
+    ks = krec[:, 2048:].contiguous().view(torch.float32).gather(1, t[:, None])[:, 0]
+    vs = vrec[:, 2048:].contiguous().view(torch.float32).gather(1, t[:, None])[:, 0]
+    return kc, vc, ks, vs

@@ -111,25 +111,25 @@ def test_plan_chooses_tensor_cores_where_they_apply():
 
 def _int8_args(**kw):
     p = C.c_void_p(16)
-    args = dict(out=p, q=p, kc=p, vc=p, ks=p, vs=p, bt=p, ctx=p, B=4, Hq=8, Hkv=2, D=128, bs=16,
-                NB=10, MB=4, scale=0.1, dtype=pa.PA_F16, ws=p, ws_bytes=1 << 30, err=None,
-                workers=0, flags=0, stream=None)
+    args = dict(out=p, q=p, kp=p, vp=p, bt=p, ctx=p, B=4, Hq=8, Hkv=2, D=128, bs=16, NB=10, MB=4,
+                scale=0.1, dtype=pa.PA_F16, ws=p, ws_bytes=1 << 30, err=None, workers=0, flags=0,
+                stream=None)
     args.update(kw)
     return args
 
 
 def _call_decode_int8(a):
     return pa.lib.pa_decode_attention_int8(
-        a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["ctx"], a["B"], a["Hq"],
-        a["Hkv"], a["D"], a["bs"], a["NB"], a["MB"], a["scale"], a["dtype"], a["ws"],
-        a["ws_bytes"], a["err"], a["workers"], a["flags"], a["stream"])
+        a["out"], a["q"], a["kp"], a["vp"], a["bt"], a["ctx"], a["B"], a["Hq"], a["Hkv"], a["D"],
+        a["bs"], a["NB"], a["MB"], a["scale"], a["dtype"], a["ws"], a["ws_bytes"], a["err"],
+        a["workers"], a["flags"], a["stream"])
 
 
 @pytest.mark.parametrize("bad", [
     dict(D=64), dict(dtype=pa.PA_F32), dict(Hq=32, Hkv=2), dict(bs=8), dict(bs=48),
-    dict(Hq=7), dict(B=-1), dict(B=5000), dict(ws_bytes=16), dict(ks=None),
-    dict(vs=C.c_void_p(8)), dict(kc=C.c_void_p(4)), dict(flags=4), dict(scale=float("nan")),
-    dict(NB=1 << 22, Hkv=8, Hq=8), dict(NB=0),
+    dict(Hq=7), dict(B=-1), dict(B=5000), dict(ws_bytes=16), dict(kp=None),
+    dict(vp=C.c_void_p(8)), dict(flags=4), dict(scale=float("nan")),
+    dict(NB=1 << 24, Hkv=8, Hq=8), dict(Hkv=5000, Hq=5000), dict(MB=1 << 30, Hkv=4, Hq=8),
 ])
 def test_int8_decode_rejects_bad_arguments_on_host(bad):
     st = _call_decode_int8(_int8_args(**bad))
@@ -140,16 +140,23 @@ def test_int8_decode_rejects_bad_arguments_on_host(bad):
 def test_int8_cache_write_rejects_bad_arguments():
     p = C.c_void_p(16)
 
-    def call(key=p, ks=p, T=4, Hkv=2, D=128, bs=16, NB=10, dt=pa.PA_F16):
-        return pa.lib.pa_reshape_and_cache_int8(key, p, p, p, ks, p, p, T, Hkv, D, bs, NB, dt,
-                                                None, None)
+    def call(key=p, kp=p, T=4, Hkv=2, D=128, bs=16, NB=10, dt=pa.PA_F16):
+        return pa.lib.pa_reshape_and_cache_int8(key, p, kp, p, p, T, Hkv, D, bs, NB, dt, None,
+                                                None)
 
-    assert call(D=96) == pa.PA_ERR_INVALID
+    assert call(D=64) == pa.PA_ERR_INVALID
     assert call(bs=8) == pa.PA_ERR_INVALID
     assert call(bs=24) == pa.PA_ERR_INVALID
     assert call(T=-1) == pa.PA_ERR_INVALID
     assert call(dt=9) == pa.PA_ERR_INVALID
     assert call(key=C.c_void_p(8)) == pa.PA_ERR_INVALID
-    assert call(ks=None) == pa.PA_ERR_INVALID
+    assert call(kp=None) == pa.PA_ERR_INVALID
     assert call(T=0) == pa.PA_OK
     assert _call_decode_int8(_int8_args(B=0, q=None, out=None)) == pa.PA_OK
+
+
+def test_int8_block_bytes():
+    assert pa.pa_int8_block_bytes(8, 128, 16) == 8 * 2112
+    assert pa.pa_int8_block_bytes(8, 128, 64) == 8 * 4 * 2112
+    assert pa.pa_int8_block_bytes(8, 64, 16) == 0
+    assert pa.pa_int8_block_bytes(8, 128, 8) == 0

@@ -51,7 +51,7 @@ def _check_cache(wl, g, o):
             kc, vc, ks, vs = (t.cpu().numpy() for t in gathered_int8(g["eng"], g["bt"],
                                                                      g["ctx"], b, h))
             assert np.array_equal(kc, cache.k[blk, h, off, :])
-            assert np.array_equal(vc, cache.v[:, h][blk, off // 16, :, off % 16])
+            assert np.array_equal(vc, cache.v[blk, h, off, :])
             assert np.array_equal(ks.view(np.uint32), cache.ks[blk, h, off].view(np.uint32))
             assert np.array_equal(vs.view(np.uint32), cache.vs[blk, h, off].view(np.uint32))
 
@@ -71,9 +71,9 @@ def test_int8_small_configs_match_the_oracle(name, workers):
     assert g["eng"].device_errors() == 0
 
 
-@pytest.mark.parametrize("dtype,D", [("f32", 128), ("f16", 64), ("bf16", 64), ("f32", 64)])
-def test_int8_cache_write_other_dtypes_and_head_dims(dtype, D):
-    wl = workloads.custom("i8w", dtype, B=4, Hq=4, Hkv=2, D=D, bs=16, ctx=[1, 17, 40, 300],
+@pytest.mark.parametrize("dtype,bs", [("f32", 16), ("f16", 32), ("bf16", 64), ("f32", 128)])
+def test_int8_cache_write_other_dtypes_and_block_sizes(dtype, bs):
+    wl = workloads.custom("i8w", dtype, B=4, Hq=4, Hkv=2, D=128, bs=bs, ctx=[1, 17, 40, 300],
                           seed=26)
     from paged_kv_cache_486_b200.engine import PagedKVCacheInt8
     eng = PagedKVCacheInt8(wl.num_blocks, wl.bs, wl.Hkv, wl.D, workloads.TORCH_DTYPE[dtype],

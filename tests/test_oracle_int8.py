@@ -1,5 +1,5 @@
 """Pins the oracle's INT8 KV cache: the quantisation rule's closed-form cases and
-error bound, the cache layout (value codes transposed in 16-token groups), and attention over the
+error bound, the cache layout, and attention over the
 dequantised rows against torch's fp64 scaled-dot-product attention."""
 import numpy as np
 import pytest
@@ -84,14 +84,12 @@ def test_cache_layout_and_attention_against_library():
         v = raw(wl.contiguous_kv(int(seq), 1)).reshape(n * wl.Hkv, wl.D)
         kc, ks = oracle.quantize_rows(k, "f16")
         vc, vs = oracle.quantize_rows(v, "f16")
-        # layout: token j of head g sits at key row (blk, g, off) and, for values, at
-        # column off % 16 of group off // 16: (blk, g, off // 16, :, off % 16)
+        # layout: token j of head g sits at row (blk, g, off) of both code arrays
         for j in range(n):
             blk, off = table[b, j // wl.bs], j % wl.bs
             for g in range(wl.Hkv):
                 assert np.array_equal(cache.k[blk, g, off], kc[j * wl.Hkv + g])
-                assert np.array_equal(cache.v[blk, g, off // 16, :, off % 16],
-                                      vc[j * wl.Hkv + g])
+                assert np.array_equal(cache.v[blk, g, off], vc[j * wl.Hkv + g])
                 assert cache.ks[blk, g, off] == ks[j * wl.Hkv + g]
         kd = torch.from_numpy((kc * ks[:, None].astype(np.float64)).reshape(n, wl.Hkv, wl.D))
         vd = torch.from_numpy((vc * vs[:, None].astype(np.float64)).reshape(n, wl.Hkv, wl.D))
