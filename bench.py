@@ -539,6 +539,102 @@ def run_int8(args, dist, rank, world):
     }
 
 
+def run_prefix(args, dist, rank, world):
+    """Prefix caching on the prefix_prompts workload: admission of every request
+    through pa_alloc_tokens (host), the K/V write of the tokens the cache does not
+    supply, and decode over the shared blocks; each against the same run without
+    the cache."""
+    import paged_kv_cache_486_b200 as pa
+    from paged_kv_cache_486_b200.engine import PagedKVCache
+    ps = workloads.prefix_prompts()
+    dt = workloads.TORCH_DTYPE[ps.dtype]
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    res = {}
+    for on in (True, False):
+        eng = PagedKVCache(ps.num_blocks, ps.bs, ps.Hkv, ps.D, dt, ps.Hq, ps.B, "cuda")
+        eng.pool.pa_set_prefix_caching(on)
+        # host admission: every request, timed on the host clock (pool work only)
+        t0 = time.perf_counter()
+        adm = [eng.pool.pa_alloc_tokens(i, ids) for i, ids in enumerate(ps.prompts)]
+        host_s = time.perf_counter() - t0
+        assert all(len(a[1]) == 0 for a in adm)
+        slots = np.concatenate([a[0] for a in adm])
+        keep = slots >= 0
+        # rows of the written tokens only, generated on the device
+        ids = np.concatenate(ps.prompts)
+        pos = np.concatenate([np.arange(len(p)) for p in ps.prompts])
+        k = workloads.token_rows(ps.seed, 0, ids[keep], pos[keep], ps.Hkv, ps.D, ps.dtype, "cuda")
+        v = workloads.token_rows(ps.seed, 1, ids[keep], pos[keep], ps.Hkv, ps.D, ps.dtype, "cuda")
+        d_slots = torch.from_numpy(slots[keep]).cuda()
+        write_ms = []
+        for it in range(args.warmup + args.steps):
+            e0.record(stream)
+            pa.pa_reshape_and_cache(k, v, eng.k_cache, eng.v_cache, d_slots, eng.dev_error)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= args.warmup:
+                write_ms.append(e0.elapsed_time(e1))
+        bt, ctx = eng.block_tables(list(range(ps.B)), max(len(p) for p in ps.prompts) // ps.bs + 1)
+        q = ps.q("cuda")
+        out = torch.empty_like(q)
+        flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        dec_ms = []
+        for it in range(args.warmup + args.steps):
+            _flush_l2(flush)
+            e0.record(stream)
+            eng.decode(q, bt, ctx, ps.scale, out=out)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= args.warmup:
+                dec_ms.append(e0.elapsed_time(e1))
+        assert eng.device_errors() == 0, "device guards fired"
+        used = ps.num_blocks - eng.pool.pa_num_free_blocks()  # the free count includes evictable
+        res[on] = dict(host_us=1e6 * host_s / ps.B, cached_tokens=int(sum(a[2] for a in adm)),
+                       written_tokens=int(keep.sum()), blocks_held=int(used),
+                       write_us=1e3 * statistics.mean(write_ms),
+                       decode_us=1e3 * statistics.mean(dec_ms), out=out.float().cpu())
+        del eng
+        torch.cuda.empty_cache()
+    on, off = res[True], res[False]
+    # decode over shared blocks reads the same logical rows: results agree
+    err = float((on["out"] - off["out"]).abs().max())
+    ctx_tokens = int(sum(len(p) for p in ps.prompts))
+    alg = ctx_tokens * ps.Hkv * ps.D * 2 * 2 + 2 * ps.B * ps.Hq * ps.D * 2
+    peak, peak_kind = _peak_hbm()
+    achieved = alg / (on["decode_us"] / 1e6) / 1e9
+    row_bytes = ps.Hkv * ps.D * 2 * 2
+    return {
+        "metric": "prefix-cache admission: requests/s through pa_alloc_tokens (host), with "
+                  "K/V write and decode over the shared blocks", "op": "prefix",
+        "value": 1e6 / on["host_us"], "unit": "requests/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "dtype": ps.dtype, "data": "synthetic (16 system prompts x 1024 tokens, U[16,256] own "
+                                   "tokens, 32000-id vocabulary; rows a function of (id, position))",
+        "config": {"workload": ps.name, "requests": ps.B, "q_heads": ps.Hq, "kv_heads": ps.Hkv,
+                   "head_dim": ps.D, "block_size": ps.bs, "context_tokens": ctx_tokens},
+        "host_us_per_request": {"cached": on["host_us"], "no_cache": off["host_us"]},
+        "cached_token_fraction": on["cached_tokens"] / ctx_tokens,
+        "blocks_held": {"cached": on["blocks_held"], "no_cache": off["blocks_held"]},
+        "kv_write": {"cached": {"tokens": on["written_tokens"], "us": on["write_us"],
+                                "bytes": on["written_tokens"] * row_bytes},
+                     "no_cache": {"tokens": off["written_tokens"], "us": off["write_us"],
+                                  "bytes": off["written_tokens"] * row_bytes}},
+        "decode_us": {"cached": on["decode_us"], "no_cache": off["decode_us"]},
+        "decode_max_abs_diff_cached_vs_not": err,
+        "decode_kv_unique_read_gbs": {
+            k: res[v]["blocks_held"] * ps.bs * row_bytes / (res[v]["decode_us"] / 1e6) / 1e9
+            for k, v in (("cached", True), ("no_cache", False))},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
+                     "traffic": None,
+                     "timed": "decode over the prefix-cached pool, logical KV bytes (each "
+                              "request's rows counted once; shared blocks are read from L2 "
+                              "after the first, so this can exceed the HBM copy peak)"},
+        "gpu_launches": 2 * 2 * (args.warmup + args.steps),
+    }
+
+
 # ---------------------------------------------------------- oracle timings
 def cpu_baseline(wl, target_s=10.0):
     import oracle
@@ -623,9 +719,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="step", choices=["step", "swap", "int8"],
+    ap.add_argument("--op", default="step", choices=["step", "swap", "int8", "prefix"],
                     help="step: the decode step (default); swap: eviction to host and back; "
-                         "int8: the decode step over an INT8 cache")
+                         "int8: the decode step over an INT8 cache; prefix: prefix caching")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -644,7 +740,7 @@ def main():
     torch.cuda.set_device(local)
     dist, rank, world = _dist()
     try:
-        run = {"swap": run_swap, "int8": run_int8}.get(args.op, run_ours)
+        run = {"swap": run_swap, "int8": run_int8, "prefix": run_prefix}.get(args.op, run_ours)
         line = run(args, dist, rank, world)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -10,6 +10,8 @@
  *  [P2] "KV Cache and PagedAttention: Why Your LLM Server Slows Down", sections
  *       "What is the KV cache?", "How PagedAttention solves this", "How does
  *       PagedAttention work?".
+ *  [P3] "The KV cache and PagedAttention: why the LLM server chokes at 10 users",
+ *       the serving example and "The trade-offs".
  *  [P5] "KV Cache for intermediates: why long context eats the GPU and how to cut
  *       it 4x", sections "The precise scientific definition" and "The four
  *       solutions".
@@ -137,6 +139,53 @@ pa_status pa_swap(pa_pool* from, pa_pool* to, int64_t seq_id, int32_t* pairs_out
  * more than max_blocks blocks; PA_ERR_NOT_FOUND if one is unknown. */
 pa_status pa_block_table(const pa_pool* pool, const int64_t* seq_ids_host, int32_t n_seqs,
                          int32_t max_blocks, int32_t* table_out_host, int32_t* ctx_lens_out_host);
+
+/* ------------------------------------------------------------------------
+ * Prefix caching.  [P3] the serving example (the lines explained after the
+ * `vllm serve` command, "--enable-prefix-caching") and "The trade-offs":
+ * blocks are reused when several requests share the same beginning, such as
+ * one system prompt, and the cached blocks take space in the pool; [P2] "How
+ * PagedAttention solves this": shared prefix pages.  Readings (the pages give
+ * no algorithm):
+ *  - Only full blocks are cached, keyed by the exact token ids from the start
+ *    of the sequence to the block's end (the library keys them with a 64-bit
+ *    chain over (parent key, the block's ids) and compares the block's ids on
+ *    every hit).  A block is keyed once it is full and every token id of its
+ *    sequence up to it is known; the first block written with a key takes the
+ *    entry, later copies of the same content are not entered.
+ *  - Lookups happen when a sequence receives its first tokens through
+ *    pa_alloc_tokens: its leading full blocks are taken from the cache while
+ *    they match, but never a block that holds the last of those tokens (that
+ *    token is always computed, so its K/V are written).
+ *  - A cached block that loses its last holder is not freed: it joins an
+ *    evictable list (a sequence's blocks in reverse logical order, so its later
+ *    blocks leave first) and can still be found.  New blocks come from the
+ *    free stack first, then from the oldest evictable cached block, whose entry
+ *    is dropped.  pa_num_free_blocks counts both.
+ *  - Sequences grown by pa_alloc / pa_alloc_batch (no token ids) stop being
+ *    keyed from then on.  pa_swap carries the keying state; the moved blocks
+ *    are not cached in the destination pool.
+ * Off by default; turning it off returns every evictable cached block to the
+ * free stack (oldest first) and drops every entry.
+ * ---------------------------------------------------------------------- */
+pa_status pa_pool_set_prefix_caching(pa_pool* pool, int32_t enable);
+
+/* pa_alloc with the new tokens' ids (token_ids_host[n_new], any int32 values).
+ * For a sequence that holds no token yet, with prefix caching on, the leading
+ * full blocks found in the cache are shared instead of allocated: their
+ * tokens get slot -1 in slot_mapping_out_host (the caller writes nothing for
+ * them; pa_reshape_and_cache skips -1) and *n_cached_out = their count (a
+ * multiple of block_size).  Every other token gets its slot as in pa_alloc,
+ * copy-on-write pairs likewise.  Full blocks are then keyed and cached.
+ * All or nothing (PA_ERR_OOM leaves the pool unchanged). */
+pa_status pa_alloc_tokens(pa_pool* pool, int64_t seq_id, const int32_t* token_ids_host,
+                          int32_t n_new, int64_t* slot_mapping_out_host,
+                          int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out,
+                          int32_t* n_cached_out);
+
+/* Cached blocks (held by sequences or evictable), and the evictable ones. */
+int32_t pa_num_cached_blocks(const pa_pool* pool);
+int32_t pa_num_evictable_blocks(const pa_pool* pool);
 
 int32_t pa_num_free_blocks(const pa_pool* pool);
 /* Number of sequences holding `block` (0 if free, -1 if out of range). */

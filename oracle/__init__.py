@@ -50,6 +50,14 @@ def lib():
         L.orc_holders.argtypes = [P, C.c_int32]
         L.orc_alloc.restype = C.c_int
         L.orc_alloc.argtypes = [P, C.c_int64, C.c_int32, P, P, P]
+        L.orc_alloc_tokens.restype = C.c_int
+        L.orc_alloc_tokens.argtypes = [P, C.c_int64, P, C.c_int32, P, P, P, P]
+        L.orc_set_prefix_caching.restype = None
+        L.orc_set_prefix_caching.argtypes = [P, C.c_int32]
+        L.orc_num_cached.restype = C.c_int32
+        L.orc_num_cached.argtypes = [P]
+        L.orc_num_releasable.restype = C.c_int32
+        L.orc_num_releasable.argtypes = [P]
         L.orc_free.restype = C.c_int
         L.orc_free.argtypes = [P, C.c_int64]
         L.orc_fork.restype = C.c_int
@@ -152,6 +160,31 @@ class Pool:
         if st != OK:
             return st, None, None
         return st, slots[:n].copy(), pair.reshape(1, 2)[: int(ncow[0])].copy()
+
+    def alloc_tokens(self, seq, ids):
+        """Grow with token ids (prefix-cache reuse for a new sequence).
+        Returns (status, slots int64[n] with -1 for cached tokens, cow pairs, n_cached)."""
+        ids = _c(ids, np.int32)
+        n = len(ids)
+        slots = np.zeros(max(n, 1), dtype=np.int64)
+        pair = np.zeros(2, dtype=np.int32)
+        ncow = np.zeros(1, dtype=np.int32)
+        ncached = np.zeros(1, dtype=np.int32)
+        st = lib().orc_alloc_tokens(self.h, seq, _ptr(ids), n, _ptr(slots), _ptr(pair),
+                                    _ptr(ncow), _ptr(ncached))
+        if st != OK:
+            return st, None, None, 0
+        return (st, slots[:n].copy(), pair.reshape(1, 2)[: int(ncow[0])].copy(),
+                int(ncached[0]))
+
+    def set_prefix_caching(self, enable):
+        lib().orc_set_prefix_caching(self.h, 1 if enable else 0)
+
+    def num_cached(self):
+        return lib().orc_num_cached(self.h)
+
+    def num_releasable(self):
+        return lib().orc_num_releasable(self.h)
 
     def free(self, seq):
         return lib().orc_free(self.h, seq)

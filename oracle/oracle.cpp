@@ -136,11 +136,32 @@ double load_elem(const void* base, int64_t idx, int dtype) {
 //    sequences also hold copies that block first (one copy pair per call); a
 //    full shared block stays shared; the last holder writes in place.
 //  * An allocation either succeeds completely or changes nothing.
+//
+// Prefix caching ([P3] the serving example with --enable-prefix-caching: a
+// request reuses the blocks of another request that began the same way, such
+// as one system prompt; [P3] "The trade-offs": those cached blocks take space
+// in the pool).  Readings where the pages are silent:
+//  * Only full blocks are cached, each under the exact list of token ids from
+//    the sequence's start to the block's end.  A full block is entered once its
+//    sequence's ids are all known (given with the tokens), unless that list
+//    already has a block.
+//  * A sequence receiving its first tokens reuses cached blocks for its
+//    leading full blocks while they match, but never one holding the last of
+//    the tokens given (that token is always computed).
+//  * A cached block whose last holder lets go stays findable, in a queue of
+//    releasable blocks (a sequence's blocks in reverse logical order).  New
+//    blocks come from the free stack first, then from the front of that queue
+//    (the block leaves the cache).
+//  * Growth without ids ends the sequence's entries; turning caching off
+//    returns the queue to the free stack (front first) and empties the cache.
 // ---------------------------------------------------------------------------
 
 struct Sequence {
   std::deque<int32_t> blocks;  // logical block j -> physical block id
   int64_t len = 0;             // tokens held
+  bool ids_known = true;       // every token came with its id
+  std::vector<int32_t> ids;    // the token ids (while ids_known)
+  int64_t considered = 0;      // full blocks already offered to the cache
 };
 
 struct Pool {
@@ -149,23 +170,75 @@ struct Pool {
   std::deque<int32_t> free_stack;      // back() is the top of the stack
   std::map<int32_t, int32_t> holders;  // physical block -> number of sequences holding it
   std::map<int64_t, Sequence> seqs;
+  bool prefix = false;                               // prefix caching on
+  std::map<std::vector<int32_t>, int32_t> cache;     // token ids from the start -> block
+  std::map<int32_t, std::vector<int32_t>> entry_of;  // cached block -> its list of ids
+  std::deque<int32_t> releasable;                    // cached, no holder; front leaves first
 };
 
 enum { ORC_OK = 0, ORC_INVALID = 1, ORC_OOM = 2, ORC_NOT_FOUND = 3 };
 
+int64_t available(const Pool* p) {
+  return static_cast<int64_t>(p->free_stack.size() + p->releasable.size());
+}
+
 int32_t take_block(Pool* p) {
-  const int32_t b = p->free_stack.back();
-  p->free_stack.pop_back();
+  int32_t b;
+  if (!p->free_stack.empty()) {
+    b = p->free_stack.back();
+    p->free_stack.pop_back();
+  } else {
+    b = p->releasable.front();
+    p->releasable.pop_front();
+    p->cache.erase(p->entry_of[b]);
+    p->entry_of.erase(b);
+  }
   p->holders[b] = 1;
   return b;
 }
 
-void drop_block(Pool* p, int32_t b) {
-  auto it = p->holders.find(b);
-  it->second -= 1;
-  if (it->second == 0) {
-    p->holders.erase(it);
-    p->free_stack.push_back(b);
+// A cached block found for a new sequence gains a holder (leaving the queue).
+void hold_block(Pool* p, int32_t b) {
+  if (p->holders[b] == 0) {
+    p->releasable.erase(std::find(p->releasable.begin(), p->releasable.end(), b));
+  }
+  p->holders[b] += 1;
+}
+
+// Each block of `list` loses one holder; those left without one go to the
+// free stack in list order, or, if cached, to the back of the queue in
+// reverse list order.
+template <typename List>
+void release_blocks(Pool* p, const List& list) {
+  std::vector<int32_t> emptied;
+  for (int32_t b : list) {
+    auto it = p->holders.find(b);
+    it->second -= 1;
+    if (it->second == 0) {
+      p->holders.erase(it);
+      if (p->entry_of.count(b)) {
+        emptied.push_back(b);
+      } else {
+        p->free_stack.push_back(b);
+      }
+    }
+  }
+  for (auto r = emptied.rbegin(); r != emptied.rend(); ++r) p->releasable.push_back(*r);
+}
+
+void drop_block(Pool* p, int32_t b) { release_blocks(p, std::vector<int32_t>{b}); }
+
+// Offer every full block of `s` not offered yet to the cache.
+void offer_full_blocks(Pool* p, Sequence& s) {
+  const int64_t bs = p->block_size;
+  while (s.ids_known && (s.considered + 1) * bs <= s.len) {
+    std::vector<int32_t> key(s.ids.begin(), s.ids.begin() + (s.considered + 1) * bs);
+    if (p->prefix && !p->cache.count(key)) {
+      const int32_t b = s.blocks[s.considered];
+      p->cache[key] = b;
+      p->entry_of[b] = key;
+    }
+    ++s.considered;
   }
 }
 
@@ -221,7 +294,27 @@ void* orc_pool_new(int32_t num_blocks, int32_t block_size) {
 void orc_pool_delete(void* pool) { delete static_cast<Pool*>(pool); }
 
 int32_t orc_num_free(const void* pool) {
-  return static_cast<int32_t>(static_cast<const Pool*>(pool)->free_stack.size());
+  return static_cast<int32_t>(available(static_cast<const Pool*>(pool)));
+}
+
+int32_t orc_num_cached(const void* pool) {
+  return static_cast<int32_t>(static_cast<const Pool*>(pool)->cache.size());
+}
+
+int32_t orc_num_releasable(const void* pool) {
+  return static_cast<int32_t>(static_cast<const Pool*>(pool)->releasable.size());
+}
+
+void orc_set_prefix_caching(void* pool, int32_t enable) {
+  Pool* p = static_cast<Pool*>(pool);
+  p->prefix = enable != 0;
+  if (p->prefix) return;
+  while (!p->releasable.empty()) {
+    p->free_stack.push_back(p->releasable.front());
+    p->releasable.pop_front();
+  }
+  p->cache.clear();
+  p->entry_of.clear();
 }
 
 int32_t orc_holders(const void* pool, int32_t block) {
@@ -247,9 +340,13 @@ int orc_alloc(void* pool, int64_t seq, int32_t n, int64_t* slots_out, int32_t* c
   const bool must_copy = into_last > 0 && holders_of(p, s.blocks.back()) > 1;
   const int64_t new_blocks = (n - into_last + bs - 1) / bs;
   const int64_t needed = (must_copy ? 1 : 0) + new_blocks;
-  if (needed > static_cast<int64_t>(p->free_stack.size())) return ORC_OOM;
+  if (needed > available(p)) return ORC_OOM;
 
   *n_cow_out = 0;
+  if (n > 0) {
+    s.ids_known = false;  // tokens without ids
+    s.ids.clear();
+  }
   if (must_copy) {
     const int32_t old_block = s.blocks.back();
     const int32_t new_block = take_block(p);
@@ -274,8 +371,66 @@ int orc_free(void* pool, int64_t seq) {
   Pool* p = static_cast<Pool*>(pool);
   auto it = p->seqs.find(seq);
   if (it == p->seqs.end()) return ORC_NOT_FOUND;
-  for (int32_t b : it->second.blocks) drop_block(p, b);
+  release_blocks(p, it->second.blocks);
   p->seqs.erase(it);
+  return ORC_OK;
+}
+
+// orc_alloc with the new tokens' ids, and prefix-cache reuse for a sequence
+// that holds no token yet.  Tokens served from the cache get slot -1; their
+// count goes to *n_cached_out.  All or nothing.
+int orc_alloc_tokens(void* pool, int64_t seq, const int32_t* ids, int32_t n, int64_t* slots_out,
+                     int32_t* cow_pair_out, int32_t* n_cow_out, int32_t* n_cached_out) {
+  Pool* p = static_cast<Pool*>(pool);
+  if (n < 0) return ORC_INVALID;
+  const int32_t bs = p->block_size;
+  Sequence fresh_seq;
+  auto it = p->seqs.find(seq);
+  Sequence& s = (it == p->seqs.end()) ? fresh_seq : it->second;
+
+  std::vector<int32_t> found;
+  if (p->prefix && s.len == 0 && s.ids_known) {
+    for (int64_t j = 0; (j + 1) * bs <= static_cast<int64_t>(n) - 1; ++j) {
+      const std::vector<int32_t> key(ids, ids + (j + 1) * bs);
+      auto c = p->cache.find(key);
+      if (c == p->cache.end()) break;
+      found.push_back(c->second);
+    }
+  }
+  int64_t found_unheld = 0;
+  for (int32_t b : found) found_unheld += holders_of(p, b) == 0 ? 1 : 0;
+  const int64_t cached_tokens = static_cast<int64_t>(found.size()) * bs;
+  const int64_t used_in_last = s.len % bs;
+  const int64_t room = used_in_last == 0 ? 0 : bs - used_in_last;
+  const int64_t into_last = std::min<int64_t>(room, n);
+  const bool must_copy = into_last > 0 && holders_of(p, s.blocks.back()) > 1;
+  const int64_t new_blocks = (n - cached_tokens - into_last + bs - 1) / bs;
+  if ((must_copy ? 1 : 0) + new_blocks > available(p) - found_unheld) return ORC_OOM;
+
+  for (int32_t b : found) {
+    hold_block(p, b);
+    s.blocks.push_back(b);
+  }
+  *n_cow_out = 0;
+  if (must_copy) {
+    const int32_t old_block = s.blocks.back();
+    const int32_t new_block = take_block(p);
+    drop_block(p, old_block);
+    s.blocks.back() = new_block;
+    cow_pair_out[0] = old_block;
+    cow_pair_out[1] = new_block;
+    *n_cow_out = 1;
+  }
+  for (int64_t k = 0; k < new_blocks; ++k) s.blocks.push_back(take_block(p));
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t pos = s.len + i;
+    slots_out[i] = i < cached_tokens ? -1 : static_cast<int64_t>(s.blocks[pos / bs]) * bs + pos % bs;
+  }
+  s.len += n;
+  if (s.ids_known) s.ids.insert(s.ids.end(), ids, ids + n);
+  offer_full_blocks(p, s);
+  *n_cached_out = static_cast<int32_t>(cached_tokens);
+  if (it == p->seqs.end()) p->seqs.emplace(seq, s);
   return ORC_OK;
 }
 
@@ -333,10 +488,9 @@ int orc_swap(void* from_pool, void* to_pool, int64_t seq, int32_t* pairs_out, in
   if (it == from->seqs.end()) return ORC_NOT_FOUND;
   if (to->seqs.count(seq) || from->block_size != to->block_size) return ORC_INVALID;
   const Sequence old = it->second;
-  if (static_cast<int64_t>(old.blocks.size()) > static_cast<int64_t>(to->free_stack.size()))
-    return ORC_OOM;
-  Sequence moved;
-  moved.len = old.len;
+  if (static_cast<int64_t>(old.blocks.size()) > available(to)) return ORC_OOM;
+  Sequence moved = old;  // length and ids move along; the new blocks are not cached
+  moved.blocks.clear();
   int32_t k = 0;
   for (int32_t b : old.blocks) {
     const int32_t nb = take_block(to);
@@ -345,7 +499,7 @@ int orc_swap(void* from_pool, void* to_pool, int64_t seq, int32_t* pairs_out, in
     pairs_out[2 * k + 1] = nb;
     ++k;
   }
-  for (int32_t b : old.blocks) drop_block(from, b);
+  release_blocks(from, old.blocks);
   from->seqs.erase(seq);
   to->seqs.emplace(seq, moved);
   *n_out = k;

@@ -37,6 +37,10 @@ SIGNATURES = {
     "pa_alloc_batch": (_I32, [_P, _P, _I32, _I32, _P, _P, _I32, _P]),
     "pa_swap": (_I32, [_P, _P, _I64, _P, _I32, _P]),
     "pa_swap_blocks": (_I32, [_P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I64, _P, _P]),
+    "pa_alloc_tokens": (_I32, [_P, _I64, _P, _I32, _P, _P, _I32, _P, _P]),
+    "pa_pool_set_prefix_caching": (_I32, [_P, _I32]),
+    "pa_num_cached_blocks": (_I32, [_P]),
+    "pa_num_evictable_blocks": (_I32, [_P]),
     "pa_free": (_I32, [_P, _I64]),
     "pa_fork": (_I32, [_P, _I64, _I64]),
     "pa_block_table": (_I32, [_P, _P, _I32, _I32, _P, _P]),
@@ -157,6 +161,29 @@ class Pool:
                                 _np_ptr(pairs), n, _np_ptr(self._ncow))
         _check(st, "pa_alloc_batch")
         return slots[:n * n_new_each], pairs[: int(self._ncow[0])].copy()
+
+    def pa_alloc_tokens(self, seq_id: int, token_ids):
+        """Grow seq_id by the given token ids -> (slot_mapping int64[n] with -1 for tokens
+        served from the prefix cache, cow_pairs int32[k, 2], n_cached)."""
+        ids = np.ascontiguousarray(token_ids, dtype=np.int32)
+        n = len(ids)
+        slots = np.empty(max(n, 1), dtype=np.int64)
+        cached = np.zeros(1, dtype=np.int32)
+        st = lib.pa_alloc_tokens(self._h, seq_id, _np_ptr(ids) if n else None, n, _np_ptr(slots),
+                                 _np_ptr(self._pair), 1, _np_ptr(self._ncow), _np_ptr(cached))
+        _check(st, "pa_alloc_tokens")
+        return (slots[:n], self._pair.reshape(1, 2)[: int(self._ncow[0])].copy(),
+                int(cached[0]))
+
+    def pa_set_prefix_caching(self, enable: bool):
+        _check(lib.pa_pool_set_prefix_caching(self._h, 1 if enable else 0),
+               "pa_pool_set_prefix_caching")
+
+    def pa_num_cached_blocks(self) -> int:
+        return lib.pa_num_cached_blocks(self._h)
+
+    def pa_num_evictable_blocks(self) -> int:
+        return lib.pa_num_evictable_blocks(self._h)
 
     def pa_free(self, seq_id: int):
         _check(lib.pa_free(self._h, seq_id), "pa_free")

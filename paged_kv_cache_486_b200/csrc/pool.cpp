@@ -8,10 +8,17 @@
 // PagedAttention: Why Your LLM Server Slows Down" / "How PagedAttention solves
 // this": on-demand pages; shared prefix pages with copy-on-write.
 //
-// Data layout: flat arrays indexed by block id (holder counts), a vector used
-// as the free stack (back = top), and a hash map from sequence id to the
-// sequence's block vector.  Every operation checks all preconditions before it
-// mutates anything, so a failed call leaves the pool unchanged.
+// Data layout: flat arrays indexed by block id (holder counts, prefix-cache
+// flags and the links of the evictable list), a vector used as the free stack
+// (back = top), and a hash map from sequence id to the sequence's block vector.
+// Every operation checks all preconditions before it mutates anything, so a
+// failed call leaves the pool unchanged.
+//
+// Prefix caching ("The KV cache and PagedAttention: why the LLM server chokes
+// at 10 users" / the serving example with --enable-prefix-caching, and "The
+// trade-offs": blocks are reused when several requests share the same
+// beginning, such as one system prompt; the cached blocks occupy the pool) is
+// opt-in per pool and described with pa_pool_set_prefix_caching in pa.h.
 #include <algorithm>
 #include <cstdint>
 #include <unordered_map>
@@ -23,21 +30,133 @@ struct pa_pool {
   struct Seq {
     std::vector<int32_t> blocks;
     int64_t len = 0;
+    // Prefix-cache state: token ids are known for every token (pa_alloc_tokens
+    // only); `hashed` full blocks have been keyed, `chain` is the key of the
+    // last of them, `tail` holds the ids of the tokens after them.
+    bool ids_known = true;
+    int64_t hashed = 0;
+    uint64_t chain = kRootKey;
+    std::vector<int32_t> tail;
   };
+  static constexpr uint64_t kRootKey = 0x9e3779b97f4a7c15ull;
+
   int32_t num_blocks = 0;
   int32_t block_size = 0;
   std::vector<int32_t> free_stack;  // back() = next block handed out
-  std::vector<int32_t> refs;        // holders per block
+  std::vector<int32_t> refs;        // holders per block (sequences)
   std::unordered_map<int64_t, Seq> seqs;
 
+  // Prefix cache: full blocks keyed by their token prefix.  A key is a 64-bit
+  // chain over (parent key, the block's token ids); each entry keeps its parent
+  // key and token ids, and a lookup compares them, so two different blocks
+  // only collide if their parents' 64-bit keys do.  A cached block with no
+  // holder waits in an LRU list (lru_*, oldest at the head) and is still found
+  // by lookups; fresh allocation takes the free stack first, then evicts the
+  // head of that list.
+  bool prefix = false;
+  struct Entry {
+    int32_t block;
+    uint64_t parent;
+    std::vector<int32_t> tokens;
+  };
+  std::unordered_map<uint64_t, Entry> entries;
+  std::vector<uint64_t> key_of;     // key of a cached block
+  std::vector<uint8_t> cached;      // block has an entry
+  std::vector<int32_t> lru_prev, lru_next;
+  int32_t lru_head = -1, lru_tail = -1, n_evictable = 0;
+
+  size_t available() const { return free_stack.size() + static_cast<size_t>(n_evictable); }
+
+  void lru_push_back(int32_t b) {
+    lru_prev[b] = lru_tail;
+    lru_next[b] = -1;
+    if (lru_tail >= 0) lru_next[lru_tail] = b; else lru_head = b;
+    lru_tail = b;
+    ++n_evictable;
+  }
+  void lru_remove(int32_t b) {
+    if (lru_prev[b] >= 0) lru_next[lru_prev[b]] = lru_next[b]; else lru_head = lru_next[b];
+    if (lru_next[b] >= 0) lru_prev[lru_next[b]] = lru_prev[b]; else lru_tail = lru_prev[b];
+    lru_prev[b] = lru_next[b] = -1;
+    --n_evictable;
+  }
+  void uncache(int32_t b) {
+    entries.erase(key_of[b]);
+    cached[b] = 0;
+  }
+  // A block for new tokens: the top of the free stack, else the least recently
+  // released cached block (its entry is dropped).
   int32_t pop() {
-    const int32_t b = free_stack.back();
-    free_stack.pop_back();
+    int32_t b;
+    if (!free_stack.empty()) {
+      b = free_stack.back();
+      free_stack.pop_back();
+    } else {
+      b = lru_head;
+      lru_remove(b);
+      uncache(b);
+    }
     refs[b] = 1;
     return b;
   }
-  void unref(int32_t b) {
-    if (--refs[b] == 0) free_stack.push_back(b);
+  // One more holder for a cached block found by a lookup.
+  void hold(int32_t b) {
+    if (refs[b]++ == 0) lru_remove(b);
+  }
+  // Drop one holder of each block of a list.  Blocks left without a holder
+  // return to the free stack in list order, or, if cached, join the LRU list
+  // in reverse list order (a sequence's later blocks are evicted first).
+  void release(const std::vector<int32_t>& bl) {
+    for (int32_t b : bl)
+      if (--refs[b] == 0 && !cached[b]) free_stack.push_back(b);
+    for (auto r = bl.rbegin(); r != bl.rend(); ++r)
+      if (refs[*r] == 0 && cached[*r]) lru_push_back(*r);
+  }
+  void unref(int32_t b) { release(std::vector<int32_t>{b}); }
+
+  static uint64_t mix(uint64_t x) {
+    x ^= x >> 31;
+    x *= 0x7fb5d329728ea185ull;
+    x ^= x >> 27;
+    x *= 0x81dadef4bc2dd44dull;
+    x ^= x >> 33;
+    return x;
+  }
+  static uint64_t block_key(uint64_t parent, const int32_t* ids, int n) {
+    uint64_t h = mix(parent ^ 0x5851f42d4c957f2dull);
+    for (int i = 0; i < n; ++i) h = mix(h + static_cast<uint32_t>(ids[i]) + 0x632be59bd9b4e019ull);
+    return h;
+  }
+  // The cached block holding (parent, ids), or -1.
+  int32_t lookup(uint64_t key, uint64_t parent, const int32_t* ids) const {
+    auto e = entries.find(key);
+    if (e == entries.end() || e->second.parent != parent ||
+        !std::equal(e->second.tokens.begin(), e->second.tokens.end(), ids))
+      return -1;
+    return e->second.block;
+  }
+  // Key every full block of `s` not keyed yet (its ids are known); register
+  // those whose key has no entry (while caching is on).
+  void key_full_blocks(Seq& s) {
+    const int64_t bs = block_size;
+    while (s.ids_known && (s.hashed + 1) * bs <= s.len) {
+      const uint64_t key = block_key(s.chain, s.tail.data(), block_size);
+      if (prefix && lookup(key, s.chain, s.tail.data()) < 0 && !entries.count(key)) {
+        const int32_t b = s.blocks[s.hashed];
+        entries.emplace(key, Entry{b, s.chain, std::vector<int32_t>(s.tail.begin(),
+                                                                    s.tail.begin() + bs)});
+        key_of[b] = key;
+        cached[b] = 1;
+      }
+      s.chain = key;
+      ++s.hashed;
+      s.tail.erase(s.tail.begin(), s.tail.begin() + bs);
+    }
+  }
+  void forget_ids(Seq& s) {
+    s.ids_known = false;
+    s.tail.clear();
+    s.tail.shrink_to_fit();
   }
 };
 
@@ -52,6 +171,10 @@ pa_status pa_pool_create(int32_t num_blocks, int32_t block_size, pa_pool** pool_
   p->num_blocks = num_blocks;
   p->block_size = block_size;
   p->refs.assign(num_blocks, 0);
+  p->key_of.assign(num_blocks, 0);
+  p->cached.assign(num_blocks, 0);
+  p->lru_prev.assign(num_blocks, -1);
+  p->lru_next.assign(num_blocks, -1);
   p->free_stack.resize(num_blocks);
   for (int32_t i = 0; i < num_blocks; ++i) p->free_stack[i] = num_blocks - 1 - i;
   *pool_out = p;
@@ -75,13 +198,14 @@ pa_status pa_alloc(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slot_m
   if (copy && (max_cow < 1 || !cow_pairs_out_host))
     return pa::fail(PA_ERR_INVALID, "pa_alloc: a copy-on-write pair is needed but max_cow=%d",
                     max_cow);
-  if ((copy ? 1 : 0) + fresh > static_cast<int64_t>(pool->free_stack.size()))
+  if ((copy ? 1 : 0) + fresh > static_cast<int64_t>(pool->available()))
     return pa::fail(PA_ERR_OOM, "pa_alloc: need %lld blocks, %zu free",
-                    static_cast<long long>((copy ? 1 : 0) + fresh), pool->free_stack.size());
+                    static_cast<long long>((copy ? 1 : 0) + fresh), pool->available());
   if (len + n_new > (int64_t(1) << 40))
     return pa::fail(PA_ERR_INVALID, "pa_alloc: sequence too long");
 
   pa_pool::Seq& s = known ? it->second : pool->seqs[seq_id];
+  if (n_new > 0) pool->forget_ids(s);  // tokens without ids: no more prefix keys
   *n_cow_out = 0;
   if (copy) {
     const int32_t src = s.blocks.back();
@@ -103,9 +227,12 @@ pa_status pa_alloc(pa_pool* pool, int64_t seq_id, int32_t n_new, int64_t* slot_m
 }
 
 // Batched growth: the same effect as n_seqs calls of pa_alloc in order, but one
-// call, and all or nothing -- on failure every sequence already grown in this
-// batch is restored exactly (blocks go back on the free stack in the order
-// they left it), so the pool is unchanged.
+// call, and all or nothing.  A first pass replays the batch on the lengths,
+// last blocks and holder counts it touches (a copy-on-write of a shared last
+// block drops that block's holder count, which can spare a later sequence its
+// copy) and checks the block demand and the copy pairs; the second pass then
+// cannot fail, so it never has to undo (an undo could not restore a cached
+// block that an allocation evicted).
 pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_seqs,
                          int32_t n_new_each, int64_t* slot_mapping_out_host,
                          int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out) {
@@ -113,46 +240,66 @@ pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_s
       (n_seqs > 0 && !seq_ids_host) ||
       (n_seqs > 0 && n_new_each > 0 && !slot_mapping_out_host) || (max_cow > 0 && !cow_pairs_out_host))
     return pa::fail(PA_ERR_INVALID, "pa_alloc_batch: bad arguments");
-  struct Undo {
-    int64_t seq;
-    bool created;
-    int64_t old_len;
-    int32_t cow_src, cow_dst;
-    int64_t fresh;
-  };
-  std::vector<Undo> log;
-  log.reserve(n_seqs);
+  const int64_t bs = pool->block_size;
+  {
+    std::unordered_map<int64_t, std::pair<int64_t, int32_t>> sim;  // id -> (len, last block)
+    std::unordered_map<int32_t, int32_t> drop;                      // block -> holders lost
+    int64_t need = 0;
+    int32_t cows = 0;
+    for (int32_t i = 0; i < n_seqs; ++i) {
+      const int64_t id = seq_ids_host[i];
+      auto si = sim.find(id);
+      int64_t len;
+      int32_t last;  // -1: none, -2: a block this batch gave the sequence
+      if (si != sim.end()) {
+        len = si->second.first;
+        last = si->second.second;
+      } else {
+        auto it = pool->seqs.find(id);
+        len = it == pool->seqs.end() ? 0 : it->second.len;
+        last = it == pool->seqs.end() || it->second.blocks.empty() ? -1 : it->second.blocks.back();
+      }
+      const int64_t tail = len % bs;
+      const int64_t fill = tail ? std::min<int64_t>(bs - tail, n_new_each) : 0;
+      const bool copy = fill > 0 && last >= 0 && pool->refs[last] - drop[last] > 1;
+      const int64_t fresh = (n_new_each - fill + bs - 1) / bs;
+      if (copy) {
+        ++cows;
+        ++drop[last];
+        last = -2;
+      }
+      if (fresh > 0) last = -2;
+      need += (copy ? 1 : 0) + fresh;
+      sim[id] = {len + n_new_each, last};
+      if (len + n_new_each > (int64_t(1) << 40))
+        return pa::fail(PA_ERR_INVALID, "pa_alloc_batch: sequence too long");
+    }
+    if (cows > max_cow)
+      return pa::fail(PA_ERR_INVALID, "pa_alloc_batch: %d copy pairs needed, room for %d", cows,
+                      max_cow);
+    if (need > static_cast<int64_t>(pool->available()))
+      return pa::fail(PA_ERR_OOM, "pa_alloc_batch: need %lld blocks, %zu free",
+                      static_cast<long long>(need), pool->available());
+  }
   int32_t n_cow = 0;
-  pa_status st = PA_OK;
   for (int32_t i = 0; i < n_seqs; ++i) {
     const int64_t id = seq_ids_host[i];
     auto it = pool->seqs.find(id);
     const bool known = it != pool->seqs.end();
-    const int64_t bs = pool->block_size;
     const int64_t len = known ? it->second.len : 0;
     const int64_t tail = len % bs;
     const int64_t fill = tail ? std::min<int64_t>(bs - tail, n_new_each) : 0;
     const bool copy = fill > 0 && pool->refs[it->second.blocks.back()] > 1;
     const int64_t fresh = (n_new_each - fill + bs - 1) / bs;
-    if (copy && n_cow >= max_cow) {
-      st = pa::fail(PA_ERR_INVALID, "pa_alloc_batch: more than max_cow=%d copy pairs", max_cow);
-      break;
-    }
-    if ((copy ? 1 : 0) + fresh > static_cast<int64_t>(pool->free_stack.size())) {
-      st = pa::fail(PA_ERR_OOM, "pa_alloc_batch: sequence %d of %d needs %lld blocks, %zu free",
-                    i, n_seqs, static_cast<long long>((copy ? 1 : 0) + fresh),
-                    pool->free_stack.size());
-      break;
-    }
     pa_pool::Seq& s = known ? it->second : pool->seqs[id];
-    Undo u{id, !known, len, -1, -1, fresh};
+    if (n_new_each > 0) pool->forget_ids(s);
     if (copy) {
-      u.cow_src = s.blocks.back();
-      u.cow_dst = pool->pop();
-      pool->unref(u.cow_src);
-      s.blocks.back() = u.cow_dst;
-      cow_pairs_out_host[2 * n_cow] = u.cow_src;
-      cow_pairs_out_host[2 * n_cow + 1] = u.cow_dst;
+      const int32_t src = s.blocks.back();
+      const int32_t dst = pool->pop();
+      pool->unref(src);
+      s.blocks.back() = dst;
+      cow_pairs_out_host[2 * n_cow] = src;
+      cow_pairs_out_host[2 * n_cow + 1] = dst;
       ++n_cow;
     }
     for (int64_t k = 0; k < fresh; ++k) s.blocks.push_back(pool->pop());
@@ -162,31 +309,115 @@ pa_status pa_alloc_batch(pa_pool* pool, const int64_t* seq_ids_host, int32_t n_s
       slots[k] = static_cast<int64_t>(s.blocks[pos / bs]) * bs + pos % bs;
     }
     s.len = len + n_new_each;
-    log.push_back(u);
-  }
-  if (st != PA_OK) {
-    for (auto r = log.rbegin(); r != log.rend(); ++r) {
-      pa_pool::Seq& s = pool->seqs[r->seq];
-      for (int64_t k = 0; k < r->fresh; ++k) {
-        const int32_t b = s.blocks.back();
-        s.blocks.pop_back();
-        pool->refs[b] = 0;
-        pool->free_stack.push_back(b);
-      }
-      if (r->cow_dst >= 0) {
-        s.blocks.back() = r->cow_src;
-        pool->refs[r->cow_src] += 1;
-        pool->refs[r->cow_dst] = 0;
-        pool->free_stack.push_back(r->cow_dst);
-      }
-      s.len = r->old_len;
-      if (r->created) pool->seqs.erase(r->seq);
-    }
-    return st;
   }
   *n_cow_out = n_cow;
   return PA_OK;
 }
+
+// Growth with token ids, and prefix-cache lookups for a new sequence (see
+// pa.h).  All or nothing: the blocks it must take (those the cache does not
+// supply, plus a copy-on-write block) are checked against the free stack plus
+// the evictable cached blocks that are not among its own hits, before anything
+// changes.
+pa_status pa_alloc_tokens(pa_pool* pool, int64_t seq_id, const int32_t* token_ids_host,
+                          int32_t n_new, int64_t* slot_mapping_out_host,
+                          int32_t* cow_pairs_out_host, int32_t max_cow, int32_t* n_cow_out,
+                          int32_t* n_cached_out) {
+  if (!pool || n_new < 0 || (n_new > 0 && (!slot_mapping_out_host || !token_ids_host)) ||
+      !n_cow_out || !n_cached_out)
+    return pa::fail(PA_ERR_INVALID, "pa_alloc_tokens: bad arguments (n_new=%d)", n_new);
+  const int64_t bs = pool->block_size;
+  auto it = pool->seqs.find(seq_id);
+  const bool known = it != pool->seqs.end();
+  const int64_t len = known ? it->second.len : 0;
+  // cache lookups: a sequence that holds no token yet, whole blocks that end
+  // before its last new token (that token is always computed)
+  std::vector<int32_t> hits;
+  uint64_t chain = pa_pool::kRootKey;
+  int32_t hits_evictable = 0;
+  if (pool->prefix && len == 0 && (!known || it->second.ids_known)) {
+    for (int64_t j = 0; (j + 1) * bs <= static_cast<int64_t>(n_new) - 1; ++j) {
+      const int32_t* ids = token_ids_host + j * bs;
+      const uint64_t key = pa_pool::block_key(chain, ids, pool->block_size);
+      const int32_t b = pool->lookup(key, chain, ids);
+      if (b < 0) break;
+      hits.push_back(b);
+      hits_evictable += pool->refs[b] == 0 ? 1 : 0;
+      chain = key;
+    }
+  }
+  const int64_t hit_tokens = static_cast<int64_t>(hits.size()) * bs;
+  const int64_t tail = len % bs;
+  const int64_t fill = tail ? std::min<int64_t>(bs - tail, n_new) : 0;
+  const bool copy = fill > 0 && pool->refs[it->second.blocks.back()] > 1;
+  const int64_t fresh = (n_new - hit_tokens - fill + bs - 1) / bs;
+  if (copy && (max_cow < 1 || !cow_pairs_out_host))
+    return pa::fail(PA_ERR_INVALID, "pa_alloc_tokens: a copy-on-write pair is needed but "
+                    "max_cow=%d", max_cow);
+  const int64_t avail = static_cast<int64_t>(pool->available()) - hits_evictable;
+  if ((copy ? 1 : 0) + fresh > avail)
+    return pa::fail(PA_ERR_OOM, "pa_alloc_tokens: need %lld blocks, %lld free",
+                    static_cast<long long>((copy ? 1 : 0) + fresh), static_cast<long long>(avail));
+  if (len + n_new > (int64_t(1) << 40))
+    return pa::fail(PA_ERR_INVALID, "pa_alloc_tokens: sequence too long");
+
+  pa_pool::Seq& s = known ? it->second : pool->seqs[seq_id];
+  for (int32_t b : hits) {
+    pool->hold(b);
+    s.blocks.push_back(b);
+  }
+  *n_cow_out = 0;
+  if (copy) {
+    const int32_t src = s.blocks.back();
+    const int32_t dst = pool->pop();
+    pool->unref(src);
+    s.blocks.back() = dst;
+    cow_pairs_out_host[0] = src;
+    cow_pairs_out_host[1] = dst;
+    *n_cow_out = 1;
+  }
+  for (int64_t k = 0; k < fresh; ++k) s.blocks.push_back(pool->pop());
+  for (int64_t i = 0; i < n_new; ++i) {
+    const int64_t pos = len + i;
+    slot_mapping_out_host[i] =
+        i < hit_tokens ? -1 : static_cast<int64_t>(s.blocks[pos / bs]) * bs + pos % bs;
+  }
+  s.len = len + n_new;
+  if (s.ids_known) {
+    if (!hits.empty()) {
+      s.hashed = static_cast<int64_t>(hits.size());
+      s.chain = chain;
+    }
+    s.tail.insert(s.tail.end(), token_ids_host + hit_tokens, token_ids_host + n_new);
+    pool->key_full_blocks(s);
+  }
+  *n_cached_out = static_cast<int32_t>(hit_tokens);
+  return PA_OK;
+}
+
+pa_status pa_pool_set_prefix_caching(pa_pool* pool, int32_t enable) {
+  if (!pool) return pa::fail(PA_ERR_INVALID, "pa_pool_set_prefix_caching: NULL pool");
+  if (enable) {
+    pool->prefix = true;
+    return PA_OK;
+  }
+  pool->prefix = false;
+  // evictable cached blocks become plain free blocks (oldest pushed first)
+  while (pool->lru_head >= 0) {
+    const int32_t b = pool->lru_head;
+    pool->lru_remove(b);
+    pool->free_stack.push_back(b);
+  }
+  pool->entries.clear();
+  std::fill(pool->cached.begin(), pool->cached.end(), 0);
+  return PA_OK;
+}
+
+int32_t pa_num_cached_blocks(const pa_pool* pool) {
+  return pool ? static_cast<int32_t>(pool->entries.size()) : -1;
+}
+
+int32_t pa_num_evictable_blocks(const pa_pool* pool) { return pool ? pool->n_evictable : -1; }
 
 // "KV Cache and PagedAttention: Why Your LLM Server Slows Down" / "How
 // PagedAttention solves this": under memory pressure small pages move to the
@@ -212,11 +443,15 @@ pa_status pa_swap(pa_pool* from, pa_pool* to, int64_t seq_id, int32_t* pairs_out
   const int32_t n = static_cast<int32_t>(src.size());
   if (n > max_pairs)
     return pa::fail(PA_ERR_INVALID, "pa_swap: %d pairs needed, room for %d", n, max_pairs);
-  if (n > static_cast<int32_t>(to->free_stack.size()))
+  if (n > static_cast<int32_t>(to->available()))
     return pa::fail(PA_ERR_OOM, "pa_swap: %d blocks needed, %zu free in the destination", n,
-                    to->free_stack.size());
+                    to->available());
   pa_pool::Seq moved;
   moved.len = it->second.len;
+  moved.ids_known = it->second.ids_known;  // keys continue; the moved blocks are not cached
+  moved.hashed = it->second.hashed;
+  moved.chain = it->second.chain;
+  moved.tail = it->second.tail;
   moved.blocks.reserve(n);
   for (int32_t k = 0; k < n; ++k) {
     const int32_t b = to->pop();
@@ -224,7 +459,7 @@ pa_status pa_swap(pa_pool* from, pa_pool* to, int64_t seq_id, int32_t* pairs_out
     pairs_out_host[2 * k] = src[k];
     pairs_out_host[2 * k + 1] = b;
   }
-  for (int32_t b : src) from->unref(b);
+  from->release(src);
   from->seqs.erase(it);
   to->seqs.emplace(seq_id, std::move(moved));
   *n_pairs_out = n;
@@ -237,7 +472,7 @@ pa_status pa_free(pa_pool* pool, int64_t seq_id) {
   if (it == pool->seqs.end())
     return pa::fail(PA_ERR_NOT_FOUND, "pa_free: unknown sequence %lld",
                     static_cast<long long>(seq_id));
-  for (int32_t b : it->second.blocks) pool->unref(b);
+  pool->release(it->second.blocks);
   pool->seqs.erase(it);
   return PA_OK;
 }
@@ -285,7 +520,7 @@ pa_status pa_block_table(const pa_pool* pool, const int64_t* seq_ids_host, int32
 }
 
 int32_t pa_num_free_blocks(const pa_pool* pool) {
-  return pool ? static_cast<int32_t>(pool->free_stack.size()) : -1;
+  return pool ? static_cast<int32_t>(pool->available()) : -1;
 }
 
 int32_t pa_refcount(const pa_pool* pool, int32_t block) {

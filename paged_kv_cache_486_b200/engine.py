@@ -38,9 +38,20 @@ class PagedKVCache:
         """Slots (host int64) for n new tokens; runs the block copy a copy-on-write needs."""
         slots, cow = self.pool.pa_alloc(seq_id, n)
         if len(cow):
-            pairs = torch.from_numpy(cow).to(self.device, non_blocking=False)
-            pa_copy_blocks([self.k_cache], [self.v_cache], pairs, self.dev_error, stream)
+            self._copy_pairs(torch.from_numpy(cow).to(self.device, non_blocking=False), stream)
         return slots, cow
+
+    def alloc_tokens(self, seq_id, token_ids, stream=None):
+        """pa_alloc_tokens (prefix-cache reuse for a new sequence when the pool has it on)
+        + the block copy a copy-on-write needs -> (slots with -1 for cached tokens,
+        cow pairs, n_cached)."""
+        slots, cow, n_cached = self.pool.pa_alloc_tokens(seq_id, token_ids)
+        if len(cow):
+            self._copy_pairs(torch.from_numpy(cow).to(self.device, non_blocking=False), stream)
+        return slots, cow, n_cached
+
+    def _copy_pairs(self, pairs, stream=None):
+        pa_copy_blocks([self.k_cache], [self.v_cache], pairs, self.dev_error, stream)
 
     def fork(self, parent, child):
         self.pool.pa_fork(parent, child)
@@ -116,12 +127,8 @@ class PagedKVCacheInt8(PagedKVCache):
         ws = pa_decode_workspace_size(max_batch, num_q_heads, num_kv_heads, head_dim)
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
 
-    def alloc(self, seq_id, n, stream=None):
-        slots, cow = self.pool.pa_alloc(seq_id, n)
-        if len(cow):
-            pairs = torch.from_numpy(cow).to(self.device, non_blocking=False)
-            pa_copy_blocks([self.k_pool], [self.v_pool], pairs, self.dev_error, stream)
-        return slots, cow
+    def _copy_pairs(self, pairs, stream=None):
+        pa_copy_blocks([self.k_pool], [self.v_pool], pairs, self.dev_error, stream)
 
     def write(self, key, value, slots, stream=None):
         if not isinstance(slots, torch.Tensor):

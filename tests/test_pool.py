@@ -235,3 +235,102 @@ def test_swap_matches_the_oracle():
                 del where[s]
             _same_state(pd, od, nd, sorted(s for s, w in where.items() if w == "d"), nd + 1)
             _same_state(ph, oh, nh, sorted(s for s, w in where.items() if w == "h"), nh + 1)
+
+
+def _prefix_state(p, o, nb, seqs):
+    _same_state(p, o, nb, seqs, nb + 1)
+    assert p.pa_num_cached_blocks() == o.num_cached()
+    assert p.pa_num_evictable_blocks() == o.num_releasable()
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_prefix_cache_scripts_match_the_oracle(seed):
+    """Prompts sharing system prompts (pa_alloc_tokens), growth with and without
+    ids, batches, forks, frees, swaps and toggles: every status, slot, copy pair,
+    cached-token count, table and counter equals the oracle's."""
+    rng = np.random.default_rng(100 + seed)
+    bs = int(rng.choice([1, 2, 4, 16]))
+    nb = int(rng.integers(8, 60))
+    p, o = pa.Pool(nb, bs), oracle.Pool(nb, bs)
+    hp, ho = pa.Pool(nb, bs), oracle.Pool(nb, bs)  # a second pool to swap into
+    p.pa_set_prefix_caching(True)
+    o.set_prefix_caching(True)
+    systems = [list(rng.integers(0, 4, size=int(rng.integers(1, 3 * bs + 3)))) for _ in range(3)]
+    live, away, nxt, hits = set(), set(), 0, 0
+    for step in range(300):
+        r = rng.random()
+        if r < 0.35 or not live:
+            ids = systems[int(rng.integers(0, 3))] + list(
+                rng.integers(0, 4, size=int(rng.integers(0, 2 * bs + 2))))
+            ids = np.array(ids or [1], dtype=np.int32)
+            st_o, slots_o, cow_o, cached_o = o.alloc_tokens(nxt, ids)
+            try:
+                slots_p, cow_p, cached_p = p.pa_alloc_tokens(nxt, ids)
+                assert st_o == oracle.OK
+                assert np.array_equal(slots_p, slots_o) and np.array_equal(cow_p, cow_o)
+                assert cached_p == cached_o
+                hits += cached_p
+                live.add(nxt)
+            except pa.PagedAttnError as e:
+                assert st_o == oracle.OOM and e.status == pa.PA_ERR_OOM
+            nxt += 1
+        elif r < 0.55:
+            s = int(rng.choice(sorted(live)))
+            if rng.random() < 0.8:
+                ids = np.array(rng.integers(0, 4, size=int(rng.integers(1, bs + 2))), np.int32)
+                st_o, slots_o, cow_o, cached_o = o.alloc_tokens(s, ids)
+                try:
+                    slots_p, cow_p, cached_p = p.pa_alloc_tokens(s, ids)
+                    assert st_o == oracle.OK and cached_p == cached_o == 0
+                    assert np.array_equal(slots_p, slots_o) and np.array_equal(cow_p, cow_o)
+                except pa.PagedAttnError as e:
+                    assert st_o == oracle.OOM and e.status == pa.PA_ERR_OOM
+            elif o.num_free() >= 2 * 3:  # growth without ids: a batch that fits
+                ids_b = sorted(live)[: int(rng.integers(1, 4))]
+                exp = []
+                for sid in ids_b:
+                    exp.append(o.alloc(sid, 1))
+                try:
+                    slots_p, cow_p = p.pa_alloc_batch(ids_b, 1)
+                    assert all(e[0] == oracle.OK for e in exp)
+                    assert np.array_equal(slots_p, np.concatenate([e[1] for e in exp]))
+                except pa.PagedAttnError as e:  # cannot happen: at most 2 blocks each
+                    raise AssertionError(f"batch failed: {e}")
+        elif r < 0.65:
+            par = int(rng.choice(sorted(live)))
+            assert o.fork(par, nxt) == oracle.OK
+            p.pa_fork(par, nxt)
+            live.add(nxt)
+            nxt += 1
+        elif r < 0.72 and live:
+            s = int(rng.choice(sorted(live)))
+            st_o, pairs_o = oracle.swap(o, ho, s)
+            try:
+                pairs_p = pa.pa_swap(p, hp, s)
+                assert st_o == oracle.OK and np.array_equal(pairs_p, pairs_o)
+                live.discard(s)
+                away.add(s)
+            except pa.PagedAttnError as e:
+                assert st_o == oracle.OOM and e.status == pa.PA_ERR_OOM
+        elif r < 0.75 and away:
+            s = int(rng.choice(sorted(away)))
+            st_o, pairs_o = oracle.swap(ho, o, s)
+            try:
+                pairs_p = pa.pa_swap(hp, p, s)
+                assert st_o == oracle.OK and np.array_equal(pairs_p, pairs_o)
+                away.discard(s)
+                live.add(s)
+            except pa.PagedAttnError as e:
+                assert st_o == oracle.OOM and e.status == pa.PA_ERR_OOM
+        elif r < 0.76:
+            on = bool(rng.random() < 0.7)
+            p.pa_set_prefix_caching(on)
+            o.set_prefix_caching(on)
+        else:
+            s = int(rng.choice(sorted(live)))
+            assert o.free(s) == oracle.OK
+            p.pa_free(s)
+            live.discard(s)
+        _prefix_state(p, o, nb, sorted(live))
+        _prefix_state(hp, ho, nb, sorted(away))
+    assert hits > 0

@@ -340,6 +340,82 @@ def custom(name="custom", dtype="f16", B=6, Hq=8, Hkv=2, D=128, bs=16, ctx=None,
                    shuffle=shuffle)
 
 
+# ------------------------------------------------------------ prompt sets
+def token_rows(seed: int, kind: int, ids, positions, Hkv: int, D: int, dtype: str,
+               device="cpu") -> torch.Tensor:
+    """[n, Hkv, D] key (kind 0) or value (kind 1) rows of tokens with the given ids at
+    the given positions.  A function of (id, position) only, so two sequences that
+    begin with the same tokens have the same rows there -- what reusing a cached
+    prefix block assumes."""
+    ids = torch.as_tensor(np.asarray(ids, dtype=np.int64), device=device)
+    pos = torch.as_tensor(np.asarray(positions, dtype=np.int64), device=device)
+    per = Hkv * D
+    key = stream_key(seed, kind, 0x7072656669)
+    idx = ((ids << 24) | pos)[:, None] * per + torch.arange(per, dtype=torch.int64, device=device)
+    return values(key, idx.reshape(-1)).to(TORCH_DTYPE[dtype]).view(len(ids), Hkv, D)
+
+
+@dataclass
+class PromptSet:
+    """Requests that begin with one of a few shared system prompts, each followed by
+    its own user tokens (token ids drawn from a vocabulary)."""
+    name: str
+    dtype: str
+    Hq: int
+    Hkv: int
+    D: int
+    bs: int
+    num_blocks: int
+    seed: int
+    prompts: list = field(default_factory=list)   # int32 token-id arrays, one per request
+    system_of: list = field(default_factory=list)  # system prompt index of each request
+
+    @property
+    def B(self):
+        return len(self.prompts)
+
+    @property
+    def G(self):
+        return self.Hq // self.Hkv
+
+    @property
+    def scale(self):
+        return 1.0 / math.sqrt(self.D)
+
+    def rows(self, i: int, kind: int, device="cpu") -> torch.Tensor:
+        ids = self.prompts[i]
+        return token_rows(self.seed, kind, ids, np.arange(len(ids)), self.Hkv, self.D,
+                          self.dtype, device)
+
+    def q(self, device="cpu") -> torch.Tensor:
+        n = self.B * self.Hq * self.D
+        return _gen(stream_key(self.seed, KIND_Q, 0), 0, n, device, self.dtype).view(
+            self.B, self.Hq, self.D)
+
+
+def prompt_set(name="prompts", dtype="f16", n_systems=3, system_lens=(100, 257, 64),
+               n_requests=24, user_len=(1, 300), vocab=1000, Hq=32, Hkv=8, D=128, bs=16,
+               seed=4865, slack_blocks=0) -> PromptSet:
+    rng = np.random.default_rng(seed)
+    lens = [system_lens[k % len(system_lens)] for k in range(n_systems)]
+    systems = [rng.integers(0, vocab, size=n).astype(np.int32) for n in lens]
+    prompts, system_of = [], []
+    for _ in range(n_requests):
+        k = int(rng.integers(0, n_systems))
+        user = rng.integers(0, vocab, size=int(rng.integers(user_len[0], user_len[1] + 1)))
+        prompts.append(np.concatenate([systems[k], user.astype(np.int32)]))
+        system_of.append(k)
+    need = sum((len(p) + bs - 1) // bs for p in prompts)
+    return PromptSet(name, dtype, Hq, Hkv, D, bs, need + slack_blocks, seed, prompts, system_of)
+
+
+def prefix_prompts(seed=4865):
+    """Llama-3-8B heads (32 / 8, d128, fp16, bs16): 512 requests over 16 shared
+    system prompts of 1024 tokens, each with U[16, 256] own tokens."""
+    return prompt_set("prefix_prompts", "f16", n_systems=16, system_lens=(1024,),
+                      n_requests=512, user_len=(16, 256), vocab=32000, seed=seed)
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama3_8b": llama3_8b,
