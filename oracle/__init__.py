@@ -52,6 +52,11 @@ def lib():
         L.orc_alloc.argtypes = [P, C.c_int64, C.c_int32, P, P, P]
         L.orc_alloc_tokens.restype = C.c_int
         L.orc_alloc_tokens.argtypes = [P, C.c_int64, P, C.c_int32, P, P, P, P]
+        L.orc_paged_prefill_attention.restype = C.c_int
+        L.orc_paged_prefill_attention.argtypes = [P, P, P, P, P, P, C.c_int32, C.c_int32,
+                                                  C.c_int32, C.c_int32, C.c_int32, C.c_int32,
+                                                  C.c_double, C.c_int, P, P, C.c_int64,
+                                                  C.c_int32]
         L.orc_set_prefix_caching.restype = None
         L.orc_set_prefix_caching.argtypes = [P, C.c_int32]
         L.orc_num_cached.restype = C.c_int32
@@ -319,6 +324,29 @@ def reshape_and_cache_int8(key, value, cache, slots, dtype):
                                             _ptr(cache.ks), _ptr(cache.vs), _ptr(slots), T, Hkv,
                                             D, cache.k.shape[2], cache.k.shape[0],
                                             DTYPE_CODE[dtype])
+
+
+def paged_prefill_attention(q, k_cache, v_cache, tables, ctx, query_start, scale, dtype,
+                            rows=None, n_threads=None):
+    """Causal attention of each sequence's new tokens (the last query_start[b+1] -
+    query_start[b] of its ctx[b] tokens) over its cached keys and values.
+    q [total_q, Hq, D] storage bits; fp64 output [total_q, Hq, D] (rows: flat
+    token * Hq + head indices to compute, others NaN)."""
+    q = np.ascontiguousarray(q)
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    tables = _c(tables, np.int32)
+    ctx = _c(ctx, np.int32)
+    qs = _c(query_start, np.int32)
+    out = np.full((T, Hq, D), np.nan)
+    r = None if rows is None else _c(rows, np.int64)
+    st = lib().orc_paged_prefill_attention(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(tables), _ptr(ctx), _ptr(qs), len(ctx), Hq,
+        Hkv, D, bs, tables.shape[1], float(scale), DTYPE_CODE[dtype], _ptr(out), _ptr(r),
+        0 if r is None else len(r), n_threads or (os.cpu_count() or 1))
+    if st != OK:
+        raise ValueError(f"oracle prefill attention rejected its arguments ({st})")
+    return out
 
 
 def paged_decode_attention_int8(q, cache, tables, ctx, scale, dtype, rows=None, n_threads=None):

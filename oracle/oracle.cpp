@@ -729,6 +729,64 @@ int orc_paged_decode_attention(const void* q, const void* k_cache, const void* v
   return ORC_OK;
 }
 
+// Paged prefill (and chunked prefill) attention.  [P4] mentions serving the
+// prompt phase over the same paged cache; the pages print no formula.
+// Reading: sequence b has n_b = query_start[b + 1] - query_start[b] new tokens,
+// the last n_b of its ctx[b] tokens (their keys and values already written);
+// new token i sits at position p = ctx[b] - n_b + i and attends causally, to
+// every token j <= p of the sequence:
+//   out[query_start[b] + i, h] = sum_{j <= p} softmax_j(scale q . K_b[j, g]) V_b[j, g]
+// with g = h / (q_heads / kv_heads).  A single new token (n_b = 1) is decode.
+//   q, out  [total_q, q_heads, head_dim]   (out fp64)
+//   query_start [batch + 1] int32 (non-decreasing, starts at 0)
+// Only the listed rows (flat (token, head) indices) are computed when rows != NULL.
+int orc_paged_prefill_attention(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* tables, const int32_t* ctx,
+                                const int32_t* query_start, int32_t batch, int32_t q_heads,
+                                int32_t kv_heads, int32_t head_dim, int32_t block_size,
+                                int32_t max_blocks, double scale, int dtype, double* out,
+                                const int64_t* rows, int64_t n_rows, int32_t n_threads) {
+  if (kv_heads <= 0 || q_heads % kv_heads != 0) return ORC_INVALID;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t n_new = query_start[b + 1] - query_start[b];
+    if (n_new < 0 || n_new > ctx[b]) return ORC_INVALID;
+  }
+  const int32_t group = q_heads / kv_heads, D = head_dim, bs = block_size;
+  const int64_t total_q = query_start[batch];
+  const int64_t total = rows ? n_rows : total_q * q_heads;
+  auto one = [&](int64_t row) {
+    const int64_t t = row / q_heads;
+    const int32_t h = static_cast<int32_t>(row % q_heads);
+    int32_t b = 0;
+    while (query_start[b + 1] <= t) ++b;  // the sequence that owns token t
+    const int64_t i = t - query_start[b];
+    const int64_t n_new = query_start[b + 1] - query_start[b];
+    const int64_t p = ctx[b] - n_new + i;  // position of the token
+    const int32_t g = h / group;
+    const int64_t n = p + 1;  // keys 0 .. p
+    std::vector<double> qq(D), kk(n * D), vv(n * D);
+    for (int32_t d = 0; d < D; ++d) qq[d] = load_elem(q, (t * q_heads + h) * D + d, dtype);
+    for (int64_t j = 0; j < n; ++j) {
+      const int64_t blk = tables[static_cast<int64_t>(b) * max_blocks + j / bs];
+      const int64_t base = ((blk * kv_heads + g) * bs + j % bs) * D;
+      for (int32_t d = 0; d < D; ++d) {
+        kk[j * D + d] = load_elem(k_cache, base + d, dtype);
+        vv[j * D + d] = load_elem(v_cache, base + d, dtype);
+      }
+    }
+    attend_one(qq.data(), kk.data(), vv.data(), n, D, scale, out + row * D);
+  };
+  if (n_threads < 1) n_threads = 1;
+  std::vector<std::thread> pool;
+  for (int32_t th = 0; th < n_threads; ++th) {
+    pool.emplace_back([&, th]() {
+      for (int64_t k = th; k < total; k += n_threads) one(rows ? rows[k] : k);
+    });
+  }
+  for (auto& x : pool) x.join();
+  return ORC_OK;
+}
+
 // Paged attention over an INT8 cache: the gather reads code * scale (exact in
 // fp64), then the same definition as above.  q / out as in the paged form.
 int orc_paged_decode_attention_int8(const void* q, const int8_t* k_codes, const int8_t* v_codes,

@@ -340,6 +340,42 @@ def custom(name="custom", dtype="f16", B=6, Hq=8, Hkv=2, D=128, bs=16, ctx=None,
                    shuffle=shuffle)
 
 
+# --------------------------------------------------------------- prefill
+def prefill(name, dtype, Hq, Hkv, D, bs, ctx, n_new, seed, slack=8) -> Workload:
+    """Sequences of ctx[b] cached tokens whose last n_new[b] are the new chunk being
+    prefilled (n_new = ctx: a whole prompt; n_new < ctx: chunked prefill on top of
+    earlier context).  The chunk's keys and values are in the cache, written by the
+    op script like every other token; `q_prefill` gives the chunk's queries
+    [sum n_new, Hq, D] and `query_start` their offsets."""
+    wl = _simple(name, dtype, len(ctx), Hq, Hkv, D, bs, ctx, seed, slack=slack, shuffle=True)
+    wl.n_new = np.asarray(n_new, dtype=np.int32)
+    assert np.all(wl.n_new <= wl.context_lens()) and np.all(wl.n_new >= 0)
+    return wl
+
+
+def query_start(wl) -> np.ndarray:
+    return np.concatenate([[0], np.cumsum(wl.n_new)]).astype(np.int32)
+
+
+def q_prefill(wl, device="cpu") -> torch.Tensor:
+    T = int(wl.n_new.sum())
+    n = T * wl.Hq * wl.D
+    return _gen(stream_key(wl.seed, KIND_Q, 1), 0, n, device, wl.dtype).view(T, wl.Hq, wl.D)
+
+
+def prefill_8b(seed=4866):
+    """Llama-3-8B heads (32 / 8, d128, fp16, bs16): 8 whole prompts of 2048 tokens."""
+    return prefill("prefill_8b", "f16", 32, 8, 128, 16, [2048] * 8, [2048] * 8, seed)
+
+
+def chunked_8b(seed=4867):
+    """Llama-3-8B heads, fp16, bs16: 16 sequences with U[1024, 8192] tokens whose last
+    512 are the chunk being prefilled on top of the earlier context."""
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(1024, 8193, size=16)
+    return prefill("chunked_8b", "f16", 32, 8, 128, 16, ctx, [512] * 16, seed)
+
+
 # ------------------------------------------------------------ prompt sets
 def token_rows(seed: int, kind: int, ids, positions, Hkv: int, D: int, dtype: str,
                device="cpu") -> torch.Tensor:
