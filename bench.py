@@ -55,6 +55,16 @@ def _peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _peak_tensor():
+    """Dense fp16/bf16 tensor peak (burst): measured bf16 (fp16 has the same nominal rate)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16 (fp16 nominal ratio 1)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
 def _kernel_sha():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_486_b200", "csrc")
@@ -635,6 +645,70 @@ def run_prefix(args, dist, rank, world):
     }
 
 
+def run_prefill(args, dist, rank, world):
+    """Paged prefill attention over the pool: whole prompts (prefill_8b) or a 512-token
+    chunk after earlier context (chunked_8b, --config chunked_8b)."""
+    import paged_kv_cache_486_b200 as pa
+    from paged_kv_cache_486_b200.engine import PagedKVCache
+    name = args.config if args.config in ("prefill_8b", "chunked_8b") else "prefill_8b"
+    wl = {"prefill_8b": workloads.prefill_8b, "chunked_8b": workloads.chunked_8b}[name]()
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda")
+    eng.apply_ops(wl.ops, lambda s_, p_, n_: (wl.tokens(s_, p_, n_, 0, "cuda"),
+                                             wl.tokens(s_, p_, n_, 1, "cuda")))
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    qsn = workloads.query_start(wl)
+    qs = torch.from_numpy(qsn).cuda()
+    q = workloads.q_prefill(wl, "cuda")
+    out = torch.empty_like(q)
+    max_q = int(wl.n_new.max())
+    flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
+                                eng.dev_error)
+
+    ms = []
+    for it in range(args.warmup + args.steps):
+        _flush_l2(flush)
+        e0.record(stream)
+        run()
+        e1.record(stream)
+        e1.synchronize()
+        if it >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert eng.device_errors() == 0, "device guards fired"
+    c = wl.context_lens().astype(np.int64)
+    n = wl.n_new.astype(np.int64)
+    # keys attended: new token i of sequence b attends ctx - n + i + 1 keys
+    pairs = int(((c - n) * n + n * (n + 1) // 2).sum())
+    flops = 4.0 * wl.D * wl.Hq * pairs
+    t = statistics.mean(ms) / 1e3
+    tflops = flops / t / 1e12
+    peak, kind = _peak_tensor()
+    tokens = int(n.sum())
+    total_ms, _, value = aggregate(dist, sum(ms), tokens * args.steps)
+    kv_bytes = int(c.sum()) * wl.Hkv * wl.D * 2 * wl.elem_bytes
+    return {
+        "metric": "paged prefill attention: new tokens/s", "op": "prefill", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded counter-based N(0,1) stand-in values, shuffled block pool)",
+        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+                   "head_dim": wl.D, "block_size": wl.bs, "new_tokens": tokens,
+                   "context_tokens": int(c.sum()), "attended_pairs": pairs,
+                   "l2": "flushed between timed calls (256 MiB read outside the events)"},
+        "prefill_us": 1e3 * statistics.mean(ms), "kv_read_bytes": kv_bytes,
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "peak_source": kind, "traffic": None,
+                     "timed": "pa_prefill_attention (one kernel, mma.sync m16n8k16)"},
+        "gpu_launches": args.steps,
+    }
+
+
 # ---------------------------------------------------------- oracle timings
 def cpu_baseline(wl, target_s=10.0):
     import oracle
@@ -719,9 +793,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--op", default="step", choices=["step", "swap", "int8", "prefix"],
+    ap.add_argument("--op", default="step",
+                    choices=["step", "swap", "int8", "prefix", "prefill"],
                     help="step: the decode step (default); swap: eviction to host and back; "
-                         "int8: the decode step over an INT8 cache; prefix: prefix caching")
+                         "int8: the decode step over an INT8 cache; prefix: prefix caching; "
+                         "prefill: paged prefill attention (--config prefill_8b | chunked_8b)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
@@ -740,7 +816,8 @@ def main():
     torch.cuda.set_device(local)
     dist, rank, world = _dist()
     try:
-        run = {"swap": run_swap, "int8": run_int8, "prefix": run_prefix}.get(args.op, run_ours)
+        run = {"swap": run_swap, "int8": run_int8, "prefix": run_prefix,
+               "prefill": run_prefill}.get(args.op, run_ours)
         line = run(args, dist, rank, world)
         if rank == 0:
             print(json.dumps(line), flush=True)

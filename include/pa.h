@@ -12,6 +12,8 @@
  *       PagedAttention work?".
  *  [P3] "The KV cache and PagedAttention: why the LLM server chokes at 10 users",
  *       the serving example and "The trade-offs".
+ *  [P4] "What is PagedAttention and what did it change in LLM serving",
+ *       "What is PagedAttention, simply".
  *  [P5] "KV Cache for intermediates: why long context eats the GPU and how to cut
  *       it 4x", sections "The precise scientific definition" and "The four
  *       solutions".
@@ -340,6 +342,35 @@ pa_status pa_decode_attention_static_ws(void* out, const void* q, const void* k_
 pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                          int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* path_out,
                          int32_t* num_workers_out);
+
+/* ------------------------------------------------------------------------
+ * Paged prefill / chunked-prefill attention.  [P4] "What is PagedAttention,
+ * simply": the prompt phase runs over the same paged cache.  Reading (the
+ * pages print no formula): sequence b has n_b = query_start[b + 1] -
+ * query_start[b] new tokens, the last n_b of its context_lens[b] tokens, whose
+ * keys and values are already in the cache (written by pa_reshape_and_cache);
+ * new token i at position p = context_lens[b] - n_b + i attends causally:
+ *   out[t, h] = sum_{j <= p} softmax_j(scale q[t, h] . K_b[j, g]) V_b[j, g],
+ * t = query_start[b] + i, g = h / (num_q_heads / num_kv_heads).  n_b equal to
+ * the context is a whole prompt, smaller a chunk after earlier context, 1 is
+ * decode.
+ * q, out: [total_q, num_q_heads, head_dim], fp16 or bf16; out is rounded once
+ *   from fp32 accumulators.
+ * query_start: [batch + 1] int32, device, non-decreasing from 0; every n_b <=
+ *   max_q (the host's bound, which sizes the launch), n_b <= context_lens[b] and
+ *   query_start[b + 1] <= total_q, else the sequence is skipped (its rows of out
+ *   untouched) and PA_DEVERR_BAD_CTX is set.
+ * head_dim 64 or 128; num_q_heads / num_kv_heads a divisor of 64; block_size a
+ * multiple of 16; batch <= 65535.  Tensor cores (mma.sync), 64 (token, head)
+ * rows of one kv head per CTA, K / V tiles of 64 keys by TMA, one launch.
+ * ---------------------------------------------------------------------- */
+pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, const int32_t* query_start,
+                               int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
+                               pa_dtype dtype, int32_t* dev_error, pa_stream stream);
 
 /* ------------------------------------------------------------------------
  * INT8 KV cache.  [P5] "The four solutions", KV-cache quantisation: keys and

@@ -59,6 +59,8 @@ SIGNATURES = {
                                       _I32, _I32, _P]),
     "pa_decode_attention_static_ws": (_I32, [_P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32,
                                              _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
+    "pa_prefill_attention": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                    _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
     "pa_int8_block_bytes": (C.c_size_t, [_I32, _I32, _I32]),
     "pa_reshape_and_cache_int8": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                          C.c_int, _P, _P]),
@@ -330,6 +332,27 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, contex
         float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32),
         _stream(stream))
     _check(st, "pa_decode_attention_static_ws")
+
+
+def pa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
+                         max_q, scale, dev_error=None, stream=None):
+    """Causal attention of each sequence's new tokens over its paged cache: q/out
+    [T, Hq, D] fp16 or bf16, query_start int32 [B+1] (device), max_q >= every
+    query_start[b+1] - query_start[b]; caches and tables as pa_decode_attention."""
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    B = context_lens.shape[0]
+    MB = block_tables.shape[1]
+    if out.shape != q.shape or query_start.shape[0] != B + 1:
+        raise ValueError("out must have q's shape and query_start batch + 1 entries")
+    st = lib.pa_prefill_attention(
+        _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache", q.dtype),
+        _dev_ptr(v_cache, "v_cache", q.dtype), _dev_ptr(block_tables, "block_tables", torch.int32),
+        _dev_ptr(context_lens, "context_lens", torch.int32),
+        _dev_ptr(query_start, "query_start", torch.int32), B, Hq, Hkv, D, bs, NB, MB, T, int(max_q),
+        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32),
+        _stream(stream))
+    _check(st, "pa_prefill_attention")
 
 
 INT8_RECORD_BYTES = 2112  # one 16-token group of one (block, kv head): codes + fp32 scales

@@ -13,6 +13,7 @@
 #include "decode_launch.h"
 #include "host_common.h"
 #include "int8_launch.h"
+#include "prefill_launch.h"
 
 namespace {
 
@@ -525,6 +526,71 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
                                                (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0,
                                                static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_decode_attention_int8 (decode kernel)");
+}
+
+pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, const int32_t* query_start,
+                               int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
+                               pa_dtype dtype, int32_t* dev_error, pa_stream stream) {
+  if (dtype != PA_F16 && dtype != PA_BF16)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: dtype must be fp16 or bf16");
+  if (total_q < 0) return fail(PA_ERR_INVALID, "pa_prefill_attention: negative total_q");
+  if (batch < 0 || batch > 65535)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: batch %d outside [0, 65535]", batch);
+  if (num_kv_heads < 1 || num_kv_heads > 65535 || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads || 64 % (num_q_heads / num_kv_heads))
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: num_q_heads %d / num_kv_heads %d must be "
+                "a divisor of 64", num_q_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: head_dim %d not in {64, 128}", head_dim);
+  if (block_size < 16 || block_size % 16 || block_size > 1024)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: block_size %d must be a multiple of 16",
+                block_size);
+  if (num_blocks < 0 || max_blocks < 0 || max_q < 0)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: negative size");
+  const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  if (rows >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(max_blocks) * block_size >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: pool or table too large");
+  const int group = num_q_heads / num_kv_heads;
+  if ((static_cast<int64_t>(max_q) * group + 63) / 64 > INT32_MAX)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: max_q too large");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_prefill_attention: scale is NaN");
+  if (batch == 0 || max_q == 0 || total_q == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: NULL pointer");
+  if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: misaligned pointer");
+  CUtensorMap kmap, vmap;
+  bool k3 = false, v3 = false;
+  if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
+      !tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || k3 != v3)
+    return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
+  pa::PrefillArgs a;
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start;
+  a.dev_error = dev_error;
+  a.batch = batch;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = num_kv_heads;
+  a.group = group;
+  a.head_dim = head_dim;
+  a.block_size = block_size;
+  a.num_blocks = num_blocks;
+  a.max_blocks = max_blocks;
+  a.max_q = max_q;
+  a.total_q = total_q;
+  a.three_d = k3 ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
 }
 
 pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {

@@ -12,7 +12,7 @@ import torch
 
 from . import (INT8_RECORD_BYTES, PA_PATH_AUTO, Pool, pa_check_device_error, pa_copy_blocks,
                pa_decode_attention, pa_decode_attention_int8, pa_decode_workspace_size,
-               pa_reshape_and_cache, pa_reshape_and_cache_int8)
+               pa_prefill_attention, pa_reshape_and_cache, pa_reshape_and_cache_int8)
 
 
 class PagedKVCache:
@@ -96,6 +96,15 @@ class PagedKVCache:
             out = torch.empty_like(q)
         pa_decode_attention(out, q, self.k_cache, self.v_cache, block_tables, context_lens, scale,
                             self.workspace, self.dev_error, path, num_workers, flags, stream)
+        return out
+
+    def prefill(self, q, block_tables, context_lens, query_start, max_q, scale, out=None,
+                stream=None):
+        """Causal attention of each sequence's new tokens (already written) over the cache."""
+        if out is None:
+            out = torch.empty_like(q)
+        pa_prefill_attention(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
+                             query_start, max_q, scale, self.dev_error, stream)
         return out
 
     def device_errors(self, stream=None):

@@ -1,0 +1,130 @@
+"""Paged prefill / chunked-prefill attention on the GPU against the oracle: every
+row within the fp16/bf16 bound on small cases (whole prompts, chunks after
+earlier context, single new tokens, ragged tiles), sampled rows at full size,
+and the guards (empty chunks, lengths the launch does not cover, bad block ids)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import paged_kv_cache_486_b200 as pa
+from gpu_side import NAN_BITS, tol_ok
+from oracle_side import raw, run_script
+from paged_kv_cache_486_b200.engine import PagedKVCache
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_cuda(cuda_ok):
+    yield
+
+
+def _build(wl):
+    dt = workloads.TORCH_DTYPE[wl.dtype]
+    eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda",
+                       fill_bits=NAN_BITS[wl.dtype])
+    eng.apply_ops(wl.ops, lambda s, p, n: (wl.tokens(s, p, n, 0, "cuda"),
+                                           wl.tokens(s, p, n, 1, "cuda")))
+    bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
+    qs = torch.from_numpy(workloads.query_start(wl)).cuda()
+    q = workloads.q_prefill(wl, "cuda")
+    torch.cuda.synchronize()
+    return eng, bt, ctx, qs, q
+
+
+def _cases():
+    P = workloads.prefill
+    return {
+        "f16_g4_d128": lambda: P("a", "f16", 32, 8, 128, 16, [1, 17, 64, 300, 700, 90],
+                                 [1, 17, 30, 120, 700, 90], 31),
+        "bf16_g8_d128": lambda: P("b", "bf16", 64, 8, 128, 16, [40, 129, 513, 1000],
+                                  [40, 1, 200, 513], 32),
+        "f16_g1_bs32": lambda: P("c", "f16", 8, 8, 128, 32, [33, 97, 400], [33, 60, 5], 33),
+        "bf16_g2_d64_bs64": lambda: P("d", "bf16", 4, 2, 64, 64, [65, 300, 777], [64, 300, 100],
+                                      34),
+        "f16_mqa_g16": lambda: P("e", "f16", 16, 1, 128, 16, [5, 250, 999], [5, 250, 31], 35),
+        "f16_g64_d64": lambda: P("f", "f16", 64, 1, 64, 16, [7, 90], [7, 45], 36),
+    }
+
+
+CASES = _cases()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_small_configs_match_the_oracle(name):
+    wl = CASES[name]()
+    eng, bt, ctx, qs, q = _build(wl)
+    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale)
+    torch.cuda.synchronize()
+    o = run_script(wl)
+    ref = oracle.paged_prefill_attention(raw(q), o["k_cache"], o["v_cache"], o["table"],
+                                         o["ctx"], workloads.query_start(wl), wl.scale, wl.dtype)
+    ok, worst = tol_ok(out.double().cpu().numpy(), ref, wl.dtype)
+    assert ok, f"worst error / bound = {worst:.3f}"
+    assert eng.device_errors() == 0
+    # a larger max_q only launches more (empty) tiles
+    again = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()) + 100, wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["prefill_8b", "chunked_8b"])
+def test_prefill_full_size_sampled_rows(name):
+    wl = {"prefill_8b": workloads.prefill_8b, "chunked_8b": workloads.chunked_8b}[name]()
+    eng, bt, ctx, qs, q = _build(wl)
+    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    o = run_script(wl, with_cache=False)
+    assert np.array_equal(bt.cpu().numpy(), o["table"])
+    # sampled rows: first, last and random new tokens of a few sequences, the oracle
+    # reading the same cache rows (built from the script on the CPU)
+    rng = np.random.default_rng(4869)
+    qsn = workloads.query_start(wl)
+    rows = []
+    for b in sorted(rng.choice(wl.B, size=3, replace=False)):
+        toks = {int(qsn[b]), int(qsn[b + 1]) - 1} | set(
+            int(x) for x in rng.integers(qsn[b], qsn[b + 1], size=3))
+        for t in sorted(toks):
+            for h in rng.choice(wl.Hq, size=2, replace=False):
+                rows.append(t * wl.Hq + int(h))
+    full = run_script(wl)
+    ref = oracle.paged_prefill_attention(raw(q), full["k_cache"], full["v_cache"],
+                                         full["table"], full["ctx"], qsn, wl.scale, wl.dtype,
+                                         rows=rows)
+    got = out.double().cpu().numpy().reshape(-1, wl.D)[rows]
+    ok, worst = tol_ok(got, ref.reshape(-1, wl.D)[rows], wl.dtype)
+    assert ok, f"worst error / bound = {worst:.3f}"
+    assert eng.device_errors() == 0
+
+
+def test_prefill_guards():
+    wl = CASES["f16_g4_d128"]()
+    eng, bt, ctx, qs, q = _build(wl)
+    ref = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale).clone()
+    torch.cuda.synchronize()
+    # a chunk longer than max_q: that sequence is skipped and reported; others unchanged
+    out = torch.zeros_like(q)
+    eng.prefill(q, bt, ctx, qs, 200, wl.scale, out=out)
+    torch.cuda.synchronize()
+    assert eng.device_errors() & pa.PA_DEVERR_BAD_CTX
+    qsn = workloads.query_start(wl)
+    for b in range(wl.B):
+        seg = slice(int(qsn[b]), int(qsn[b + 1]))
+        if wl.n_new[b] <= 200:
+            assert torch.equal(out[seg].view(torch.int16), ref[seg].view(torch.int16))
+        else:
+            assert not out[seg].float().any()
+    # an out-of-range block id: reported, its keys skipped, nothing faults
+    bt2 = bt.clone()
+    bt2[3, 2] = wl.num_blocks + 7
+    eng.prefill(q, bt2, ctx, qs, int(wl.n_new.max()), wl.scale)
+    torch.cuda.synchronize()
+    assert eng.device_errors() & pa.PA_DEVERR_BAD_BLOCK
+    # no new tokens anywhere
+    empty = torch.zeros_like(qs)
+    eng.prefill(q[:0], bt, ctx, empty, 0, wl.scale)
+    torch.cuda.synchronize()
+    assert eng.device_errors() == 0

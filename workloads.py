@@ -459,6 +459,8 @@ CONFIGS = {
     "shared_prefix": shared_prefix,
     "long_mha": long_mha,
     "long_mha_bs32": lambda: long_mha(bs=32),
+    "prefill_8b": prefill_8b,
+    "chunked_8b": chunked_8b,
 }
 
 
