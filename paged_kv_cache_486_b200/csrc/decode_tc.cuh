@@ -261,8 +261,25 @@ __device__ __forceinline__ UnitDesc shfl_desc(const UnitDesc& d, int k) {
 }
 
 
+// Warp roles.  A CTA runs kWarps worker (consumer) warps and, paired with
+// each, one producer warp (warp w + kWarps): the producer walks the worker's
+// ranges and issues the copies of its stages into the worker's ring; the
+// worker waits for a stage (the slot's "full" mbarrier, which counts the
+// copied bytes), copies it into registers, releases the slot (its "empty"
+// mbarrier) and computes.  Issue and math overlap instead of alternating in one
+// warp.  Registers: the CTA is launched with kLaunchRegs per thread; producer
+// warpgroups give most of theirs up (setmaxnreg.dec to kProducerRegs), worker
+// warpgroups take them (setmaxnreg.inc to kConsumerRegs).  The two counts add
+// up to twice the launch count, the most the hand-over can provide.
+constexpr int kLaunchRegs = 128;
+constexpr int kConsumerRegs = 216;
+constexpr int kProducerRegs = 40;
+static_assert(kConsumerRegs + kProducerRegs <= 2 * kLaunchRegs, "register split");
+static_assert(kLaunchRegs * kWarps * 2 * 32 <= 65536, "launch registers");
+constexpr int kDone = 64;  // stage metadata: the worker has no more stages
+
 template <typename T, int D, class P>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+__global__ void __launch_bounds__(2 * kWarps * 32, 1)
     decode_tc_kernel(const __grid_constant__ typename P::Maps maps, DecodeArgs a) {
   constexpr int KC = D / 16;  // 16-wide chunks of head_dim
   constexpr int kStages = P::kStages;
@@ -270,97 +287,126 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t ring0 = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (ring0 - raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + P::kRingBytes);
-  StageMeta* meta = reinterpret_cast<StageMeta*>(bars + kWarps * kStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(gbase + P::kRingBytes);
+  uint64_t* empty = full + kWarps * kStages;
+  StageMeta* meta = reinterpret_cast<StageMeta*>(empty + kWarps * kStages);
   int32_t* cum = reinterpret_cast<int32_t*>(meta + kWarps * kStages);
   int32_t* ctx_s = cum + a.batch + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i < kWarps * kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     P::prefetch(maps);
   }
   prefetch_tables(a);
   scan_context(a, cum, ctx_s);  // ends with __syncthreads()
+  // Until here the kernel has read only context_lens and block_tables: with
+  // overlap enabled this prologue runs while the preceding kernel finishes.
+  wait_prior_grid();
+  zero_empty_rows<T>(a, ctx_s);
 
-  // Until wait_prior_grid() below the kernel reads only its inputs
-  // (context_lens, block_tables, q): with overlap enabled this prologue runs
-  // while the preceding kernel (typically the cache write) is still finishing.
   const int B = a.batch, Hkv = a.num_kv_heads, G = a.group, Hq = a.num_q_heads;
-  const int bs = a.block_size;
   const Split sp = make_split(static_cast<int64_t>(Hkv) * cum[B], a.workers);
-  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const bool active = w < sp.W;  // false for every warp when there is no work
+  const int ww = warp % kWarps;  // the worker this warp belongs to
+  const int64_t w = static_cast<int64_t>(blockIdx.x) * kWarps + ww;
+  const bool active = w < sp.W;  // the same for a worker and its producer
+  const uint32_t full0 = smem_u32(&full[ww * kStages]);
+  const uint32_t empty0 = smem_u32(&empty[ww * kStages]);
+  StageMeta* wmeta = meta + ww * kStages;
 
-  const uint32_t bar0 = smem_u32(&bars[warp * kStages]);
-  StageMeta* wmeta = meta + warp * kStages;
-
-  // ---------------- producer state (uniform across the warp) ----------------
-  // The warp walks its range(s) unit by unit; `cur` is the unit being issued.
-  int64_t prange = w;
-  int64_t pr0 = active ? sp.start(w) : 0;
-  int64_t pend = active ? sp.end(w) : 0;
-  int64_t pu = pr0;     // next unit to enter
-  int64_t win = pr0;    // first unit of the descriptor window
-  UnitDesc dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
-  UnitDesc dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
-  UnitDesc cur{-1, 0, 0, 0};
-  int psub = 0, pnsub = 0;
-  bool pdone = !active;
-
-  // Issues the next stage into `slot` (claiming a tail chunk when the current
-  // range is used up); false when there is nothing left to issue.
-  auto produce = [&](int slot) -> bool {
-    if (pdone) return false;
-    if (psub == 0) {
-      if (pu >= pend) {
-        const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
-        if (chunk >= sp.NC) {
-          pdone = true;
-          return false;
+  if (warp >= kWarps) {
+    // =============================== producer ===============================
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (!active) return;
+    int64_t prange = w;
+    int64_t pr0 = sp.start(w);
+    int64_t pend = sp.end(w);
+    int64_t pu = pr0;   // next unit to enter
+    int64_t win = pr0;  // first unit of the descriptor window
+    UnitDesc dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
+    UnitDesc dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+    UnitDesc cur{-1, 0, 0, 0};
+    int psub = 0, pnsub = 0;
+    int k = 0;  // stages issued
+    for (;; ++k) {
+      const int slot = k % kStages;
+      if (k >= kStages) {
+        // the worker must have released this slot's previous stage
+        if (!__all_sync(kFull, mbar_wait_bounded(empty0 + slot * 8, ((k / kStages) - 1) & 1))) {
+          if (lane == 0) report(a.dev_error, PA_DEVERR_TIMEOUT);
+          break;
         }
-        prange = sp.W + chunk;
-        pr0 = pu = win = sp.start(prange);
-        pend = sp.end(prange);
-        dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
-        dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
       }
-      if (pu >= win + 32) {
-        win += 32;
-        dcur = dnext;
-        dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+      bool more = true;
+      if (psub == 0) {
+        if (pu >= pend) {
+          const int64_t chunk = sp.NC ? claim_chunk(a, lane) : sp.NC;
+          if (chunk >= sp.NC) {
+            more = false;
+          } else {
+            prange = sp.W + chunk;
+            pr0 = pu = win = sp.start(prange);
+            pend = sp.end(prange);
+            dcur = unit_desc(a, cum, ctx_s, win + lane, pr0, pend);
+            dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+          }
+        }
+        if (more) {
+          if (pu >= win + 32) {
+            win += 32;
+            dcur = dnext;
+            dnext = unit_desc(a, cum, ctx_s, win + 32 + lane, pr0, pend);
+          }
+          cur = shfl_desc(dcur, static_cast<int>(pu - win));
+          pnsub = ((cur.nf & 0xff) + kTok - 1) / kTok;
+        }
       }
-      cur = shfl_desc(dcur, static_cast<int>(pu - win));
-      pnsub = ((cur.nf & 0xff) + kTok - 1) / kTok;
-    }
-    const int uflags = cur.nf >> 8;
-    const int left = (cur.nf & 0xff) - psub * kTok;
-    const bool ok = cur.id >= 0 && cur.id < a.num_blocks;
-    const int flags = (ok ? kHasData : 0) | (psub == 0 ? uflags & kSegStart : 0) |
-                      (psub + 1 == pnsub ? uflags & kSegEnd : 0) |
-                      (uflags & (kComplete | kFirstInRange | kMoreInRange));
-    if (lane == 0) {
-      const int kvh = cur.bk & 0xffff;
-      wmeta[slot] = StageMeta{cur.bk >> 16, (kvh << 16) | flags, left < kTok ? left : kTok,
-                              static_cast<int32_t>(prange)};
-      const uint32_t bar = bar0 + slot * 8;
-      if (ok) {
-        mbar_arrive_expect_tx(bar, P::kStageBytes);
-        P::issue(maps, a, ring0, warp, slot, cur.id * Hkv + kvh, psub * kTok, bar);
-      } else {
-        report(a.dev_error, PA_DEVERR_BAD_BLOCK);
-        mbar_arrive(bar);
+      const uint32_t bar = full0 + slot * 8;
+      if (!more) {
+        if (lane == 0) {
+          wmeta[slot] = StageMeta{0, kDone, 0, 0};
+          mbar_arrive(bar);
+        }
+        ++k;
+        break;
+      }
+      const int uflags = cur.nf >> 8;
+      const int left = (cur.nf & 0xff) - psub * kTok;
+      const bool ok = cur.id >= 0 && cur.id < a.num_blocks;
+      const int flags = (ok ? kHasData : 0) | (psub == 0 ? uflags & kSegStart : 0) |
+                        (psub + 1 == pnsub ? uflags & kSegEnd : 0) |
+                        (uflags & (kComplete | kFirstInRange | kMoreInRange));
+      if (lane == 0) {
+        const int kvh = cur.bk & 0xffff;
+        wmeta[slot] = StageMeta{cur.bk >> 16, (kvh << 16) | flags, left < kTok ? left : kTok,
+                                static_cast<int32_t>(prange)};
+        if (ok) {
+          mbar_arrive_expect_tx(bar, P::kStageBytes);
+          P::issue(maps, a, ring0, ww, slot, cur.id * Hkv + kvh, psub * kTok, bar);
+        } else {
+          report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+          mbar_arrive(bar);
+        }
+      }
+      if (++psub == pnsub) {
+        psub = 0;
+        ++pu;
       }
     }
-    if (++psub == pnsub) {
-      psub = 0;
-      ++pu;
-    }
-    return true;
-  };
+    worker_finished(a, sp.W, lane);
+    // copies still in flight land before the CTA's shared memory goes away
+    for (int i = k - kStages > 0 ? k - kStages : 0; i < k; ++i)
+      mbar_wait_bounded(full0 + (i % kStages) * 8, (i / kStages) & 1);
+    return;
+  }
 
-  // ---------------- consumer state ----------------
+  // ================================ worker ==================================
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+  if (!active) return;
   const int g = lane >> 2, cq = lane & 3;
   uint32_t qf[KC][2], qn[KC][2];
   int qn_b = -1, qn_kvh = -1;
@@ -382,33 +428,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       }
     }
   };
-  if (active) {
-    const UnitDesc d0 = shfl_desc(dcur, 0);
-    qn_b = d0.bk >> 16;
-    qn_kvh = d0.bk & 0xffff;
-    load_q(qn, qn_b, qn_kvh);
-  }
 
-  wait_prior_grid();  // from here on the cache, the output and the workspace are used
-  zero_empty_rows<T>(a, ctx_s);
-  if (!active) return;
-
-  int issued = 0;
-  while (issued < kStages && produce(issued)) ++issued;
-
-  int slot = 0, consumed = 0;
-  uint32_t phases = 0;
-  bool timed_out = false;
-  while (consumed < issued) {
-    const uint32_t bar = bar0 + slot * 8;
+  for (int k = 0;; ++k) {
+    const int slot = k % kStages;
     // all lanes take the same decision, so the warp never splits on a timeout
-    if (!__all_sync(kFull, mbar_wait_bounded(bar, (phases >> slot) & 1u))) {
+    if (!__all_sync(kFull, mbar_wait_bounded(full0 + slot * 8, (k / kStages) & 1))) {
       if (lane == 0) report(a.dev_error, PA_DEVERR_TIMEOUT);
-      timed_out = true;
-      break;
+      // let stages the producer issued after this one land before exiting
+      for (int i = 1; i < kStages; ++i)
+        mbar_wait_bounded(full0 + ((k + i) % kStages) * 8, ((k + i) / kStages) & 1);
+      return;
     }
-    phases ^= 1u << slot;
     const StageMeta md = wmeta[slot];
+    if (md.kvh_flags & kDone) break;
     const int b = md.b, kvh = md.kvh_flags >> 16, flags = md.kvh_flags & 0xffff;
 
     if (flags & kSegStart) {
@@ -447,13 +479,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
 
     const int n_valid = md.n_valid;
     const bool have = (flags & kHasData) != 0;
-    // Move the stage into registers first and hand the slot straight back to
-    // TMA, so the ring keeps loading while this warp computes.
+    // Move the stage into registers and hand the slot straight back.
     typename P::Frag fr;
-    if (have) P::load(a, ring0, warp, slot, n_valid, lane, fr);
+    if (have) P::load(a, ring0, ww, slot, n_valid, lane, fr);
     fence_proxy_async_smem();
     __syncwarp();
-    if (produce(slot)) ++issued;
+    if (lane == 0) mbar_arrive(empty0 + slot * 8);
 
     if (have) {
       // scores of (row g, head 2cq), (g, 2cq+1), (g+8, 2cq), (g+8, 2cq+1), base-2
@@ -540,26 +571,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         piece_done<T, D>(a, cum, b, kvh, sp, lane);
       }
     }
-    slot = slot + 1 == kStages ? 0 : slot + 1;
-    ++consumed;
   }
-
-  if (timed_out) {
-    // let copies already in flight land before the CTA's shared memory goes away
-    for (int k = consumed; k < issued; ++k) {
-      const int s_ = k % kStages;
-      mbar_wait_bounded(bar0 + s_ * 8, (phases >> s_) & 1u);
-      phases ^= 1u << s_;
-    }
-  }
-  worker_finished(a, sp.W, lane);
 }
 
-// Shared memory of one CTA: the rings (1024-aligned), then per stage an
-// mbarrier and a StageMeta, then the context scan (2 * batch + 1 words).
+// Shared memory of one CTA: the rings (1024-aligned), then per stage two
+// mbarriers (full, empty) and a StageMeta, then the context scan (2 * batch + 1
+// words).
 template <class P>
 inline size_t tc_smem_bytes(int batch) {
-  return 1024 + P::kRingBytes + kWarps * P::kStages * (8 + sizeof(StageMeta)) +
+  return 1024 + P::kRingBytes + kWarps * P::kStages * (16 + sizeof(StageMeta)) +
          sizeof(int32_t) * (2 * static_cast<size_t>(batch) + 1);
 }
 
@@ -582,7 +602,7 @@ cudaError_t launch_tc(const DecodeArgs& a, const typename P::Maps& maps, int num
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_ctas);
-  cfg.blockDim = dim3(kWarps * 32);
+  cfg.blockDim = dim3(2 * kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
