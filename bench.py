@@ -186,10 +186,14 @@ def _unique_kv_bytes(wl, table, ctx):
 
 
 # --------------------------------------------------------------- our arm
-def _setup(wl):
+def _setup(wl, extra_blocks=0):
+    """Engine with the workload's pool (plus `extra_blocks` at the bottom of the free
+    stack, so the workload's own allocations get the same block ids) after the
+    prefill ops and the decode step's allocations."""
     from paged_kv_cache_486_b200.engine import PagedKVCache
     dt = workloads.TORCH_DTYPE[wl.dtype]
-    eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda")
+    eng = PagedKVCache(wl.num_blocks + extra_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B,
+                       "cuda")
 
     def tokens(seq, pos0, n):
         return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
@@ -217,7 +221,8 @@ def _setup(wl):
 def run_ours(args, dist, rank, world):
     import paged_kv_cache_486_b200 as pa
     wl = workloads.make(args.config)
-    eng, st = _setup(wl)
+    # room for the end-to-end leg, which grows every sequence by one token per step
+    eng, st = _setup(wl, extra_blocks=wl.B * ((args.warmup + args.steps) // wl.bs + 2))
     flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     n_pairs = st["pairs"].shape[0]
     launches_per_step = 2 + (1 if n_pairs else 0)  # [copy_blocks] + cache write + decode
