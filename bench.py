@@ -673,7 +673,7 @@ def run_prefill(args, dist, rank, world):
 
     def run():
         pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
-                                eng.dev_error)
+                                eng.dev_error, args.prefill_path)
 
     ms = []
     for it in range(args.warmup + args.steps):
@@ -709,7 +709,9 @@ def run_prefill(args, dist, rank, world):
         "prefill_us": 1e3 * statistics.mean(ms), "kv_read_bytes": kv_bytes,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "peak_source": kind, "traffic": None,
-                     "timed": "pa_prefill_attention (one kernel, mma.sync m16n8k16)"},
+                     "timed": "pa_prefill_attention (one kernel, " +
+                              ("mma.sync m16n8k16" if args.prefill_path == 2 or wl.D != 128
+                               else "tcgen05 UMMA, TMEM accumulators") + ")"},
         "gpu_launches": args.steps,
     }
 
@@ -803,6 +805,9 @@ def main():
                     help="step: the decode step (default); swap: eviction to host and back; "
                          "int8: the decode step over an INT8 cache; prefix: prefix caching; "
                          "prefill: paged prefill attention (--config prefill_8b | chunked_8b)")
+    ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2],
+                    help="--op prefill kernel: 0 automatic (tcgen05 at head_dim 128), "
+                         "1 tcgen05, 2 mma.sync")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()

@@ -361,8 +361,13 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  *   query_start[b + 1] <= total_q, else the sequence is skipped (its rows of out
  *   untouched) and PA_DEVERR_BAD_CTX is set.
  * head_dim 64 or 128; num_q_heads / num_kv_heads a divisor of 64; block_size a
- * multiple of 16; batch <= 65535.  Tensor cores (mma.sync), 64 (token, head)
- * rows of one kv head per CTA, K / V tiles of 64 keys by TMA, one launch.
+ * multiple of 16; batch <= 65535.  One launch.  head_dim 128 (and a group
+ * dividing 128) runs on the 5th-generation tensor cores (tcgen05 UMMA with
+ * TMEM accumulators, 128 (token, head) rows of one kv head per CTA, K / V
+ * tiles of 128 keys); otherwise mma.sync (64 rows, 64-key tiles).
+ * Alignment: k_cache, v_cache 16 bytes; q, out 4 (q 16 for the tcgen05
+ * kernel, which the automatic choice then skips).  Errors: PA_ERR_INVALID for
+ * shapes or pointers outside these limits, nothing launched.
  * ---------------------------------------------------------------------- */
 pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
                                const void* v_cache, const int32_t* block_tables,
@@ -371,6 +376,23 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
                                int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
                                pa_dtype dtype, int32_t* dev_error, pa_stream stream);
+
+/* Kernels for pa_prefill_attention_ex. */
+#define PA_PREFILL_AUTO 0      /* tcgen05 where it applies, else mma.sync */
+#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, q 16-byte aligned */
+#define PA_PREFILL_MMA_SYNC 2  /* every supported shape */
+
+/* pa_prefill_attention with the kernel chosen by the caller (same results up to
+ * fp32 rounding order).  An unknown path, or PA_PREFILL_TCGEN05 for a shape it
+ * does not take, is PA_ERR_INVALID with nothing launched. */
+pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, const int32_t* query_start,
+                                  int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
+                                  pa_dtype dtype, int32_t* dev_error, int32_t path,
+                                  pa_stream stream);
 
 /* ------------------------------------------------------------------------
  * INT8 KV cache.  [P5] "The four solutions", KV-cache quantisation: keys and

@@ -21,6 +21,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_OOM, PA_ERR_NOT_FOUND, PA_ERR_CUDA, PA_ERR_DEVICE 
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 PA_PATH_AUTO, PA_PATH_TC, PA_PATH_SIMT = 0, 1, 2
 PA_DECODE_OVERLAP_PROLOGUE = 1
+PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA_SYNC = 0, 1, 2
 PA_DEVERR_BAD_SLOT, PA_DEVERR_BAD_BLOCK, PA_DEVERR_BAD_CTX, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 DTYPE_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
@@ -61,6 +62,8 @@ SIGNATURES = {
                                              _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
     "pa_prefill_attention": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                     _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
+    "pa_prefill_attention_ex": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                       _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _I32, _P]),
     "pa_int8_block_bytes": (C.c_size_t, [_I32, _I32, _I32]),
     "pa_reshape_and_cache_int8": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                          C.c_int, _P, _P]),
@@ -335,7 +338,7 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, contex
 
 
 def pa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
-                         max_q, scale, dev_error=None, stream=None):
+                         max_q, scale, dev_error=None, path=PA_PREFILL_AUTO, stream=None):
     """Causal attention of each sequence's new tokens over its paged cache: q/out
     [T, Hq, D] fp16 or bf16, query_start int32 [B+1] (device), max_q >= every
     query_start[b+1] - query_start[b]; caches and tables as pa_decode_attention."""
@@ -345,12 +348,12 @@ def pa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, q
     MB = block_tables.shape[1]
     if out.shape != q.shape or query_start.shape[0] != B + 1:
         raise ValueError("out must have q's shape and query_start batch + 1 entries")
-    st = lib.pa_prefill_attention(
+    st = lib.pa_prefill_attention_ex(
         _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache", q.dtype),
         _dev_ptr(v_cache, "v_cache", q.dtype), _dev_ptr(block_tables, "block_tables", torch.int32),
         _dev_ptr(context_lens, "context_lens", torch.int32),
         _dev_ptr(query_start, "query_start", torch.int32), B, Hq, Hkv, D, bs, NB, MB, T, int(max_q),
-        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32),
+        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32), path,
         _stream(stream))
     _check(st, "pa_prefill_attention")
 

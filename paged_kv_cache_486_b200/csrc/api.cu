@@ -93,6 +93,24 @@ bool make_tile_map(CUtensorMap* map, bool* three_d, const void* base, int64_t ro
          CUDA_SUCCESS;
 }
 
+// The {D, rows} form with a {64, 16} box only (the tcgen05 prefill addresses
+// each 64-column block itself).
+bool make_tile_map_2d(CUtensorMap* map, const void* base, int64_t rows, int head_dim,
+                      pa_dtype dt) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType t =
+      dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  cuuint32_t box[2] = {64, 16};
+  cuuint32_t es[2] = {1, 1};
+  return enc(map, t, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // Small per-thread cache: encoding is cheap but not free, and decode is called
 // with the same pools every step.
 struct MapEntry {
@@ -528,13 +546,16 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_decode_attention_int8 (decode kernel)");
 }
 
-pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
-                               const void* v_cache, const int32_t* block_tables,
-                               const int32_t* context_lens, const int32_t* query_start,
-                               int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
-                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
-                               int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
-                               pa_dtype dtype, int32_t* dev_error, pa_stream stream) {
+pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
+                                  const void* v_cache, const int32_t* block_tables,
+                                  const int32_t* context_lens, const int32_t* query_start,
+                                  int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
+                                  pa_dtype dtype, int32_t* dev_error, int32_t path,
+                                  pa_stream stream) {
+  if (path != PA_PREFILL_AUTO && path != PA_PREFILL_TCGEN05 && path != PA_PREFILL_MMA_SYNC)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: unknown path %d", path);
   if (dtype != PA_F16 && dtype != PA_BF16)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: dtype must be fp16 or bf16");
   if (total_q < 0) return fail(PA_ERR_INVALID, "pa_prefill_attention: negative total_q");
@@ -565,11 +586,21 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
   if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
     return fail(PA_ERR_INVALID, "pa_prefill_attention: misaligned pointer");
+  const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16);
+  if (path == PA_PREFILL_TCGEN05 && !tc5_ok)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: the tcgen05 kernel needs head_dim 128, "
+                "num_q_heads / num_kv_heads dividing 128 and q 16-byte aligned");
+  const bool use_tc5 = path == PA_PREFILL_TCGEN05 || (path == PA_PREFILL_AUTO && tc5_ok);
   CUtensorMap kmap, vmap;
   bool k3 = false, v3 = false;
-  if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
-      !tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || k3 != v3)
+  if (use_tc5) {
+    if (!make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
+        !make_tile_map_2d(&vmap, v_cache, rows, head_dim, dtype))
+      return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
+  } else if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
+             !tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || k3 != v3) {
     return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
+  }
   pa::PrefillArgs a;
   a.out = out;
   a.q = q;
@@ -589,8 +620,25 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
   a.total_q = total_q;
   a.three_d = k3 ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e = pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  const cudaError_t e =
+      use_tc5 ? pa::launch_prefill_tc5(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream))
+              : pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
+}
+
+pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, const int32_t* query_start,
+                               int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                               int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                               int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
+                               pa_dtype dtype, int32_t* dev_error, pa_stream stream) {
+  return pa_prefill_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens,
+                                 query_start, batch, num_q_heads, num_kv_heads, head_dim,
+                                 block_size, num_blocks, max_blocks, total_q, max_q, scale, dtype,
+                                 dev_error, PA_PREFILL_AUTO, stream);
 }
 
 pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {

@@ -99,12 +99,12 @@ class PagedKVCache:
         return out
 
     def prefill(self, q, block_tables, context_lens, query_start, max_q, scale, out=None,
-                stream=None):
+                path=0, stream=None):
         """Causal attention of each sequence's new tokens (already written) over the cache."""
         if out is None:
             out = torch.empty_like(q)
         pa_prefill_attention(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
-                             query_start, max_q, scale, self.dev_error, stream)
+                             query_start, max_q, scale, self.dev_error, path, stream)
         return out
 
     def device_errors(self, stream=None):

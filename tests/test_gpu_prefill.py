@@ -52,11 +52,15 @@ def _cases():
 CASES = _cases()
 
 
+PATHS = [pa.PA_PREFILL_AUTO, pa.PA_PREFILL_MMA_SYNC]
+
+
 @pytest.mark.parametrize("name", list(CASES))
-def test_prefill_small_configs_match_the_oracle(name):
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_small_configs_match_the_oracle(name, path):
     wl = CASES[name]()
     eng, bt, ctx, qs, q = _build(wl)
-    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale)
+    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale, path=path)
     torch.cuda.synchronize()
     o = run_script(wl)
     ref = oracle.paged_prefill_attention(raw(q), o["k_cache"], o["v_cache"], o["table"],
@@ -65,16 +69,17 @@ def test_prefill_small_configs_match_the_oracle(name):
     assert ok, f"worst error / bound = {worst:.3f}"
     assert eng.device_errors() == 0
     # a larger max_q only launches more (empty) tiles
-    again = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()) + 100, wl.scale)
+    again = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()) + 100, wl.scale, path=path)
     torch.cuda.synchronize()
     assert torch.equal(again.view(torch.int16), out.view(torch.int16))
 
 
 @pytest.mark.parametrize("name", ["prefill_8b", "chunked_8b"])
-def test_prefill_full_size_sampled_rows(name):
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_full_size_sampled_rows(name, path):
     wl = {"prefill_8b": workloads.prefill_8b, "chunked_8b": workloads.chunked_8b}[name]()
     eng, bt, ctx, qs, q = _build(wl)
-    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale)
+    out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale, path=path)
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
     o = run_script(wl, with_cache=False)
@@ -100,14 +105,15 @@ def test_prefill_full_size_sampled_rows(name):
     assert eng.device_errors() == 0
 
 
-def test_prefill_guards():
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_guards(path):
     wl = CASES["f16_g4_d128"]()
     eng, bt, ctx, qs, q = _build(wl)
-    ref = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale).clone()
+    ref = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale, path=path).clone()
     torch.cuda.synchronize()
     # a chunk longer than max_q: that sequence is skipped and reported; others unchanged
     out = torch.zeros_like(q)
-    eng.prefill(q, bt, ctx, qs, 200, wl.scale, out=out)
+    eng.prefill(q, bt, ctx, qs, 200, wl.scale, out=out, path=path)
     torch.cuda.synchronize()
     assert eng.device_errors() & pa.PA_DEVERR_BAD_CTX
     qsn = workloads.query_start(wl)
@@ -120,11 +126,11 @@ def test_prefill_guards():
     # an out-of-range block id: reported, its keys skipped, nothing faults
     bt2 = bt.clone()
     bt2[3, 2] = wl.num_blocks + 7
-    eng.prefill(q, bt2, ctx, qs, int(wl.n_new.max()), wl.scale)
+    eng.prefill(q, bt2, ctx, qs, int(wl.n_new.max()), wl.scale, path=path)
     torch.cuda.synchronize()
     assert eng.device_errors() & pa.PA_DEVERR_BAD_BLOCK
     # no new tokens anywhere
     empty = torch.zeros_like(qs)
-    eng.prefill(q[:0], bt, ctx, empty, 0, wl.scale)
+    eng.prefill(q[:0], bt, ctx, empty, 0, wl.scale, path=path)
     torch.cuda.synchronize()
     assert eng.device_errors() == 0
