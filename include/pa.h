@@ -361,8 +361,8 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  *   query_start[b + 1] <= total_q, else the sequence is skipped (its rows of out
  *   untouched) and PA_DEVERR_BAD_CTX is set.
  * head_dim 64 or 128; num_q_heads / num_kv_heads a divisor of 64; block_size a
- * multiple of 16; batch <= 65535.  One launch.  head_dim 128 (and a group
- * dividing 128) runs on the 5th-generation tensor cores (tcgen05 UMMA with
+ * multiple of 16; batch <= 65535.  One launch.  head_dim 128 (with a group
+ * dividing 128 and scale > 0) runs on the 5th-generation tensor cores (tcgen05 UMMA with
  * TMEM accumulators, 128 (token, head) rows of one kv head per CTA, K / V
  * tiles of 128 keys); otherwise mma.sync (64 rows, 64-key tiles).
  * Alignment: k_cache, v_cache 16 bytes; q, out 4 (q 16 for the tcgen05
@@ -379,7 +379,8 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
 
 /* Kernels for pa_prefill_attention_ex. */
 #define PA_PREFILL_AUTO 0      /* tcgen05 where it applies, else mma.sync */
-#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, q 16-byte aligned */
+#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, scale > 0, q 16-byte
+                                  aligned */
 #define PA_PREFILL_MMA_SYNC 2  /* every supported shape */
 
 /* pa_prefill_attention with the kernel chosen by the caller (same results up to

@@ -93,6 +93,26 @@ bool make_tile_map(CUtensorMap* map, bool* three_d, const void* base, int64_t ro
          CUDA_SUCCESS;
 }
 
+// q as {head_dim, num_q_heads, total_q} with a {64, group, 128 / group} box:
+// 128 rows of (token, head of one kv head's group) pairs per 64-column block.
+static bool make_q_map(CUtensorMap* map, const void* q, int total_q, int num_q_heads,
+                       int head_dim, int group, pa_dtype dt) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const CUtensorMapDataType t =
+      dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(total_q)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(head_dim) * 2 * num_q_heads};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(128 / group)};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(map, t, 3, const_cast<void*>(q), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // The {D, rows} form with a {64, 16} box only (the tcgen05 prefill addresses
 // each 64-column block itself).
 bool make_tile_map_2d(CUtensorMap* map, const void* base, int64_t rows, int head_dim,
@@ -586,15 +606,16 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
     return fail(PA_ERR_INVALID, "pa_prefill_attention: misaligned pointer");
-  const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16);
+  const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16) && scale > 0.f;
   if (path == PA_PREFILL_TCGEN05 && !tc5_ok)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: the tcgen05 kernel needs head_dim 128, "
-                "num_q_heads / num_kv_heads dividing 128 and q 16-byte aligned");
+                "num_q_heads / num_kv_heads dividing 128, scale > 0 and q 16-byte aligned");
   const bool use_tc5 = path == PA_PREFILL_TCGEN05 || (path == PA_PREFILL_AUTO && tc5_ok);
-  CUtensorMap kmap, vmap;
+  CUtensorMap qmap, kmap, vmap;
   bool k3 = false, v3 = false;
   if (use_tc5) {
-    if (!make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
+    if (!make_q_map(&qmap, q, total_q, num_q_heads, head_dim, group, dtype) ||
+        !make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
         !make_tile_map_2d(&vmap, v_cache, rows, head_dim, dtype))
       return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
   } else if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
@@ -623,7 +644,8 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   a.k_cache = k_cache;
   a.v_cache = v_cache;
   const cudaError_t e =
-      use_tc5 ? pa::launch_prefill_tc5(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream))
+      use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap,
+                                       static_cast<cudaStream_t>(stream))
               : pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
 }

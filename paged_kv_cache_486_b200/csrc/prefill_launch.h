@@ -34,9 +34,12 @@ template <> struct PrefillPSplit<__half> { static constexpr bool value = false; 
 cudaError_t launch_prefill(const PrefillArgs& a, pa_dtype dtype, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, cudaStream_t stream);
 
-// tcgen05 kernel: head_dim 128, 128 % group == 0; kmap2d / vmap2d are {head_dim,
-// rows} maps with a {64, 16} box and the 128-byte swizzle.
-cudaError_t launch_prefill_tc5(const PrefillArgs& a, pa_dtype dtype, const CUtensorMap& kmap2d,
-                               const CUtensorMap& vmap2d, cudaStream_t stream);
+// tcgen05 kernel: head_dim 128, 128 % group == 0, scale > 0, q 16-byte aligned;
+// qmap is the {head_dim, num_q_heads, total_q} map of q with a {64, group, 128 /
+// group} box, kmap2d / vmap2d are {head_dim, rows} maps of the pools with a
+// {64, 16} box, all with the 128-byte swizzle.
+cudaError_t launch_prefill_tc5(const PrefillArgs& a, pa_dtype dtype, const CUtensorMap& qmap,
+                               const CUtensorMap& kmap2d, const CUtensorMap& vmap2d,
+                               cudaStream_t stream);
 
 }  // namespace pa

@@ -2,28 +2,36 @@
 //
 // Same definition and row layout as prefill.cu (causal attention of each
 // sequence's new tokens over its paged cache; a CTA owns rows = (new token,
-// head of one kv head's group) pairs), head_dim 128, fp16 / bf16.
+// head of one kv head's group) pairs), head_dim 128, fp16 / bf16, scale > 0.
 //
 // Per CTA: 128 query rows and key tiles of 128 keys.
-//   S = Q . K_tile^T   UMMA M=128 N=128, K=128 in 8 steps of 16 (Q and K from
-//                      shared memory, 128-byte-swizzled K-major), fp32 in TMEM;
-//   softmax            one thread per row reads its S row from TMEM (no
-//                      shuffles), masks (causal), updates its running max
-//                      lazily (rescale O only when the max moves by > 2^8),
-//                      writes P as 16-bit values back to TMEM;
+//   S = Q . K_tile^T   UMMA M=128 N=128 (the last tile: N rounded up to 16
+//                      past its keys), K=128 in 8 steps of 16, Q and K from
+//                      shared memory (128-byte-swizzled, K-major), fp32 in TMEM;
+//   softmax            one thread per row reads its S row from TMEM, masks
+//                      (causal, diagonal tiles only), keeps its running max
+//                      lazily (O is rescaled only when the max rises by more
+//                      than 2^8) and writes P as 16-bit values over its own S
+//                      columns;
 //   O += P . V_tile    UMMA with A = P from TMEM (K-major), B = V from shared
 //                      memory (MN-major: head_dim contiguous), fp32 in TMEM.
 // bf16 keeps P as a head + tail pair (two products), fp16 a single value.
-// Warps: 0 loads K / V tiles (TMA, two stages), 1 allocates TMEM and issues
-// every UMMA (one thread), 2..5 run the softmax and the epilogue (warp w reads
-// TMEM lanes 32 (w mod 4) .. +31, which is its rows).  S is double buffered in
-// TMEM, so the tensor core computes the next tile's scores while the softmax
-// works on this one.  TMEM columns: S0 0..127, S1 128..255, P head 256..319,
-// P tail 320..383, O 384..511.
+//
+// Warps: 0 loads Q once and the K / V tiles (TMA; K and V have their own
+// stages, so the next keys load as soon as S is done), 1 allocates TMEM and
+// issues every UMMA from one thread, as soon as each product's inputs are
+// ready, 2..5 run the softmax and the epilogue (warp w reads TMEM lanes
+// 32 (w mod 4) .. +31, which are its rows).  S / P has three buffers in TMEM
+// (columns 0, 128, 256), so the tensor core computes the next tile's scores
+// while the softmax works on this one, and the softmax writes the next P
+// while the tensor core is still multiplying this one; a buffer takes new
+// scores only once the product that read its P has completed.  O is in
+// 384..511.
 //
 // Shared memory (1024-byte aligned, every tile in 64-column blocks of rows of
-// 128 bytes, 128-byte swizzle): Q 32 KB, K 2 x 32 KB, V 2 x 32 KB.  That keeps
-// one CTA per SM, so the 512-column TMEM allocation never waits.
+// 128 bytes, 128-byte swizzle): Q 32 KB (O is staged there for coalesced
+// stores at the end), K and V 32 KB per stage.  That keeps one CTA per SM, so
+// the 512-column TMEM allocation never waits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -42,14 +50,18 @@ constexpr int kD = 128;
 constexpr int kThreads = 192;
 constexpr int kColBlock = kRows * 128;     // one 64-column block of 128 rows: 16 KB
 constexpr int kTileBytes = 2 * kColBlock;  // 128 rows x 128 columns x 2 bytes
+constexpr int kGroupBytes = 16 * 128;      // 16 rows of one 64-column block
+constexpr int kStages = 2;                 // K and V tiles in flight, each
 constexpr int kQOff = 0;
-constexpr int kKOff = kTileBytes;                 // 2 stages
-constexpr int kVOff = kKOff + 2 * kTileBytes;     // 2 stages
-constexpr int kRing = kVOff + 2 * kTileBytes;     // 160 KB
+constexpr int kKOff = kTileBytes;
+constexpr int kVOff = kKOff + kStages * kTileBytes;
+constexpr int kRing = kVOff + kStages * kTileBytes;  // 160 KB at two stages
 constexpr int kSmem = 1024 + kRing + 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColP = 256, kColPT = 320, kColO = 384;
+constexpr int kSBuf = 3;  // S / P buffers in TMEM
+constexpr uint32_t kColS = 0, kColO = kSBuf * kKeys;
 constexpr float kSlack = 8.f;
+constexpr long long kSpinLimit = 1ll << 31;  // clock cycles without progress
 
 // ---- PTX wrappers ----
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -61,10 +73,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 }
 
 // kind::f16 instruction descriptor: fp32 accumulator, A / B in fp16 (0) or
-// bf16 (1), A K-major, B K-major (0) or MN-major (1), N = 128, M = 128.
-__host__ __device__ constexpr uint32_t idesc(uint32_t ab_format, uint32_t b_major) {
-  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_major << 16) |
-         ((kKeys >> 3) << 17) | ((kRows >> 4) << 24);
+// bf16 (1), A K-major, B K-major (0) or MN-major (1), M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc(uint32_t ab_format, uint32_t b_major, uint32_t n) {
+  return (1u << 4) | (ab_format << 7) | (ab_format << 10) | (b_major << 16) | ((n >> 3) << 17) |
+         ((kRows >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t id,
@@ -97,6 +109,28 @@ __device__ __forceinline__ void fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Non-blocking: has the phase of this parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: results below 2^-126
+// flush to zero, which for softmax weights relative to the row's reference is
+// immaterial).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 32 consecutive columns of this thread's lane, not yet waited for.
 __device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -127,14 +161,6 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  tmem_ld32_issue(taddr, r);
-  tmem_ld_wait(r);
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -148,8 +174,48 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                       uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x),
+      "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                       uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
 }
 
 // Byte offset of 16-byte chunk c (0..15) of row r in a tile (64-column blocks
@@ -158,25 +224,39 @@ __device__ __forceinline__ uint32_t tile_off(int r, int c) {
   return (c >> 3) * kColBlock + r * 128 + (((c & 7) ^ (r & 7)) << 4);
 }
 
+// Byte offset of 16-byte chunk c of row r of the output staging (rows of 256
+// bytes, chunks permuted within each 128-byte half so that 8 consecutive rows
+// writing the same chunk hit distinct banks).
+__device__ __forceinline__ uint32_t out_off(int r, int c) {
+  return r * 256 + (((c & 8) | ((c ^ r) & 7)) << 4);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_tc5_kernel(const __grid_constant__ CUtensorMap kmap,
+    prefill_tc5_kernel(const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap, PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kRing);
-  // barriers: kv_full[2], kv_empty[2], s_full[2], p_full, o_done, q_ready, mma_final
-  const uint32_t b_kv_full = tc::smem_u32(&bars[0]);
-  const uint32_t b_kv_empty = tc::smem_u32(&bars[2]);
-  const uint32_t b_s_full = tc::smem_u32(&bars[4]);
-  const uint32_t b_p_full = tc::smem_u32(&bars[6]);
-  const uint32_t b_o_done = tc::smem_u32(&bars[7]);
-  const uint32_t b_q_ready = tc::smem_u32(&bars[8]);
-  const uint32_t b_final = tc::smem_u32(&bars[9]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
-  volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(bars + 11);
+  // barriers: k_full, k_empty, v_full, v_empty (one per stage each), then per
+  // S / P buffer s_full (scores written), p_full (P written), pv_done (its
+  // P . V completed), then q_full, final
+  constexpr int kB = 4 * kStages;
+  const uint32_t b_k_full = tc::smem_u32(&bars[0]);
+  const uint32_t b_k_empty = tc::smem_u32(&bars[kStages]);
+  const uint32_t b_v_full = tc::smem_u32(&bars[2 * kStages]);
+  const uint32_t b_v_empty = tc::smem_u32(&bars[3 * kStages]);
+  const uint32_t b_s_full = tc::smem_u32(&bars[kB]);
+  const uint32_t b_p_full = tc::smem_u32(&bars[kB + kSBuf]);
+  const uint32_t b_pv_done = tc::smem_u32(&bars[kB + 2 * kSBuf]);
+  const uint32_t b_q_full = tc::smem_u32(&bars[kB + 3 * kSBuf]);
+  const uint32_t b_final = tc::smem_u32(&bars[kB + 3 * kSBuf + 1]);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kB + 3 * kSBuf + 2);
+  volatile int32_t* abort_flag =
+      reinterpret_cast<volatile int32_t*>(bars + kB + 3 * kSBuf + 3);
 
   const int b = blockIdx.z, g = blockIdx.y;
   const int tile_q = gridDim.x - 1 - blockIdx.x;  // later query tiles first
@@ -196,24 +276,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int past = ctx - nq;
   const int n_keys = past + (min(r0 + kRows, rows) - 1) / G + 1;
   const int n_tiles = (n_keys + kKeys - 1) / kKeys;
+  // keys of the last tile rounded up to 16: its S product's N, its P . V steps
+  const int n_last = ((n_keys - (n_tiles - 1) * kKeys) + 15) & ~15;
   const int bs = a.block_size;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr uint32_t kAB = PrefillPSplit<T>::value ? 1u : 0u;  // operand format: bf16 1, fp16 0
-  constexpr uint32_t kIdS = idesc(kAB, 0), kIdO = idesc(kAB, 1);
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(b_kv_full, 1);
-    tc::mbar_init(b_kv_full + 8, 1);
-    tc::mbar_init(b_kv_empty, 1);
-    tc::mbar_init(b_kv_empty + 8, 1);
-    tc::mbar_init(b_s_full, 1);
-    tc::mbar_init(b_s_full + 8, 1);
-    tc::mbar_init(b_p_full, 4);
-    tc::mbar_init(b_o_done, 1);
-    tc::mbar_init(b_q_ready, 4);
+    for (int i = 0; i < kB; ++i) tc::mbar_init(tc::smem_u32(&bars[i]), 1);
+    for (int i = 0; i < kSBuf; ++i) {
+      tc::mbar_init(b_s_full + 8 * i, 1);
+      tc::mbar_init(b_p_full + 8 * i, 4);
+      tc::mbar_init(b_pv_done + 8 * i, 1);
+    }
+    tc::mbar_init(b_q_full, 1);
     tc::mbar_init(b_final, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&qmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&kmap)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
   }
@@ -228,147 +308,158 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ============================ K / V producer ============================
-    for (int t = 0; t < n_tiles && !*abort_flag; ++t) {
-      const int stage = t & 1;
-      if (t >= 2 && !__all_sync(kFull, tc::mbar_wait_bounded(b_kv_empty + 8 * stage,
-                                                             ((t >> 1) - 1) & 1))) {
+    // ============================ Q, K / V producer ============================
+    // Q: the CTA's 128 rows are 128 / G consecutive tokens x the G heads of kv
+    // head g, one {64, G, 128 / G} box per 64-column block (rows past the
+    // sequence's tokens are other tokens or zeros; their rows are never stored).
+    if (lane == 0) {
+      tc::mbar_arrive_expect_tx(b_q_full, kTileBytes);
+      tma_3d(base + kQOff, &qmap, 0, g * G, q0 + r0 / G, b_q_full);
+      tma_3d(base + kQOff + kColBlock, &qmap, 64, g * G, q0 + r0 / G, b_q_full);
+    }
+    // Lane k (< 8) reads the block id of 16-key group k of the next tile while
+    // this one is loaded; an id is checked where it is used.
+    const int32_t* bt = a.block_tables + static_cast<int64_t>(b) * a.max_blocks;
+    auto raw_id = [&](int t) {
+      const int key = t * kKeys + 16 * (lane & 7);
+      return (lane < 8 && key < n_keys) ? __ldg(&bt[key / bs]) : -1;
+    };
+    int id_next = raw_id(0);
+    bool live = true;
+    for (int t = 0; t < n_tiles && live && !*abort_flag; ++t) {
+      const int stage = t % kStages;
+      const int n_grp = t == n_tiles - 1 ? n_last / 16 : kKeys / 16;
+      int id_mine = id_next;
+      if (t + 1 < n_tiles) id_next = raw_id(t + 1);
+      const int key_mine = t * kKeys + 16 * (lane & 7);
+      if (lane < n_grp && key_mine < n_keys && (id_mine < 0 || id_mine >= a.num_blocks)) {
+        report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+        id_mine = -1;
+      }
+      // whole groups in a valid block go by tensor map; the group holding key
+      // n_keys - 1 when it is partial, and groups of invalid blocks, by hand
+      // with zeros in the rows that hold no key; groups past the tile's N are
+      // never read
+      const uint32_t tma_mask =
+          __ballot_sync(kFull, lane < n_grp && id_mine >= 0 && key_mine + 16 <= n_keys);
+      const uint32_t hand_mask = __ballot_sync(kFull, lane < n_grp) & ~tma_mask;
+      const int row_mine =
+          (id_mine < 0 ? 0 : id_mine * a.num_kv_heads + g) * bs + key_mine % bs;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // 0: keys, 1: values
+        const uint32_t full = (which ? b_v_full : b_k_full) + 8 * stage;
+        const uint32_t empty = (which ? b_v_empty : b_k_empty) + 8 * stage;
+        if (t >= kStages &&
+            !__all_sync(kFull, tc::mbar_wait_bounded(empty, ((t / kStages) - 1) & 1))) {
+          if (lane == 0) {
+            report(a.dev_error, PA_DEVERR_TIMEOUT);
+            *abort_flag = 1;
+          }
+          live = false;
+          break;
+        }
+        const uint32_t dst = base + (which ? kVOff : kKOff) + stage * kTileBytes;
+        if (hand_mask) {
+          const T* src = static_cast<const T*>(which ? a.v_cache : a.k_cache);
+          for (int k = 0; k < kKeys / 16; ++k) {
+            if (!(hand_mask >> k & 1)) continue;
+            const int id = __shfl_sync(kFull, id_mine, k);
+            const int key = t * kKeys + 16 * k;
+            const int valid = id >= 0 ? min(16, n_keys - key) : 0;
+            const T* rows0 = src + (static_cast<int64_t>(id < 0 ? 0 : id * a.num_kv_heads + g) *
+                                        bs + key % bs) * kD;
+            for (int i = lane; i < 16 * 16; i += 32) {
+              const int rr = i >> 4, c = i & 15;
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (rr < valid) v = __ldg(reinterpret_cast<const uint4*>(rows0 + rr * kD) + c);
+              st_shared4(dst + tile_off(16 * k + rr, c), v);
+            }
+          }
+          // generic writes above are read by the tensor core (async proxy)
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
         if (lane == 0) {
-          report(a.dev_error, PA_DEVERR_TIMEOUT);
-          *abort_flag = 1;
+          if (tma_mask)
+            tc::mbar_arrive_expect_tx(full, __popc(tma_mask) * 2 * kGroupBytes);
+          else
+            tc::mbar_arrive(full);
         }
-        break;
-      }
-      const uint32_t kt = base + kKOff + stage * kTileBytes;
-      const uint32_t vt = base + kVOff + stage * kTileBytes;
-      // 16-key groups: whole and in a valid block -> TMA; partial (the one
-      // holding key n_keys - 1) -> loaded here with the rows past it zeroed;
-      // past n_keys or in an invalid block -> V rows zeroed (P is 0 there).
-      int tma_groups = 0;
-      for (int k = 0; k < kKeys / 16; ++k) {
-        const int key = t * kKeys + k * 16;
-        bool tma = false;
-        int id = -1;
-        if (key < n_keys) {
-          id = __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + key / bs]);
-          if (id < 0 || id >= a.num_blocks) {
-            if (lane == 0) report(a.dev_error, PA_DEVERR_BAD_BLOCK);
-            id = -1;
-          }
-          tma = id >= 0 && key + 16 <= n_keys;
-        }
-        if (tma) {
-          ++tma_groups;
-          continue;
-        }
-        // this group by hand: 16 rows x 16 chunks per tensor, 32 lanes
-        const int valid = id >= 0 ? n_keys - key : 0;  // rows of the group to load
-        const T* ks = nullptr;
-        const T* vs = nullptr;
-        if (id >= 0) {
-          const int64_t row0 =
-              (static_cast<int64_t>(id) * a.num_kv_heads + g) * bs + (key % bs);
-          ks = static_cast<const T*>(a.k_cache) + row0 * kD;
-          vs = static_cast<const T*>(a.v_cache) + row0 * kD;
-        }
-        for (int i = lane; i < 16 * 16; i += 32) {
-          const int rr = i >> 4, c = i & 15;
-          uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-          if (rr < valid) {
-            kv = __ldg(reinterpret_cast<const uint4*>(ks + rr * kD) + c);
-            vv = __ldg(reinterpret_cast<const uint4*>(vs + rr * kD) + c);
-          }
-          const uint32_t off = tile_off(k * 16 + rr, c);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(kt + off), "r"(kv.x),
-                       "r"(kv.y), "r"(kv.z), "r"(kv.w) : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(vt + off), "r"(vv.x),
-                       "r"(vv.y), "r"(vv.z), "r"(vv.w) : "memory");
-        }
-      }
-      // generic writes above are read by the tensor core (async proxy)
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) {
-        const uint32_t bar = b_kv_full + 8 * stage;
-        if (tma_groups)
-          tc::mbar_arrive_expect_tx(bar, tma_groups * 4 * (16 * 128));
-        else
-          tc::mbar_arrive(bar);
-        for (int k = 0; k < kKeys / 16; ++k) {
-          const int key = t * kKeys + k * 16;
-          if (key >= n_keys || key + 16 > n_keys) continue;
-          const int id = __ldg(&a.block_tables[static_cast<int64_t>(b) * a.max_blocks + key / bs]);
-          if (id < 0 || id >= a.num_blocks) continue;
-          const int row = (id * a.num_kv_heads + g) * bs + key % bs;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                " [%0], [%1, {%2, %3}], [%4];" ::"r"(kt + h * kColBlock + k * 16 * 128),
-                "l"(reinterpret_cast<uint64_t>(&kmap)), "r"(64 * h), "r"(row), "r"(bar)
-                : "memory");
-            asm volatile(
-                "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-                " [%0], [%1, {%2, %3}], [%4];" ::"r"(vt + h * kColBlock + k * 16 * 128),
-                "l"(reinterpret_cast<uint64_t>(&vmap)), "r"(64 * h), "r"(row), "r"(bar)
-                : "memory");
-          }
+        __syncwarp();
+        if (tma_mask >> lane & 1) {
+          const CUtensorMap* map = which ? &vmap : &kmap;
+          tma_2d(dst + lane * kGroupBytes, map, 0, row_mine, full);
+          tma_2d(dst + kColBlock + lane * kGroupBytes, map, 64, row_mine, full);
         }
       }
     }
   } else if (warp == 1) {
     // ============================= UMMA issuer ==============================
+    // S_t needs K_t and its TMEM buffer, which held P_{t-3}: free once
+    // P_{t-3} . V has completed.  P_t . V needs P_t and V_t.  Each is issued
+    // as soon as it can go.
     const bool leader = lane == 0;
-    bool ok = __all_sync(kFull, tc::mbar_wait_bounded(b_q_ready, 0));
     const uint32_t q_s = base + kQOff;
-    auto issue_s = [&](int t) {  // S[t & 1] = Q . K_t^T
-      const uint32_t kt = base + kKOff + (t & 1) * kTileBytes;
-      const uint32_t d = tmem + kColS + (t & 1) * kKeys;
+    bool ok = __all_sync(kFull, tc::mbar_wait_bounded(b_q_full, 0));
+    int ns = 0, npv = 0;
+    long long idle0 = clock64();
+    while (ok && npv < n_tiles) {
+      bool progress = false;
+      if (ns < n_tiles && ns <= npv + kSBuf - 1) {
+        const bool ready = __shfl_sync(
+            kFull, leader ? ((ns < kSBuf || mbar_test(b_pv_done + 8 * (ns % kSBuf),
+                                                      ((ns - kSBuf) / kSBuf) & 1)) &&
+                             mbar_test(b_k_full + 8 * (ns % kStages), (ns / kStages) & 1))
+                          : false, 0);
+        if (ready) {
+          if (leader) {
+            fence_after();
+            const uint32_t kt = base + kKOff + (ns % kStages) * kTileBytes;
+            const uint32_t d = tmem + kColS + (ns % kSBuf) * kKeys;
+            const uint32_t id = idesc(kAB, 0, ns == n_tiles - 1 ? n_last : kKeys);
 #pragma unroll
-      for (int s = 0; s < kD / 16; ++s) {
-        const uint32_t off = (s >> 2) * kColBlock + (s & 3) * 32;
-        mma_ss(d, smem_desc(q_s + off, 16, 1024), smem_desc(kt + off, 16, 1024), kIdS, s > 0);
-      }
-      commit(b_s_full + 8 * (t & 1));
-    };
-    if (ok && leader) fence_after();
-    if (ok) {
-      if (!__all_sync(kFull, tc::mbar_wait_bounded(b_kv_full, 0))) ok = false;
-    }
-    if (ok && leader) {
-      fence_after();
-      issue_s(0);
-    }
-    for (int t = 0; ok && t < n_tiles; ++t) {
-      // the next tile's scores while the softmax works on this one
-      if (t + 1 < n_tiles) {
-        if (!__all_sync(kFull, tc::mbar_wait_bounded(b_kv_full + 8 * ((t + 1) & 1),
-                                                     ((t + 1) >> 1) & 1))) {
-          ok = false;
-          break;
-        }
-        if (leader) {
-          fence_after();
-          issue_s(t + 1);
+            for (int s = 0; s < kD / 16; ++s) {
+              const uint32_t off = (s >> 2) * kColBlock + (s & 3) * 32;
+              mma_ss(d, smem_desc(q_s + off, 16, 1024), smem_desc(kt + off, 16, 1024), id, s > 0);
+            }
+            commit(b_s_full + 8 * (ns % kSBuf));
+            commit(b_k_empty + 8 * (ns % kStages));  // K_ns may be refilled
+          }
+          ++ns;
+          progress = true;
         }
       }
-      // O += P_t . V_t once the softmax has written P_t
-      if (!__all_sync(kFull, tc::mbar_wait_bounded(b_p_full, t & 1))) {
-        ok = false;
-        break;
-      }
-      if (leader) {
-        fence_after();
-        const uint32_t vt = base + kVOff + (t & 1) * kTileBytes;
-#pragma unroll
-        for (int s = 0; s < kKeys / 16; ++s) {
-          const uint64_t bd = smem_desc(vt + s * 16 * 128, kColBlock, 1024);
-          mma_ts(tmem + kColO, tmem + kColP + 8 * s, bd, kIdO, (t > 0 || s > 0) ? 1u : 0u);
-          if (PrefillPSplit<T>::value) mma_ts(tmem + kColO, tmem + kColPT + 8 * s, bd, kIdO, 1u);
+      if (npv < ns) {
+        const bool ready = __shfl_sync(
+            kFull, leader ? (mbar_test(b_p_full + 8 * (npv % kSBuf), (npv / kSBuf) & 1) &&
+                             mbar_test(b_v_full + 8 * (npv % kStages), (npv / kStages) & 1))
+                          : false, 0);
+        if (ready) {
+          if (leader) {
+            fence_after();
+            const uint32_t vt = base + kVOff + (npv % kStages) * kTileBytes;
+            const uint32_t p = tmem + kColS + (npv % kSBuf) * kKeys;  // P head: columns 0..63
+            const int steps = npv == n_tiles - 1 ? n_last / 16 : kKeys / 16;
+            constexpr uint32_t kIdO = idesc(kAB, 1, kD);
+            for (int s = 0; s < steps; ++s) {
+              const uint64_t bd = smem_desc(vt + s * kGroupBytes, kColBlock, 1024);
+              mma_ts(tmem + kColO, p + 8 * s, bd, kIdO, (npv > 0 || s > 0) ? 1u : 0u);
+              if (PrefillPSplit<T>::value) mma_ts(tmem + kColO, p + 64 + 8 * s, bd, kIdO, 1u);
+            }
+            commit(b_v_empty + 8 * (npv % kStages));  // V_npv may be refilled
+            commit(b_pv_done + 8 * (npv % kSBuf));    // O holds P_0 .. P_npv
+          }
+          ++npv;
+          progress = true;
         }
-        commit(b_kv_empty + 8 * (t & 1));  // K_t / V_t may be refilled
-        commit(b_o_done);                  // O (and P) are free again
       }
+      if (progress) {
+        idle0 = clock64();
+      } else {
+        if (clock64() - idle0 > kSpinLimit || *abort_flag) ok = false;
+        __nanosleep(20);
+      }
+      ok = __all_sync(kFull, ok);
     }
     if (!ok && lane == 0) {
       report(a.dev_error, PA_DEVERR_TIMEOUT);
@@ -380,152 +471,164 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::mbar_wait_bounded(b_final, 0);
   } else {
     // ======================= softmax and epilogue ===========================
-    const int sw = warp - 2;                 // 0..3
     const int quarter = warp & 3;            // TMEM lanes 32 quarter .. +31
     const int r = 32 * quarter + lane;       // this thread's row of the CTA
     const int grow = r0 + r;
     const bool valid = grow < rows;
-    const int tok = valid ? grow / G : 0;
-    const int hh = valid ? grow - tok * G : 0;
-    const int pos = valid ? past + tok : -1;
+    const int pos = valid ? past + grow / G : -1;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
-    // Q row into shared memory (swizzled), zeros past the rows
-    {
-      const T* qr = static_cast<const T*>(a.q) +
-                    (static_cast<int64_t>(q0 + tok) * a.num_q_heads + g * G + hh) * kD;
-      for (int c = 0; c < 16; ++c) {
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (valid) v = __ldg(reinterpret_cast<const uint4*>(qr) + c);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
-                     ::"r"(base + kQOff + tile_off(r, c)), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-                     : "memory");
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(b_q_ready);
-    }
-    (void)sw;
-    float m = -INFINITY, l = 0.f;
+    const float c = a.scale_log2;  // > 0
+    float m = -INFINITY;           // running reference, scaled (log2) domain
+    float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
     bool ok = true;
     for (int t = 0; t < n_tiles; ++t) {
-      if (!__all_sync(kFull, tc::mbar_wait_bounded(b_s_full + 8 * (t & 1), (t >> 1) & 1))) {
+      if (!__all_sync(kFull, tc::mbar_wait_bounded(b_s_full + 8 * (t % kSBuf),
+                                                   (t / kSBuf) & 1))) {
         ok = false;
         break;
       }
       fence_after();
-      const uint32_t srow = trow + kColS + (t & 1) * kKeys;
-      // pass 1: this row's maximum over the tile (masked)
-      float mx = -INFINITY;
+      const uint32_t sp = trow + kColS + (t % kSBuf) * kKeys;
       uint32_t su[4][32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld32_issue(srow + 32 * ch, su[ch]);
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32_issue(sp + 32 * ch, su[ch]);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(su[ch]);  // the first waits for all four
       float sv[4][32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int j = t * kKeys + 32 * ch + i;
-          float v = __uint_as_float(su[ch][i]) * a.scale_log2;
-          if (j > pos) v = -INFINITY;
-          sv[ch][i] = v;
-          mx = fmaxf(mx, v);
+        for (int i = 0; i < 32; ++i) sv[ch][i] = __uint_as_float(su[ch][i]);
+      // causal mask where the tile reaches past some row's position (and for
+      // rows past the sequence); columns past the tile's N are masked too
+      if (__any_sync(kFull, t * kKeys + kKeys - 1 > pos)) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (t * kKeys + 32 * ch + i > pos) sv[ch][i] = -INFINITY;
+      }
+      float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          x0 = fmaxf(x0, sv[ch][i]);
+          x1 = fmaxf(x1, sv[ch][i + 1]);
+          x2 = fmaxf(x2, sv[ch][i + 2]);
+          x3 = fmaxf(x3, sv[ch][i + 3]);
         }
-      }
-      // P must not be overwritten before the previous P . V has read it
-      if (t > 0 && !__all_sync(kFull, tc::mbar_wait_bounded(b_o_done, (t - 1) & 1))) {
-        ok = false;
-        break;
-      }
-      fence_after();
+      const float mx_raw = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+      const float mx = mx_raw == -INFINITY ? -INFINITY : mx_raw * c;
       // a row whose maximum rose by more than 2^kSlack takes it as its new
-      // reference and rescales its row of O (after the previous P . V).  TMEM
+      // reference and rescales its row of O once P_{t-1} . V is done.  TMEM
       // loads and stores are warp-collective, so the warp does this together;
       // rows that keep their reference scale by 1.
       const bool moves = mx > m + kSlack;
       if (__any_sync(kFull, moves)) {
         const float mnew = moves ? mx : m;
-        const float alpha = m == -INFINITY ? 0.f : exp2f(m - mnew);
+        const float alpha = m == -INFINITY ? 0.f : ex2(m - mnew);
         if (t > 0) {
-#pragma unroll
+          if (!__all_sync(kFull, tc::mbar_wait_bounded(b_pv_done + 8 * ((t - 1) % kSBuf),
+                                                       ((t - 1) / kSBuf) & 1))) {
+            ok = false;
+            break;
+          }
+          fence_after();
+#pragma unroll 1
           for (int ch = 0; ch < 4; ++ch) {
-            float ov[32];
-            tmem_ld32(trow + kColO + 32 * ch, ov);
             uint32_t ou[32];
+            tmem_ld32_issue(trow + kColO + 32 * ch, ou);
+            tmem_ld_wait(ou);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ou[i] = __float_as_uint(ov[i] * alpha);
+            for (int i = 0; i < 32; ++i) ou[i] = __float_as_uint(__uint_as_float(ou[i]) * alpha);
             tmem_st32(trow + kColO + 32 * ch, ou);
           }
         }
-        l *= alpha;
+        l0 *= alpha;
+        l1 *= alpha;
+        l2 *= alpha;
+        l3 *= alpha;
         m = mnew;
       }
-      const float mref = m == -INFINITY ? 0.f : m;
+      const float neg = m == -INFINITY ? 0.f : -m;
+      // P over this tile's S columns: head pairs in columns 0..63, tails in 64..127
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t ph[16], pt[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = exp2f(sv[ch][2 * i] - mref);
-          const float p1 = exp2f(sv[ch][2 * i + 1] - mref);
-          l += p0 + p1;
-          if (PrefillPSplit<T>::value)
+        for (int i = 0; i < 16; i += 2) {
+          const float p0 = ex2(fmaf(sv[ch][2 * i], c, neg));
+          const float p1 = ex2(fmaf(sv[ch][2 * i + 1], c, neg));
+          const float p2 = ex2(fmaf(sv[ch][2 * i + 2], c, neg));
+          const float p3 = ex2(fmaf(sv[ch][2 * i + 3], c, neg));
+          l0 += p0;
+          l1 += p1;
+          l2 += p2;
+          l3 += p3;
+          if (PrefillPSplit<T>::value) {
             tc::split2<T>(p0, p1, ph[i], pt[i]);
-          else
-            ph[i] = pt[i] = tc::pack2<T>(p0, p1);
+            tc::split2<T>(p2, p3, ph[i + 1], pt[i + 1]);
+          } else {
+            ph[i] = tc::pack2<T>(p0, p1);
+            ph[i + 1] = tc::pack2<T>(p2, p3);
+          }
         }
-        // 16 columns of packed pairs per 32 keys
-        uint32_t buf[32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          buf[i] = ph[i];
-          buf[16 + i] = pt[i];
-        }
-        // head pairs -> P columns 16 ch .. +15, tail pairs -> P tail columns
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-            "%10, %11, %12, %13, %14, %15, %16};"
-            ::"r"(trow + kColP + 16 * ch), "r"(buf[0]), "r"(buf[1]), "r"(buf[2]), "r"(buf[3]),
-              "r"(buf[4]), "r"(buf[5]), "r"(buf[6]), "r"(buf[7]), "r"(buf[8]), "r"(buf[9]),
-              "r"(buf[10]), "r"(buf[11]), "r"(buf[12]), "r"(buf[13]), "r"(buf[14]), "r"(buf[15])
-            : "memory");
-        if (PrefillPSplit<T>::value) {
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-              "%10, %11, %12, %13, %14, %15, %16};"
-              ::"r"(trow + kColPT + 16 * ch), "r"(buf[16]), "r"(buf[17]), "r"(buf[18]),
-                "r"(buf[19]), "r"(buf[20]), "r"(buf[21]), "r"(buf[22]), "r"(buf[23]),
-                "r"(buf[24]), "r"(buf[25]), "r"(buf[26]), "r"(buf[27]), "r"(buf[28]),
-                "r"(buf[29]), "r"(buf[30]), "r"(buf[31])
-              : "memory");
-        }
+        tmem_st16(sp + 16 * ch, ph);
+        if (PrefillPSplit<T>::value) tmem_st16(sp + 64 + 16 * ch, pt);
       }
       tmem_st_wait();
       fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(b_p_full);
+      if (lane == 0) tc::mbar_arrive(b_p_full + 8 * (t % kSBuf));
     }
-    // epilogue: O / l once the last P . V is done
-    if (ok && __all_sync(kFull, tc::mbar_wait_bounded(b_o_done, (n_tiles - 1) & 1))) {
+    // epilogue: O / l once the last P . V is done, staged in the Q tile (free
+    // then) and stored by the four warps as whole 16-byte chunks
+    ok = ok && __all_sync(kFull, tc::mbar_wait_bounded(b_pv_done + 8 * ((n_tiles - 1) % kSBuf),
+                                                       ((n_tiles - 1) / kSBuf) & 1));
+    const uint32_t stage_out = base + kQOff;
+    if (ok) {
       fence_after();
-      T* dst = static_cast<T*>(a.out) +
-               (static_cast<int64_t>(q0 + tok) * a.num_q_heads + g * G + hh) * kD;
-      const float inv = 1.f / l;
-#pragma unroll
+      const float inv = 1.f / ((l0 + l1) + (l2 + l3));
+#pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
-        float ov[32];
-        tmem_ld32(trow + kColO + 32 * ch, ov);
-        if (valid) {
+        uint32_t ou[32];
+        tmem_ld32_issue(trow + kColO + 32 * ch, ou);
+        tmem_ld_wait(ou);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            reinterpret_cast<uint32_t*>(dst)[16 * ch + i] =
-                tc::pack2<T>(ov[2 * i] * inv, ov[2 * i + 1] * inv);
+        for (int k = 0; k < 4; ++k) {
+          uint4 v;
+          v.x = tc::pack2<T>(__uint_as_float(ou[8 * k]) * inv,
+                             __uint_as_float(ou[8 * k + 1]) * inv);
+          v.y = tc::pack2<T>(__uint_as_float(ou[8 * k + 2]) * inv,
+                             __uint_as_float(ou[8 * k + 3]) * inv);
+          v.z = tc::pack2<T>(__uint_as_float(ou[8 * k + 4]) * inv,
+                             __uint_as_float(ou[8 * k + 5]) * inv);
+          v.w = tc::pack2<T>(__uint_as_float(ou[8 * k + 6]) * inv,
+                             __uint_as_float(ou[8 * k + 7]) * inv);
+          st_shared4(stage_out + out_off(r, 4 * ch + k), v);
         }
       }
     } else if (lane == 0) {
       report(a.dev_error, PA_DEVERR_TIMEOUT);
       *abort_flag = 1;
+    }
+    // the four softmax warps (named barrier 1), every one of them exactly once
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (__all_sync(kFull, ok)) {
+      const int i = threadIdx.x - 64;  // 0..127
+      const int cc = i & 15;
+#pragma unroll 4
+      for (int k = 0; k < kRows / 8; ++k) {
+        const int rr = 8 * k + (i >> 4);
+        const int gr = r0 + rr;
+        if (gr < rows) {
+          const int tok = gr / G, hh = gr - tok * G;
+          T* dst = static_cast<T*>(a.out) +
+                   (static_cast<int64_t>(q0 + tok) * a.num_q_heads + g * G + hh) * kD;
+          reinterpret_cast<uint4*>(dst)[cc] = ld_shared4(stage_out + out_off(rr, cc));
+        }
+      }
     }
   }
 
@@ -540,8 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <typename T>
-static cudaError_t launch_t(const PrefillArgs& a, const CUtensorMap& kmap, const CUtensorMap& vmap,
-                            int tiles, cudaStream_t stream) {
+static cudaError_t launch_t(const PrefillArgs& a, const CUtensorMap& qmap, const CUtensorMap& kmap,
+                            const CUtensorMap& vmap, int tiles, cudaStream_t stream) {
   auto kern = prefill_tc5_kernel<T>;
   static bool raised[64] = {};
   int dev = 0;
@@ -553,20 +656,20 @@ static cudaError_t launch_t(const PrefillArgs& a, const CUtensorMap& kmap, const
     if (dev >= 0 && dev < 64) raised[dev] = true;
   }
   dim3 grid(tiles, a.num_kv_heads, a.batch);
-  kern<<<grid, kThreads, kSmem, stream>>>(kmap, vmap, a);
+  kern<<<grid, kThreads, kSmem, stream>>>(qmap, kmap, vmap, a);
   return cudaGetLastError();
 }
 
 }  // namespace t5
 
-// 2-D maps {head_dim, rows} with a {64, 16} box, 128-byte swizzle: one 16-key
-// group of one 64-column block per copy.
-cudaError_t launch_prefill_tc5(const PrefillArgs& a, pa_dtype dtype, const CUtensorMap& kmap2d,
-                               const CUtensorMap& vmap2d, cudaStream_t stream) {
+cudaError_t launch_prefill_tc5(const PrefillArgs& a, pa_dtype dtype, const CUtensorMap& qmap,
+                               const CUtensorMap& kmap2d, const CUtensorMap& vmap2d,
+                               cudaStream_t stream) {
   const int64_t tiles = (static_cast<int64_t>(a.max_q) * a.group + t5::kRows - 1) / t5::kRows;
   return dtype == PA_F16
-             ? t5::launch_t<__half>(a, kmap2d, vmap2d, static_cast<int>(tiles), stream)
-             : t5::launch_t<__nv_bfloat16>(a, kmap2d, vmap2d, static_cast<int>(tiles), stream);
+             ? t5::launch_t<__half>(a, qmap, kmap2d, vmap2d, static_cast<int>(tiles), stream)
+             : t5::launch_t<__nv_bfloat16>(a, qmap, kmap2d, vmap2d, static_cast<int>(tiles),
+                                           stream);
 }
 
 }  // namespace pa
