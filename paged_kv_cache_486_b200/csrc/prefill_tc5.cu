@@ -17,10 +17,11 @@
 //                      memory (MN-major: head_dim contiguous), fp32 in TMEM.
 // bf16 keeps P as a head + tail pair (two products), fp16 a single value.
 //
-// Warps: 0 loads Q once and the K / V tiles (TMA; K and V have their own
-// stages, so the next keys load as soon as S is done), 1 allocates TMEM and
-// issues every UMMA from one thread, as soon as each product's inputs are
-// ready, 2..5 run the softmax and the epilogue (warp w reads TMEM lanes
+// Warps: 0 loads Q once and the K tiles, 6 the V tiles (TMA, each tensor with
+// its own stages, so keys load as soon as an S product has released their
+// stage, whatever the P . V products are doing), 1 allocates TMEM and issues
+// every UMMA from one thread, as soon as each product's inputs are ready,
+// 2..5 run the softmax and the epilogue (warp w reads TMEM lanes
 // 32 (w mod 4) .. +31, which are its rows).  S / P has three buffers in TMEM
 // (columns 0, 128, 256), so the tensor core computes the next tile's scores
 // while the softmax works on this one, and the softmax writes the next P
@@ -30,7 +31,7 @@
 //
 // Shared memory (1024-byte aligned, every tile in 64-column blocks of rows of
 // 128 bytes, 128-byte swizzle): Q 32 KB (O is staged there for coalesced
-// stores at the end), K and V 32 KB per stage.  That keeps one CTA per SM, so
+// stores at the end), K 3 x 32 KB, V 2 x 32 KB.  That keeps one CTA per SM, so
 // the 512-column TMEM allocation never waits.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -47,15 +48,17 @@ using tc::kFull;
 constexpr int kRows = 128;   // query rows per CTA
 constexpr int kKeys = 128;   // keys per tile
 constexpr int kD = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
+constexpr int kVWarp = 6;                  // the V producer (warp 0 loads Q and K)
 constexpr int kColBlock = kRows * 128;     // one 64-column block of 128 rows: 16 KB
 constexpr int kTileBytes = 2 * kColBlock;  // 128 rows x 128 columns x 2 bytes
 constexpr int kGroupBytes = 16 * 128;      // 16 rows of one 64-column block
-constexpr int kStages = 2;                 // K and V tiles in flight, each
+constexpr int kKStages = 3;                // K tiles in flight
+constexpr int kVStages = 2;                // V tiles in flight
 constexpr int kQOff = 0;
 constexpr int kKOff = kTileBytes;
-constexpr int kVOff = kKOff + kStages * kTileBytes;
-constexpr int kRing = kVOff + kStages * kTileBytes;  // 160 KB at two stages
+constexpr int kVOff = kKOff + kKStages * kTileBytes;
+constexpr int kRing = kVOff + kVStages * kTileBytes;  // 192 KB
 constexpr int kSmem = 1024 + kRing + 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBuf = 3;  // S / P buffers in TMEM
@@ -241,14 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kRing);
-  // barriers: k_full, k_empty, v_full, v_empty (one per stage each), then per
-  // S / P buffer s_full (scores written), p_full (P written), pv_done (its
-  // P . V completed), then q_full, final
-  constexpr int kB = 4 * kStages;
+  // barriers: k_full, k_empty (one per K stage each), v_full, v_empty (one per
+  // V stage each), then per S / P buffer s_full (scores written), p_full (P
+  // written), pv_done (its P . V completed), then q_full, final
+  constexpr int kB = 2 * (kKStages + kVStages);
   const uint32_t b_k_full = tc::smem_u32(&bars[0]);
-  const uint32_t b_k_empty = tc::smem_u32(&bars[kStages]);
-  const uint32_t b_v_full = tc::smem_u32(&bars[2 * kStages]);
-  const uint32_t b_v_empty = tc::smem_u32(&bars[3 * kStages]);
+  const uint32_t b_k_empty = tc::smem_u32(&bars[kKStages]);
+  const uint32_t b_v_full = tc::smem_u32(&bars[2 * kKStages]);
+  const uint32_t b_v_empty = tc::smem_u32(&bars[2 * kKStages + kVStages]);
   const uint32_t b_s_full = tc::smem_u32(&bars[kB]);
   const uint32_t b_p_full = tc::smem_u32(&bars[kB + kSBuf]);
   const uint32_t b_pv_done = tc::smem_u32(&bars[kB + 2 * kSBuf]);
@@ -307,16 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ============================ Q, K / V producer ============================
+  if (warp == 0 || warp == kVWarp) {
+    // ======================== Q and K / V producers =========================
+    const int which = warp == 0 ? 0 : 1;  // 0: keys (and Q), 1: values
+    const int n_st = which ? kVStages : kKStages;
     // Q: the CTA's 128 rows are 128 / G consecutive tokens x the G heads of kv
     // head g, one {64, G, 128 / G} box per 64-column block (rows past the
     // sequence's tokens are other tokens or zeros; their rows are never stored).
-    if (lane == 0) {
+    if (which == 0 && lane == 0) {
       tc::mbar_arrive_expect_tx(b_q_full, kTileBytes);
       tma_3d(base + kQOff, &qmap, 0, g * G, q0 + r0 / G, b_q_full);
       tma_3d(base + kQOff + kColBlock, &qmap, 64, g * G, q0 + r0 / G, b_q_full);
     }
+    const uint32_t full0 = which ? b_v_full : b_k_full;
+    const uint32_t empty0 = which ? b_v_empty : b_k_empty;
+    const uint32_t ring = base + (which ? kVOff : kKOff);
+    const T* src = static_cast<const T*>(which ? a.v_cache : a.k_cache);
+    const CUtensorMap* map = which ? &vmap : &kmap;
     // Lane k (< 8) reads the block id of 16-key group k of the next tile while
     // this one is loaded; an id is checked where it is used.
     const int32_t* bt = a.block_tables + static_cast<int64_t>(b) * a.max_blocks;
@@ -325,15 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       return (lane < 8 && key < n_keys) ? __ldg(&bt[key / bs]) : -1;
     };
     int id_next = raw_id(0);
-    bool live = true;
-    for (int t = 0; t < n_tiles && live && !*abort_flag; ++t) {
-      const int stage = t % kStages;
+    for (int t = 0; t < n_tiles && !*abort_flag; ++t) {
+      const int stage = t % n_st;
       const int n_grp = t == n_tiles - 1 ? n_last / 16 : kKeys / 16;
       int id_mine = id_next;
       if (t + 1 < n_tiles) id_next = raw_id(t + 1);
       const int key_mine = t * kKeys + 16 * (lane & 7);
       if (lane < n_grp && key_mine < n_keys && (id_mine < 0 || id_mine >= a.num_blocks)) {
-        report(a.dev_error, PA_DEVERR_BAD_BLOCK);
+        if (which == 0) report(a.dev_error, PA_DEVERR_BAD_BLOCK);
         id_mine = -1;
       }
       // whole groups in a valid block go by tensor map; the group holding key
@@ -345,52 +354,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t hand_mask = __ballot_sync(kFull, lane < n_grp) & ~tma_mask;
       const int row_mine =
           (id_mine < 0 ? 0 : id_mine * a.num_kv_heads + g) * bs + key_mine % bs;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {  // 0: keys, 1: values
-        const uint32_t full = (which ? b_v_full : b_k_full) + 8 * stage;
-        const uint32_t empty = (which ? b_v_empty : b_k_empty) + 8 * stage;
-        if (t >= kStages &&
-            !__all_sync(kFull, tc::mbar_wait_bounded(empty, ((t / kStages) - 1) & 1))) {
-          if (lane == 0) {
-            report(a.dev_error, PA_DEVERR_TIMEOUT);
-            *abort_flag = 1;
-          }
-          live = false;
-          break;
-        }
-        const uint32_t dst = base + (which ? kVOff : kKOff) + stage * kTileBytes;
-        if (hand_mask) {
-          const T* src = static_cast<const T*>(which ? a.v_cache : a.k_cache);
-          for (int k = 0; k < kKeys / 16; ++k) {
-            if (!(hand_mask >> k & 1)) continue;
-            const int id = __shfl_sync(kFull, id_mine, k);
-            const int key = t * kKeys + 16 * k;
-            const int valid = id >= 0 ? min(16, n_keys - key) : 0;
-            const T* rows0 = src + (static_cast<int64_t>(id < 0 ? 0 : id * a.num_kv_heads + g) *
-                                        bs + key % bs) * kD;
-            for (int i = lane; i < 16 * 16; i += 32) {
-              const int rr = i >> 4, c = i & 15;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (rr < valid) v = __ldg(reinterpret_cast<const uint4*>(rows0 + rr * kD) + c);
-              st_shared4(dst + tile_off(16 * k + rr, c), v);
-            }
-          }
-          // generic writes above are read by the tensor core (async proxy)
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        __syncwarp();
+      const uint32_t full = full0 + 8 * stage;
+      if (t >= n_st &&
+          !__all_sync(kFull, tc::mbar_wait_bounded(empty0 + 8 * stage, ((t / n_st) - 1) & 1))) {
         if (lane == 0) {
-          if (tma_mask)
-            tc::mbar_arrive_expect_tx(full, __popc(tma_mask) * 2 * kGroupBytes);
-          else
-            tc::mbar_arrive(full);
+          report(a.dev_error, PA_DEVERR_TIMEOUT);
+          *abort_flag = 1;
         }
-        __syncwarp();
-        if (tma_mask >> lane & 1) {
-          const CUtensorMap* map = which ? &vmap : &kmap;
-          tma_2d(dst + lane * kGroupBytes, map, 0, row_mine, full);
-          tma_2d(dst + kColBlock + lane * kGroupBytes, map, 64, row_mine, full);
+        break;
+      }
+      const uint32_t dst = ring + stage * kTileBytes;
+      if (hand_mask) {
+        for (int k = 0; k < kKeys / 16; ++k) {
+          if (!(hand_mask >> k & 1)) continue;
+          const int id = __shfl_sync(kFull, id_mine, k);
+          const int key = t * kKeys + 16 * k;
+          const int valid = id >= 0 ? min(16, n_keys - key) : 0;
+          const T* rows0 = src + (static_cast<int64_t>(id < 0 ? 0 : id * a.num_kv_heads + g) *
+                                      bs + key % bs) * kD;
+          for (int i = lane; i < 16 * 16; i += 32) {
+            const int rr = i >> 4, c = i & 15;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (rr < valid) v = __ldg(reinterpret_cast<const uint4*>(rows0 + rr * kD) + c);
+            st_shared4(dst + tile_off(16 * k + rr, c), v);
+          }
         }
+        // generic writes above are read by the tensor core (async proxy)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (tma_mask)
+          tc::mbar_arrive_expect_tx(full, __popc(tma_mask) * 2 * kGroupBytes);
+        else
+          tc::mbar_arrive(full);
+      }
+      __syncwarp();
+      if (tma_mask >> lane & 1) {
+        tma_2d(dst + lane * kGroupBytes, map, 0, row_mine, full);
+        tma_2d(dst + kColBlock + lane * kGroupBytes, map, 64, row_mine, full);
       }
     }
   } else if (warp == 1) {
@@ -409,12 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool ready = __shfl_sync(
             kFull, leader ? ((ns < kSBuf || mbar_test(b_pv_done + 8 * (ns % kSBuf),
                                                       ((ns - kSBuf) / kSBuf) & 1)) &&
-                             mbar_test(b_k_full + 8 * (ns % kStages), (ns / kStages) & 1))
+                             mbar_test(b_k_full + 8 * (ns % kKStages), (ns / kKStages) & 1))
                           : false, 0);
         if (ready) {
           if (leader) {
             fence_after();
-            const uint32_t kt = base + kKOff + (ns % kStages) * kTileBytes;
+            const uint32_t kt = base + kKOff + (ns % kKStages) * kTileBytes;
             const uint32_t d = tmem + kColS + (ns % kSBuf) * kKeys;
             const uint32_t id = idesc(kAB, 0, ns == n_tiles - 1 ? n_last : kKeys);
 #pragma unroll
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_ss(d, smem_desc(q_s + off, 16, 1024), smem_desc(kt + off, 16, 1024), id, s > 0);
             }
             commit(b_s_full + 8 * (ns % kSBuf));
-            commit(b_k_empty + 8 * (ns % kStages));  // K_ns may be refilled
+            commit(b_k_empty + 8 * (ns % kKStages));  // K_ns may be refilled
           }
           ++ns;
           progress = true;
@@ -432,12 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (npv < ns) {
         const bool ready = __shfl_sync(
             kFull, leader ? (mbar_test(b_p_full + 8 * (npv % kSBuf), (npv / kSBuf) & 1) &&
-                             mbar_test(b_v_full + 8 * (npv % kStages), (npv / kStages) & 1))
+                             mbar_test(b_v_full + 8 * (npv % kVStages), (npv / kVStages) & 1))
                           : false, 0);
         if (ready) {
           if (leader) {
             fence_after();
-            const uint32_t vt = base + kVOff + (npv % kStages) * kTileBytes;
+            const uint32_t vt = base + kVOff + (npv % kVStages) * kTileBytes;
             const uint32_t p = tmem + kColS + (npv % kSBuf) * kKeys;  // P head: columns 0..63
             const int steps = npv == n_tiles - 1 ? n_last / 16 : kKeys / 16;
             constexpr uint32_t kIdO = idesc(kAB, 1, kD);
@@ -446,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_ts(tmem + kColO, p + 8 * s, bd, kIdO, (npv > 0 || s > 0) ? 1u : 0u);
               if (PrefillPSplit<T>::value) mma_ts(tmem + kColO, p + 64 + 8 * s, bd, kIdO, 1u);
             }
-            commit(b_v_empty + 8 * (npv % kStages));  // V_npv may be refilled
+            commit(b_v_empty + 8 * (npv % kVStages));  // V_npv may be refilled
             commit(b_pv_done + 8 * (npv % kSBuf));    // O holds P_0 .. P_npv
           }
           ++npv;
