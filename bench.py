@@ -673,7 +673,7 @@ def run_prefill(args, dist, rank, world):
 
     def run():
         pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
-                                eng.dev_error, args.prefill_path)
+                                eng.dev_error, args.prefill_path, eng.prefill_ws)
 
     ms = []
     for it in range(args.warmup + args.steps):

@@ -363,10 +363,12 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  * head_dim 64 or 128; num_q_heads / num_kv_heads a divisor of 64; block_size a
  * multiple of 16; batch <= 65535.  One launch.  head_dim 128 (with a group
  * dividing 128 and scale > 0) runs on the 5th-generation tensor cores (tcgen05 UMMA with
- * TMEM accumulators, 128 (token, head) rows of one kv head per CTA, K / V
- * tiles of 128 keys); otherwise mma.sync (64 rows, 64-key tiles).
- * Alignment: k_cache, v_cache 16 bytes; q, out 4 (q 16 for the tcgen05
- * kernel, which the automatic choice then skips).  Errors: PA_ERR_INVALID for
+ * TMEM accumulators; persistent, one CTA per SM walking items of 128 (token,
+ * head) rows of one kv head, K / V tiles of 128 keys); otherwise mma.sync (64
+ * rows per CTA, 64-key tiles).
+ * Alignment: k_cache, v_cache 16 bytes; q, out 4 (16 for the tcgen05
+ * kernel, which the automatic choice then skips).  max_q * (num_q_heads /
+ * num_kv_heads) < 2^31 - 256.  Errors: PA_ERR_INVALID for
  * shapes or pointers outside these limits, nothing launched.
  * ---------------------------------------------------------------------- */
 pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
@@ -379,21 +381,32 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
 
 /* Kernels for pa_prefill_attention_ex. */
 #define PA_PREFILL_AUTO 0      /* tcgen05 where it applies, else mma.sync */
-#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, scale > 0, q 16-byte
-                                  aligned */
+#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, scale > 0, q and out
+                                  16-byte aligned */
 #define PA_PREFILL_MMA_SYNC 2  /* every supported shape */
 
+/* Bytes of the optional scheduling workspace of pa_prefill_attention_ex. */
+#define PA_PREFILL_WORKSPACE_BYTES 16
+
 /* pa_prefill_attention with the kernel chosen by the caller (same results up to
- * fp32 rounding order).  An unknown path, or PA_PREFILL_TCGEN05 for a shape it
- * does not take, is PA_ERR_INVALID with nothing launched. */
+ * fp32 rounding order), and an optional scheduling workspace.
+ * workspace: NULL, or PA_PREFILL_WORKSPACE_BYTES of device memory, 8-byte
+ *   aligned, owned by the caller, zero-filled once before its first use (e.g.
+ *   cudaMemset); every call leaves it zero.  With it the tcgen05 kernel is
+ *   persistent (one CTA per SM taking 128-row items, longest first, from a
+ *   counter there), without it each CTA runs one item; the results are the
+ *   same bits.  Calls sharing one workspace must not overlap on the GPU (order
+ *   them on one stream).  The mma.sync kernel ignores it.
+ * An unknown path, or PA_PREFILL_TCGEN05 for a shape it does not take, is
+ * PA_ERR_INVALID with nothing launched. */
 pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
                                   const void* v_cache, const int32_t* block_tables,
                                   const int32_t* context_lens, const int32_t* query_start,
                                   int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                   int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                   int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
-                                  pa_dtype dtype, int32_t* dev_error, int32_t path,
-                                  pa_stream stream);
+                                  pa_dtype dtype, int32_t* dev_error, void* workspace,
+                                  int32_t path, pa_stream stream);
 
 /* ------------------------------------------------------------------------
  * INT8 KV cache.  [P5] "The four solutions", KV-cache quantisation: keys and

@@ -22,6 +22,7 @@ PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 PA_PATH_AUTO, PA_PATH_TC, PA_PATH_SIMT = 0, 1, 2
 PA_DECODE_OVERLAP_PROLOGUE = 1
 PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA_SYNC = 0, 1, 2
+PA_PREFILL_WORKSPACE_BYTES = 16
 PA_DEVERR_BAD_SLOT, PA_DEVERR_BAD_BLOCK, PA_DEVERR_BAD_CTX, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 DTYPE_CODE = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
@@ -63,7 +64,8 @@ SIGNATURES = {
     "pa_prefill_attention": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                     _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _P]),
     "pa_prefill_attention_ex": (_I32, [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
-                                       _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _I32, _P]),
+                                       _I32, _I32, _I32, _I32, C.c_float, C.c_int, _P, _P, _I32,
+                                       _P]),
     "pa_int8_block_bytes": (C.c_size_t, [_I32, _I32, _I32]),
     "pa_reshape_and_cache_int8": (_I32, [_P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
                                          C.c_int, _P, _P]),
@@ -338,23 +340,28 @@ def pa_decode_attention_static_ws(out, q, k_cache, v_cache, block_tables, contex
 
 
 def pa_prefill_attention(out, q, k_cache, v_cache, block_tables, context_lens, query_start,
-                         max_q, scale, dev_error=None, path=PA_PREFILL_AUTO, stream=None):
+                         max_q, scale, dev_error=None, path=PA_PREFILL_AUTO, workspace=None,
+                         stream=None):
     """Causal attention of each sequence's new tokens over its paged cache: q/out
     [T, Hq, D] fp16 or bf16, query_start int32 [B+1] (device), max_q >= every
-    query_start[b+1] - query_start[b]; caches and tables as pa_decode_attention."""
+    query_start[b+1] - query_start[b]; caches and tables as pa_decode_attention.
+    workspace: None or int64 [2] zero-filled once (persistent tcgen05 kernel)."""
     T, Hq, D = q.shape
     NB, Hkv, bs, _ = k_cache.shape
     B = context_lens.shape[0]
     MB = block_tables.shape[1]
     if out.shape != q.shape or query_start.shape[0] != B + 1:
         raise ValueError("out must have q's shape and query_start batch + 1 entries")
+    if workspace is not None and workspace.numel() * workspace.element_size() < \
+            PA_PREFILL_WORKSPACE_BYTES:
+        raise ValueError(f"workspace needs {PA_PREFILL_WORKSPACE_BYTES} bytes")
     st = lib.pa_prefill_attention_ex(
         _dev_ptr(out, "out", q.dtype), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache", q.dtype),
         _dev_ptr(v_cache, "v_cache", q.dtype), _dev_ptr(block_tables, "block_tables", torch.int32),
         _dev_ptr(context_lens, "context_lens", torch.int32),
         _dev_ptr(query_start, "query_start", torch.int32), B, Hq, Hkv, D, bs, NB, MB, T, int(max_q),
-        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32), path,
-        _stream(stream))
+        float(scale), DTYPE_CODE[q.dtype], _dev_ptr(dev_error, "dev_error", torch.int32),
+        _dev_ptr(workspace, "workspace", torch.int64), path, _stream(stream))
     _check(st, "pa_prefill_attention")
 
 

@@ -93,8 +93,9 @@ bool make_tile_map(CUtensorMap* map, bool* three_d, const void* base, int64_t ro
          CUDA_SUCCESS;
 }
 
-// q as {head_dim, num_q_heads, total_q} with a {64, group, 128 / group} box:
-// 128 rows of (token, head of one kv head's group) pairs per 64-column block.
+// q (or out) as {head_dim, num_q_heads, total_q} with a {64, group, 128 /
+// group} box: 128 rows of (token, head of one kv head's group) pairs per
+// 64-column block.
 static bool make_q_map(CUtensorMap* map, const void* q, int total_q, int num_q_heads,
                        int head_dim, int group, pa_dtype dt) {
   auto enc = encode_fn();
@@ -572,8 +573,8 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
                                   int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
                                   int32_t head_dim, int32_t block_size, int32_t num_blocks,
                                   int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
-                                  pa_dtype dtype, int32_t* dev_error, int32_t path,
-                                  pa_stream stream) {
+                                  pa_dtype dtype, int32_t* dev_error, void* workspace,
+                                  int32_t path, pa_stream stream) {
   if (path != PA_PREFILL_AUTO && path != PA_PREFILL_TCGEN05 && path != PA_PREFILL_MMA_SYNC)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: unknown path %d", path);
   if (dtype != PA_F16 && dtype != PA_BF16)
@@ -597,26 +598,29 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
       static_cast<int64_t>(max_blocks) * block_size >= (int64_t(1) << 31))
     return fail(PA_ERR_INVALID, "pa_prefill_attention: pool or table too large");
   const int group = num_q_heads / num_kv_heads;
-  if ((static_cast<int64_t>(max_q) * group + 63) / 64 > INT32_MAX)
+  if (static_cast<int64_t>(max_q) * group > INT32_MAX - 256)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: max_q too large");
   if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_prefill_attention: scale is NaN");
   if (batch == 0 || max_q == 0 || total_q == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: NULL pointer");
   if (!aligned(q, 4) || !aligned(out, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4))
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start, 4) ||
+      !aligned(workspace, 8))
     return fail(PA_ERR_INVALID, "pa_prefill_attention: misaligned pointer");
-  const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16) && scale > 0.f;
+  const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16) &&
+                      aligned(out, 16) && scale > 0.f;
   if (path == PA_PREFILL_TCGEN05 && !tc5_ok)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: the tcgen05 kernel needs head_dim 128, "
-                "num_q_heads / num_kv_heads dividing 128, scale > 0 and q 16-byte aligned");
+                "num_q_heads / num_kv_heads dividing 128, scale > 0 and q, out 16-byte aligned");
   const bool use_tc5 = path == PA_PREFILL_TCGEN05 || (path == PA_PREFILL_AUTO && tc5_ok);
-  CUtensorMap qmap, kmap, vmap;
+  CUtensorMap qmap, omap, kmap, vmap;
   bool k3 = false, v3 = false;
   if (use_tc5) {
     if (!make_q_map(&qmap, q, total_q, num_q_heads, head_dim, group, dtype) ||
+        !make_q_map(&omap, out, total_q, num_q_heads, head_dim, group, dtype) ||
         !make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
-        !make_tile_map_2d(&vmap, v_cache, rows, head_dim, dtype))
+        !make_tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || !v3)
       return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
   } else if (!tile_map(&kmap, &k3, k_cache, rows, head_dim, dtype) ||
              !tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || k3 != v3) {
@@ -643,8 +647,10 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   a.scale_log2 = scale * 1.4426950408889634f;
   a.k_cache = k_cache;
   a.v_cache = v_cache;
+  a.tiles = 0;
+  a.sched = static_cast<uint64_t*>(workspace);
   const cudaError_t e =
-      use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap,
+      use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap, omap,
                                        static_cast<cudaStream_t>(stream))
               : pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
@@ -660,7 +666,7 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
   return pa_prefill_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens,
                                  query_start, batch, num_q_heads, num_kv_heads, head_dim,
                                  block_size, num_blocks, max_blocks, total_q, max_q, scale, dtype,
-                                 dev_error, PA_PREFILL_AUTO, stream);
+                                 dev_error, nullptr, PA_PREFILL_AUTO, stream);
 }
 
 pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_stream stream) {

@@ -32,6 +32,8 @@ class PagedKVCache:
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
         ws = pa_decode_workspace_size(max_batch, num_q_heads, num_kv_heads, head_dim)
         self.workspace = torch.zeros(ws, dtype=torch.uint8, device=self.device)
+        # prefill's item counter (persistent tcgen05 kernel); every call leaves it zero
+        self.prefill_ws = torch.zeros(2, dtype=torch.int64, device=self.device)
 
     # ---- pool ops (host) with their device side effects ----
     def alloc(self, seq_id, n, stream=None):
@@ -104,7 +106,8 @@ class PagedKVCache:
         if out is None:
             out = torch.empty_like(q)
         pa_prefill_attention(out, q, self.k_cache, self.v_cache, block_tables, context_lens,
-                             query_start, max_q, scale, self.dev_error, path, stream)
+                             query_start, max_q, scale, self.dev_error, path, self.prefill_ws,
+                             stream)
         return out
 
     def device_errors(self, stream=None):

@@ -134,3 +134,25 @@ def test_prefill_guards(path):
     eng.prefill(q[:0], bt, ctx, empty, 0, wl.scale, path=path)
     torch.cuda.synchronize()
     assert eng.device_errors() == 0
+
+
+@pytest.mark.parametrize("name", ["f16_g4_d128", "bf16_g8_d128", "f16_g1_bs32"])
+def test_prefill_persistent_and_per_item_launches_agree(name):
+    """The tcgen05 kernel with a scheduling workspace (persistent, items handed
+    out by a counter) and without (one item per CTA) computes every item the
+    same way: identical bits, and the workspace is left zero for the next call."""
+    wl = CASES[name]()
+    eng, bt, ctx, qs, q = _build(wl)
+    max_q = int(wl.n_new.max())
+    ws = torch.zeros(2, dtype=torch.int64, device="cuda")
+    outs = []
+    for workspace in (ws, None, ws):
+        out = torch.full_like(q, float("nan"))
+        pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
+                                eng.dev_error, pa.PA_PREFILL_TCGEN05, workspace)
+        torch.cuda.synchronize()
+        outs.append(out)
+        assert not ws.any(), "the scheduling counter was not returned to zero"
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
+    assert eng.device_errors() == 0
