@@ -65,24 +65,29 @@ def _peak_tensor():
         return 1590.0, "fallback"
 
 
-def _kernel_sha():
+DECODE_SOURCES = ("decode_tc.cuh", "decode_tc.cu", "decode_common.cuh", "decode_simt.cu")
+PREFILL_SOURCES = ("prefill_tc5.cu", "prefill_launch.h", "decode_tc.cuh", "decode_common.cuh")
+INT8_SOURCES = ("decode_tc.cuh", "decode_int8.cu", "decode_common.cuh", "int8_launch.h")
+
+
+def _kernel_sha(names=DECODE_SOURCES):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_486_b200", "csrc")
-    for name in ("decode_tc.cuh", "decode_tc.cu", "decode_common.cuh", "decode_simt.cu"):
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def _traffic(config):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+def _traffic(config, names=DECODE_SOURCES):
+    """DRAM bytes per launch of the timed kernel from the committed ncu summary, if
+    it was taken on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         e = d.get(config)
-        if e and e.get("kernel_sha") == _kernel_sha():
+        if e and e.get("kernel_sha") == _kernel_sha(names):
             return e["dram_bytes_per_launch"]
     except (OSError, ValueError):
         pass
@@ -548,7 +553,7 @@ def run_int8(args, dist, rank, world):
         "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3, "decode_us_min": min(decode_ms) * 1e3,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
-                     "traffic": None,
+                     "traffic": _traffic(wl.name + "_int8", INT8_SOURCES),
                      "timed": "pa_decode_attention_int8 call (one kernel), graph replay"},
         "gpu_launches": launches * args.steps, "clocks": clocks,
     }
@@ -708,7 +713,9 @@ def run_prefill(args, dist, rank, world):
                    "l2": "flushed between timed calls (256 MiB read outside the events)"},
         "prefill_us": 1e3 * statistics.mean(ms), "kv_read_bytes": kv_bytes,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tflops / peak, "peak_source": kind, "traffic": None,
+                     "frac": tflops / peak, "peak_source": kind,
+                     "traffic": (_traffic(wl.name, PREFILL_SOURCES)
+                                 if args.prefill_path != 2 and wl.D == 128 else None),
                      "timed": "pa_prefill_attention (one kernel, " +
                               ("mma.sync m16n8k16" if args.prefill_path == 2 or wl.D != 128
                                else "tcgen05 UMMA, TMEM accumulators") + ")"},
