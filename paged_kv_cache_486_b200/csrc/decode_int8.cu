@@ -23,6 +23,8 @@
 //
 // Roofline.  Per context token and KV head the kernel must read 128 + 128 bytes
 // of codes and 4 + 4 bytes of scales: 264 bytes against 512 for fp16.
+#include <type_traits>
+
 #include "decode_tc.cuh"
 #include "int8_launch.h"
 
@@ -178,18 +180,30 @@ struct Tiles8 {
       seg.inv = 1.f / mx;
     }
     const float u0 = w0 * seg.inv, u1 = w1 * seg.inv;
-    uint32_t h01, t01, h23, t23;
-    split2<T>(p[0] * u0, p[1] * u0, h01, t01);
-    split2<T>(p[2] * u1, p[3] * u1, h23, t23);
+    // fp16 weights (11-bit significand, p' <= 2^12) in one product; bf16 as a
+    // head + tail pair, whose 8-bit significand alone would cost ~2^-9 |v|
+    constexpr bool kSplit = !std::is_same<T, __half>::value;
+    uint32_t h01, t01 = 0, h23, t23 = 0;
+    if (kSplit) {
+      split2<T>(p[0] * u0, p[1] * u0, h01, t01);
+      split2<T>(p[2] * u1, p[3] * u1, h23, t23);
+    } else {
+      h01 = pack2<T>(p[0] * u0, p[1] * u0);
+      h23 = pack2<T>(p[2] * u1, p[3] * u1);
+    }
     const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
-    const uint32_t pt[2] = {transpose8x8(t01), transpose8x8(t23)};
+    uint32_t pt[2] = {0u, 0u};
+    if (kSplit) {
+      pt[0] = transpose8x8(t01);
+      pt[1] = transpose8x8(t23);
+    }
 #pragma unroll
     for (int mt = 0; mt < KC; ++mt) {
       const uint2 r0 = codes_to<T>(f.v[mt][0]);
       const uint2 r1 = codes_to<T>(f.v[mt][1]);
       const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
       mma16816<T>(o[mt], A, pb);
-      mma16816<T>(o[mt], A, pt);
+      if (kSplit) mma16816<T>(o[mt], A, pt);
     }
   }
 };
