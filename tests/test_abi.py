@@ -160,3 +160,43 @@ def test_int8_block_bytes():
     assert pa.pa_int8_block_bytes(8, 128, 64) == 8 * 4 * 2112
     assert pa.pa_int8_block_bytes(8, 64, 16) == 0
     assert pa.pa_int8_block_bytes(8, 128, 8) == 0
+
+
+def _prefill_args(**kw):
+    p = C.c_void_p(16)
+    args = dict(out=p, q=p, kc=p, vc=p, bt=p, ctx=p, qs=p, B=4, Hq=8, Hkv=2, D=128, bs=16, NB=10,
+                MB=4, T=8, max_q=4, scale=0.1, dtype=pa.PA_F16, err=None, ws=None,
+                path=pa.PA_PREFILL_AUTO, stream=None)
+    args.update(kw)
+    return args
+
+
+def _call_prefill(a):
+    return pa.lib.pa_prefill_attention_ex(
+        a["out"], a["q"], a["kc"], a["vc"], a["bt"], a["ctx"], a["qs"], a["B"], a["Hq"], a["Hkv"],
+        a["D"], a["bs"], a["NB"], a["MB"], a["T"], a["max_q"], a["scale"], a["dtype"], a["err"],
+        a["ws"], a["path"], a["stream"])
+
+
+@pytest.mark.parametrize("bad", [
+    dict(path=3), dict(path=-1), dict(dtype=pa.PA_F32), dict(T=-1), dict(B=-1), dict(B=70000),
+    dict(Hkv=0), dict(Hq=7), dict(Hq=256, Hkv=2), dict(D=96), dict(bs=8), dict(bs=24),
+    dict(NB=-1), dict(max_q=1 << 30), dict(scale=float("nan")), dict(kc=None),
+    dict(q=C.c_void_p(2)), dict(kc=C.c_void_p(8)), dict(ws=C.c_void_p(4)),
+    # the tcgen05 kernel asked for where it does not apply
+    dict(path=pa.PA_PREFILL_TCGEN05, D=64), dict(path=pa.PA_PREFILL_TCGEN05, scale=-1.0),
+    dict(path=pa.PA_PREFILL_TCGEN05, q=C.c_void_p(20)),
+    dict(path=pa.PA_PREFILL_TCGEN05, out=C.c_void_p(36)),
+])
+def test_prefill_rejects_bad_arguments_on_host(bad):
+    """Every limit pa.h states for pa_prefill_attention_ex is checked before anything
+    reaches the device: PA_ERR_INVALID with a message, nothing launched."""
+    st = _call_prefill(_prefill_args(**bad))
+    assert st == pa.PA_ERR_INVALID, pa.pa_last_error()
+    assert pa.pa_last_error()
+
+
+def test_prefill_empty_calls_are_no_ops():
+    assert _call_prefill(_prefill_args(B=0, q=None, out=None)) == pa.PA_OK
+    assert _call_prefill(_prefill_args(max_q=0)) == pa.PA_OK
+    assert _call_prefill(_prefill_args(T=0)) == pa.PA_OK
