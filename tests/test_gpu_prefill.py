@@ -46,6 +46,9 @@ def _cases():
                                       34),
         "f16_mqa_g16": lambda: P("e", "f16", 16, 1, 128, 16, [5, 250, 999], [5, 250, 31], 35),
         "f16_g64_d64": lambda: P("f", "f16", 64, 1, 64, 16, [7, 90], [7, 45], 36),
+        # large groups at head_dim 128: the tcgen05 kernel's query boxes of 4 and 2 tokens
+        "bf16_g32_d128": lambda: P("g", "bf16", 64, 2, 128, 16, [3, 70, 260], [3, 37, 260], 37),
+        "f16_g64_d128": lambda: P("h", "f16", 64, 1, 128, 32, [130, 9], [66, 9], 38),
     }
 
 
