@@ -422,11 +422,12 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
  * [num_blocks, num_kv_heads, block_size / 16] records of 2112 bytes, one record
  * per 16-token group of a (block, kv head) (so a pool is
  * pa_int8_block_bytes(...) bytes per block):
- *   key record:   16 lines of 128 signed code bytes, then 16 fp32 key scales
+ * Codes are stored offset-binary: the byte is code + 128 (code XOR 0x80).
+ *   key record:   16 lines of 128 code bytes, then 16 fp32 key scales
  *                 (token order).  Group token t = 4i + 2h + e is on line
  *                 L = 2i + e + 8h; the codes of head_dim 16c .. 16c + 15 sit at
  *                 bytes L * 128 + 16 (c xor (L mod 8)) .. + 15.
- *   value record: 128 rows of 16 signed code bytes (row d: head_dim d of
+ *   value record: 128 rows of 16 code bytes (row d: head_dim d of
  *                 tokens 0 .. 15 in token order), then 16 fp32 value scales.
  * Each record is what the decode kernel keeps in shared memory for one stage,
  * so one bulk copy moves it.  Block copies (copy-on-write, eviction) of an

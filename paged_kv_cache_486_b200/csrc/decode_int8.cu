@@ -31,18 +31,17 @@
 namespace pa {
 namespace tc {
 
-// Four int8 codes (bytes of w) as two pairs of 16-bit values: .x = bytes 0, 1,
-// .y = bytes 2, 3.  fp16: 0x64 in the high byte makes 1024 + u with u the
-// biased code c + 128, and 1152 is subtracted.  bf16 (7-bit significand) goes
+// Four codes (bytes of w, stored offset-binary: u = c + 128) as two pairs of
+// 16-bit values: .x = bytes 0, 1, .y = bytes 2, 3.  fp16: 0x64 in the high byte
+// makes 1024 + u, and 1152 is subtracted.  bf16 (7-bit significand) goes
 // through fp32 the same way: 0x4B0000uu is 2^23 + u, minus 2^23 + 128.
 template <typename T>
 __device__ __forceinline__ uint2 codes_to(uint32_t w);
 
 template <>
 __device__ __forceinline__ uint2 codes_to<__half>(uint32_t w) {
-  const uint32_t x = w ^ 0x80808080u;
-  uint32_t lo = __byte_perm(x, 0x64646464u, 0x5140);
-  uint32_t hi = __byte_perm(x, 0x64646464u, 0x7362);
+  uint32_t lo = __byte_perm(w, 0x64646464u, 0x5140);
+  uint32_t hi = __byte_perm(w, 0x64646464u, 0x7362);
   const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));
   const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
   const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
@@ -51,11 +50,10 @@ __device__ __forceinline__ uint2 codes_to<__half>(uint32_t w) {
 
 template <>
 __device__ __forceinline__ uint2 codes_to<__nv_bfloat16>(uint32_t w) {
-  const uint32_t x = w ^ 0x80808080u;
   float f[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
-    f[i] = __uint_as_float(__byte_perm(x, 0x4Bu, 0x4650 + i)) - 8388736.0f;
+    f[i] = __uint_as_float(__byte_perm(w, 0x4Bu, 0x4650 + i)) - 8388736.0f;
   return make_uint2(pack2<__nv_bfloat16>(f[0], f[1]), pack2<__nv_bfloat16>(f[2], f[3]));
 }
 

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_int8_kernel(
     for (int i = 0; i < PER; ++i) {
       c[i] = 0;
       if (scale > 0.f) c[i] = max(-127, min(127, __float2int_rn(__fdiv_rn(x[i], scale))));
-      packed |= (static_cast<uint32_t>(c[i]) & 0xffu) << (8 * i);
+      // stored offset-binary: the byte code + 128 (code XOR 0x80)
+      packed |= ((static_cast<uint32_t>(c[i]) & 0xffu) ^ 0x80u) << (8 * i);
     }
     uint8_t* r = (kind ? v_pool : k_pool) + rec * i8::kRecordBytes;
     if (kind == 0) {
@@ -65,7 +66,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_int8_kernel(
       *reinterpret_cast<uint32_t*>(r + i8::key_byte(i8::key_line(gt), lane * PER)) = packed;
     } else {
 #pragma unroll
-      for (int i = 0; i < PER; ++i) r[(lane * PER + i) * i8::kGroup + gt] = static_cast<uint8_t>(c[i]);
+      for (int i = 0; i < PER; ++i)
+        r[(lane * PER + i) * i8::kGroup + gt] = static_cast<uint8_t>((c[i] & 0xff) ^ 0x80);
     }
     if (lane == 0) reinterpret_cast<float*>(r + i8::kCodeBytes)[gt] = scale;
   }

@@ -113,9 +113,10 @@ def gathered_int8(eng, bt, ctx, b, kvh):
     t = pos % 16
     krec = eng.k_pool[:, kvh][blk, grp]           # [n, 2112] uint8
     vrec = eng.v_pool[:, kvh][blk, grp]
-    kc = torch.gather(krec, 1, _KEY_OFF.to(dev)[t]).view(torch.int8)
+    # codes are stored offset-binary (code + 128)
+    kc = (torch.gather(krec, 1, _KEY_OFF.to(dev)[t]) ^ 0x80).view(torch.int8)
     d = torch.arange(128, device=dev)
-    vc = torch.gather(vrec, 1, d[None, :] * 16 + t[:, None]).view(torch.int8)
+    vc = (torch.gather(vrec, 1, d[None, :] * 16 + t[:, None]) ^ 0x80).view(torch.int8)
     ks = krec[:, 2048:].contiguous().view(torch.float32).gather(1, t[:, None])[:, 0]
     vs = vrec[:, 2048:].contiguous().view(torch.float32).gather(1, t[:, None])[:, 0]
     return kc, vc, ks, vs
