@@ -45,8 +45,8 @@
 // a sequence), K 3 x 32 KB, V 2 x 32 KB.  Q and K tiles are two 64-column
 // blocks of 128 rows (the S product's K-major operands); a V tile is eight
 // 16-key groups of two 64-column blocks of 16 rows, so one 4 KB copy brings a
-// group (fewer, larger copies: the copy engine's requests in flight are what
-// bounds the rate here).
+// group (half the copies of two 2 KB boxes; the P . V operand is described
+// group by group either way).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
