@@ -362,10 +362,11 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  *   untouched) and PA_DEVERR_BAD_CTX is set.
  * head_dim 64 or 128; num_q_heads / num_kv_heads a divisor of 64; block_size a
  * multiple of 16; batch <= 65535.  One launch.  head_dim 128 (with a group
- * dividing 128 and scale > 0) runs on the 5th-generation tensor cores (tcgen05 UMMA with
- * TMEM accumulators; persistent, one CTA per SM walking items of 128 (token,
- * head) rows of one kv head, K / V tiles of 128 keys); otherwise mma.sync (64
- * rows per CTA, 64-key tiles).
+ * dividing 128 and scale > 0) runs on the 5th-generation tensor cores (tcgen05
+ * UMMA with TMEM accumulators; items of 128 (token, head) rows of one kv head,
+ * K / V tiles of 128 keys; here one item per CTA, persistent through
+ * pa_prefill_attention_ex with a workspace); otherwise mma.sync (64 rows per
+ * CTA, 64-key tiles).
  * Alignment: k_cache, v_cache 16 bytes; q, out 4 (16 for the tcgen05
  * kernel, which the automatic choice then skips).  max_q * (num_q_heads /
  * num_kv_heads) < 2^31 - 256.  Errors: PA_ERR_INVALID for
@@ -393,9 +394,9 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
  * workspace: NULL, or PA_PREFILL_WORKSPACE_BYTES of device memory, 8-byte
  *   aligned, owned by the caller, zero-filled once before its first use (e.g.
  *   cudaMemset); every call leaves it zero.  With it the tcgen05 kernel is
- *   persistent (one CTA per SM taking 128-row items, longest first, from a
- *   counter there), without it each CTA runs one item; the results are the
- *   same bits.  Calls sharing one workspace must not overlap on the GPU (order
+ *   persistent (one CTA per SM taking 128-row items from a counter there, by
+ *   sequence and kv head with the latest query tile first), without it each
+ *   CTA runs one item; the results are the same bits.  Calls sharing one workspace must not overlap on the GPU (order
  *   them on one stream).  The mma.sync kernel ignores it.
  * An unknown path, or PA_PREFILL_TCGEN05 for a shape it does not take, is
  * PA_ERR_INVALID with nothing launched. */
