@@ -84,3 +84,17 @@ def test_more_new_tokens_than_context_is_rejected():
     except ValueError:
         return
     raise AssertionError("accepted n_new > ctx")
+
+
+def test_prefill_at_head_dim_128_with_groups_of_8():
+    """The shapes the GPU parity cases run (head_dim 128, eight query heads per kv
+    head): a chunk after context, a whole prompt and a single token, against torch."""
+    wl = workloads.prefill("p128", "f16", 16, 2, 128, 16, [150, 37, 9], [20, 37, 1], 9)
+    o = run_script(wl)
+    qs = workloads.query_start(wl)
+    q = workloads.q_prefill(wl)
+    out = oracle.paged_prefill_attention(raw(q), o["k_cache"], o["v_cache"], o["table"],
+                                         o["ctx"], qs, wl.scale, wl.dtype)
+    for b in range(wl.B):
+        ref = _sdpa_rows(wl, b, q[qs[b]:qs[b + 1]].double())
+        np.testing.assert_allclose(out[qs[b]:qs[b + 1]], ref.numpy(), rtol=1e-12, atol=1e-12)
