@@ -20,15 +20,24 @@ def tol_ok(got, ref, dtype):
     return ok, worst
 
 
-def build(wl, poison=True, batched_step=True, path=0, workers=0, stream=None):
+def _tokens_fn(wl, gen):
+    """tokens(seq, pos0, n) -> device (key, value) rows.  gen='cuda' draws them on the
+    device; gen='cpu' draws them on the host and copies them over (no generator
+    kernels on the device: used where the device's launch list should hold the
+    library's kernels only)."""
+    def tokens(seq, pos0, n):
+        k, v = wl.tokens(seq, pos0, n, 0, gen), wl.tokens(seq, pos0, n, 1, gen)
+        return k.to("cuda"), v.to("cuda")
+    return tokens
+
+
+def build(wl, poison=True, batched_step=True, path=0, workers=0, stream=None, gen="cuda"):
     """Prefill the pools from the op script, then run the decode step: one new
     token per sequence (one batched cache write), then decode attention."""
     dt = workloads.TORCH_DTYPE[wl.dtype]
     eng = PagedKVCache(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda",
                        fill_bits=NAN_BITS[wl.dtype] if poison else None)
-
-    def tokens(seq, pos0, n):
-        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
+    tokens = _tokens_fn(wl, gen)
 
     pre = eng.apply_ops(wl.ops[:wl.n_prefill_ops], tokens, stream)
     step_ops = wl.ops[wl.n_prefill_ops:]
@@ -46,7 +55,7 @@ def build(wl, poison=True, batched_step=True, path=0, workers=0, stream=None):
     else:
         step = eng.apply_ops(step_ops, tokens, stream)
     bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
-    q = wl.q("cuda")
+    q = wl.q(gen).to("cuda")
     out = eng.decode(q, bt, ctx, wl.scale, path=path, num_workers=workers, stream=stream)
     torch.cuda.synchronize()
     return dict(eng=eng, records=pre + step, bt=bt, ctx=ctx, q=q, out=out)
@@ -68,19 +77,15 @@ def bits(t):
     return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)
 
 
-def build_int8(wl, poison=True, workers=0, stream=None):
+def build_int8(wl, poison=True, workers=0, stream=None, gen="cuda"):
     """As build(), over an INT8 cache (PagedKVCacheInt8)."""
     from paged_kv_cache_486_b200.engine import PagedKVCacheInt8
     dt = workloads.TORCH_DTYPE[wl.dtype]
     eng = PagedKVCacheInt8(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda",
                            fill_bits=0x5A if poison else None)
-
-    def tokens(seq, pos0, n):
-        return wl.tokens(seq, pos0, n, 0, "cuda"), wl.tokens(seq, pos0, n, 1, "cuda")
-
-    eng.apply_ops(wl.ops, tokens, stream)
+    eng.apply_ops(wl.ops, _tokens_fn(wl, gen), stream)
     bt, ctx = eng.block_tables(wl.batch, wl.max_blocks)
-    q = wl.q("cuda")
+    q = wl.q(gen).to("cuda")
     out = eng.decode(q, bt, ctx, wl.scale, num_workers=workers, stream=stream)
     torch.cuda.synchronize()
     return dict(eng=eng, bt=bt, ctx=ctx, q=q, out=out)
