@@ -268,8 +268,13 @@ pa_status pa_swap_blocks(void* const* dst_k_host, void* const* dst_v_host,
  * workspace: device scratch of at least pa_decode_workspace_size(...) bytes,
  *   16-byte aligned, zero-filled once before its first use (e.g. cudaMemset);
  *   every call that completes leaves it zero-filled again, so it is reused
- *   without clearing.  After a call that reported PA_DEVERR_TIMEOUT, zero it
- *   again.  Calls that share a workspace must be ordered on one stream.
+ *   without clearing.  Its layout does not depend on the batch or head counts:
+ *   the first 256 + 4 * 262144 bytes hold counters (a 256-byte header, then one
+ *   4-byte arrival count per (sequence, kv head) pair, pair b * num_kv_heads +
+ *   kv_head), the rest partial results that are written before they are read.
+ *   So one workspace sized for the largest group and head_dim serves calls of
+ *   any batch.  After a call that reported PA_DEVERR_TIMEOUT, zero the counter
+ *   bytes again.  Calls that share a workspace must be ordered on one stream.
  * The work is split across the GPU by KV blocks: 7/8 of them evenly over the
  * workers, the rest in chunks claimed by whichever workers finish first.  A
  * sequence that fits in one worker's share is done in a single pass; a longer
@@ -302,6 +307,17 @@ pa_status pa_decode_attention(void* out, const void* q, const void* k_cache, con
  * pa_copy_blocks, which write only the caches. */
 #define PA_DECODE_OVERLAP_PROLOGUE 1
 
+/* PA_DECODE_TEST_WAIT_EXPIRY: for tests of the failure path only, never for
+ * results.  Every worker of the tensor-core kernels (pa_decode_attention_ex on
+ * the tensor-core path, pa_decode_attention_int8) treats its first wait for a
+ * tile as if its time limit had run out and stops; the warp that feeds it then
+ * waits for the tile slot to be released, and that wait really runs out, after
+ * about a second.  Each warp lets its copies in flight land before it exits.
+ * The call then reports PA_DEVERR_TIMEOUT, leaves output rows of non-empty
+ * contexts unwritten, and the workspace's counters must be zeroed again before
+ * the next call, as after any timeout.  PA_ERR_INVALID on the CUDA-core path. */
+#define PA_DECODE_TEST_WAIT_EXPIRY 0x100
+
 /* As pa_decode_attention, with the path, the number of workers (warps that
  * split the KV blocks; 0 = automatic, else clamped to the supported range) and
  * flags chosen by the caller.  Every path and worker count gives the same result
@@ -323,13 +339,17 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
  * declares in device memory; every GPU that loads the library holds it until
  * the process exits.  Arguments, results and errors are those of
  * pa_decode_attention, plus PA_ERR_INVALID if a shape would need more scratch
- * than the area holds.  Nothing is allocated by this call.
- * The first call on a device looks up the area's device address and zero-fills
- * the area, waiting for the device to finish (once per device, with that device
- * current); make that first call before any stream capture begins.  All calls share the one area, which keeps whatever the last
- * call left in it: calls whose work overlaps on the GPU (different streams,
- * or different host threads on one device) race on it and must be ordered by
- * the caller. */
+ * than the area holds: every shape whose group (num_q_heads / num_kv_heads) is
+ * at most 2048 fits, larger groups may not.  Every argument is checked before
+ * the device is touched.  Nothing is allocated by this call.
+ * The first call on a device looks up the area's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins.  Each call first clears, on `stream`, the counters it will
+ * use (256 + 4 * batch * num_kv_heads bytes at the start of the area), so a call
+ * that follows one that reported PA_DEVERR_TIMEOUT starts clean.  All calls
+ * share the one area, which keeps whatever the last call left in it: calls
+ * whose work overlaps on the GPU (different streams, or different host threads
+ * on one device) race on it and must be ordered by the caller. */
 pa_status pa_decode_attention_static_ws(void* out, const void* q, const void* k_cache,
                                         const void* v_cache, const int32_t* block_tables,
                                         const int32_t* context_lens, int32_t batch,

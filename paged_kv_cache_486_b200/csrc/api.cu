@@ -178,12 +178,55 @@ bool tc_applies(int group, int head_dim, int block_size, pa_dtype dt) {
          block_size % 16 == 0;
 }
 
-// Workspace: [256-byte header: chunk counter, finished-worker counter]
-//            [arrival counts: B * Hkv x 4 bytes][piece slots].
-size_t pieces_offset(int batch, int num_kv_heads) {
-  const size_t arrivals =
-      (sizeof(uint32_t) * static_cast<size_t>(batch) * num_kv_heads + 255) & ~size_t(255);
-  return 256 + arrivals;
+// Workspace layout, the same for every shape so that one zero-filled
+// workspace can serve calls of any batch and head count:
+//   [0, 256)                  chunk counter, finished-worker counter
+//   [256, kArrivalsEnd)       one arrival count per (sequence, kv head), for
+//                             up to kMaxArrivals pairs (pair b * Hkv + kvh)
+//   [kArrivalsEnd, ...)       piece slots (written before they are read)
+// Only the first two regions must start at zero, and a completed call leaves
+// every word it used there at zero.
+constexpr size_t kArrivalsOffset = 256;
+constexpr size_t kArrivalsEnd = kArrivalsOffset + sizeof(uint32_t) * pa::kMaxArrivals;
+
+size_t pieces_bytes(int group, int head_dim) {
+  return sizeof(float) * 2 * static_cast<size_t>(pa::max_ranges(max_workers(group))) * group *
+         (head_dim + 2);
+}
+
+// Host checks shared by the 16-bit decode entry points (nothing touches the
+// device here).
+pa_status check_decode_args(pa_dtype dtype, int32_t batch, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                            int32_t num_blocks, int32_t max_blocks, float scale) {
+  if (!valid_dtype(dtype))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: unknown dtype %d", static_cast<int>(dtype));
+  if (batch < 0 || batch > pa::kMaxBatch)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: batch %d outside [0, %d]", batch,
+                pa::kMaxBatch);
+  if (num_kv_heads < 1 || num_kv_heads > pa::kMaxKvHeads || num_q_heads < num_kv_heads ||
+      num_q_heads % num_kv_heads)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_q_heads %d not a multiple of "
+                "num_kv_heads %d (at most %d)", num_q_heads, num_kv_heads, pa::kMaxKvHeads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: head_dim %d not in {64, 128}", head_dim);
+  if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
+      block_size != 128)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: block_size %d not in {8,16,32,64,128}",
+                block_size);
+  if (num_blocks < 0 || max_blocks < 0)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: negative num_blocks or max_blocks");
+  const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
+  if (rows >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_blocks * num_kv_heads * block_size "
+                "= %lld >= 2^31", static_cast<long long>(rows));
+  if (static_cast<int64_t>(num_kv_heads) * max_blocks >= (int64_t(1) << 31))
+    return fail(PA_ERR_INVALID, "pa_decode_attention: num_kv_heads * max_blocks >= 2^31");
+  if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention: scale is NaN");
+  if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: batch * num_kv_heads = %lld > %d",
+                static_cast<long long>(batch) * num_kv_heads, pa::kMaxArrivals);
+  return PA_OK;
 }
 
 }  // namespace
@@ -302,10 +345,7 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t num_
   if (batch < 0 || num_kv_heads < 1 || num_q_heads < num_kv_heads ||
       num_q_heads % num_kv_heads || head_dim < 1)
     return 0;
-  const int group = num_q_heads / num_kv_heads;
-  return pieces_offset(batch, num_kv_heads) +
-         sizeof(float) * 2 * static_cast<size_t>(pa::max_ranges(max_workers(group))) * group *
-             (head_dim + 2);
+  return kArrivalsEnd + pieces_bytes(num_q_heads / num_kv_heads, head_dim);
 }
 
 pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
@@ -339,36 +379,13 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
                                  pa_dtype dtype, void* workspace, size_t workspace_bytes,
                                  int32_t* dev_error, int32_t path, int32_t num_workers,
                                  int32_t flags, pa_stream stream) {
-  if (!valid_dtype(dtype))
-    return fail(PA_ERR_INVALID, "pa_decode_attention: unknown dtype %d", static_cast<int>(dtype));
-  if (batch < 0 || batch > pa::kMaxBatch)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: batch %d outside [0, %d]", batch,
-                pa::kMaxBatch);
-  if (num_kv_heads < 1 || num_kv_heads > pa::kMaxKvHeads || num_q_heads < num_kv_heads ||
-      num_q_heads % num_kv_heads)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: num_q_heads %d not a multiple of "
-                "num_kv_heads %d (at most %d)", num_q_heads, num_kv_heads, pa::kMaxKvHeads);
-  if (head_dim != 64 && head_dim != 128)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: head_dim %d not in {64, 128}", head_dim);
-  if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
-      block_size != 128)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: block_size %d not in {8,16,32,64,128}",
-                block_size);
-  if (num_blocks < 0 || max_blocks < 0)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: negative num_blocks or max_blocks");
+  const pa_status chk = check_decode_args(dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                                          block_size, num_blocks, max_blocks, scale);
+  if (chk != PA_OK) return chk;
   const int64_t rows = static_cast<int64_t>(num_blocks) * num_kv_heads * block_size;
-  if (rows >= (int64_t(1) << 31))
-    return fail(PA_ERR_INVALID, "pa_decode_attention: num_blocks * num_kv_heads * block_size "
-                "= %lld >= 2^31", static_cast<long long>(rows));
-  if (static_cast<int64_t>(num_kv_heads) * max_blocks >= (int64_t(1) << 31))
-    return fail(PA_ERR_INVALID, "pa_decode_attention: num_kv_heads * max_blocks >= 2^31");
-  if (!(scale == scale)) return fail(PA_ERR_INVALID, "pa_decode_attention: scale is NaN");
-  if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
-    return fail(PA_ERR_INVALID, "pa_decode_attention: batch * num_kv_heads = %lld > %d",
-                static_cast<long long>(batch) * num_kv_heads, pa::kMaxArrivals);
   if (path != PA_PATH_AUTO && path != PA_PATH_TC && path != PA_PATH_SIMT)
     return fail(PA_ERR_INVALID, "pa_decode_attention: unknown path %d", path);
-  if (flags & ~PA_DECODE_OVERLAP_PROLOGUE)
+  if (flags & ~(PA_DECODE_OVERLAP_PROLOGUE | PA_DECODE_TEST_WAIT_EXPIRY))
     return fail(PA_ERR_INVALID, "pa_decode_attention: unknown flags 0x%x", flags);
   const bool overlap = (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0;
   if (batch == 0) return PA_OK;
@@ -388,6 +405,9 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_INVALID, "pa_decode_attention: tensor-core path needs fp16/bf16, "
                 "group <= 8 and block_size a multiple of 16");
   const bool use_tc = path == PA_PATH_TC || (path == PA_PATH_AUTO && tc_ok);
+  if ((flags & PA_DECODE_TEST_WAIT_EXPIRY) && !use_tc)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: PA_DECODE_TEST_WAIT_EXPIRY needs the "
+                "tensor-core path");
   int32_t planned_path = 0, workers = 0;
   pa_status st = pa_decode_plan(batch, num_q_heads, num_kv_heads, head_dim, block_size, dtype,
                                 &planned_path, &workers);
@@ -405,9 +425,8 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.context_lens = context_lens;
   a.dev_error = dev_error;
   a.ws_ctrl = static_cast<uint32_t*>(workspace);
-  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + 256);
-  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         pieces_offset(batch, num_kv_heads));
+  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + kArrivalsOffset);
+  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) + kArrivalsEnd);
   a.batch = batch;
   a.num_q_heads = num_q_heads;
   a.num_kv_heads = num_kv_heads;
@@ -418,6 +437,7 @@ pa_status pa_decode_attention_ex(void* out, const void* q, const void* k_cache,
   a.max_blocks = max_blocks;
   a.workers = workers;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.test_expire = (flags & PA_DECODE_TEST_WAIT_EXPIRY) ? 1 : 0;
 
   cudaError_t e;
   if (use_tc) {
@@ -521,7 +541,7 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
   if (static_cast<int64_t>(batch) * num_kv_heads > pa::kMaxArrivals)
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: batch * num_kv_heads > %d",
                 pa::kMaxArrivals);
-  if (flags & ~PA_DECODE_OVERLAP_PROLOGUE)
+  if (flags & ~(PA_DECODE_OVERLAP_PROLOGUE | PA_DECODE_TEST_WAIT_EXPIRY))
     return fail(PA_ERR_INVALID, "pa_decode_attention_int8: unknown flags 0x%x", flags);
   if (batch == 0) return PA_OK;
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !workspace)
@@ -547,9 +567,8 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
   a.context_lens = context_lens;
   a.dev_error = dev_error;
   a.ws_ctrl = static_cast<uint32_t*>(workspace);
-  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + 256);
-  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                         pieces_offset(batch, num_kv_heads));
+  a.ws_arrivals = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + kArrivalsOffset);
+  a.ws_pieces = reinterpret_cast<float*>(static_cast<char*>(workspace) + kArrivalsEnd);
   a.batch = batch;
   a.num_q_heads = num_q_heads;
   a.num_kv_heads = num_kv_heads;
@@ -560,6 +579,7 @@ pa_status pa_decode_attention_int8(void* out, const void* q, const void* k_pool,
   a.max_blocks = max_blocks;
   a.workers = workers;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.test_expire = (flags & PA_DECODE_TEST_WAIT_EXPIRY) ? 1 : 0;
   const int per = pa::decode_int8_workers_per_cta();
   const cudaError_t e = pa::launch_decode_int8(a, dtype, (workers + per - 1) / per,
                                                (flags & PA_DECODE_OVERLAP_PROLOGUE) != 0,
@@ -700,11 +720,13 @@ pa_status pa_check_device_error(int32_t* dev_error, int32_t* flags_out, pa_strea
 // scratch area of its own in device memory, declared below, and
 // pa_decode_attention_static_ws uses it instead of a caller buffer.
 //
-// The area is kStaticScratchBytes (28 MiB): enough for the largest workspace
-// any shape pa_decode_attention accepts can ask for (3073 ranges x 2 piece
-// slots x 8 heads x (128 + 2) floats, plus a 4-byte arrival count for each of
-// at most 262144 (sequence, kv head) pairs).  Every GPU that loads this
-// library holds those 28 MiB until the process exits.
+// The area is kStaticScratchBytes (28 MiB).  That covers the workspace of every
+// shape pa_decode_attention accepts whose group (num_q_heads / num_kv_heads)
+// is at most 2048 -- at most 3073 ranges x 2 piece slots x 8 heads x
+// (128 + 2) floats for groups up to 8, and no more than 27.7 MB of pieces for
+// any group up to 2048 -- plus the 1 MiB of arrival counts and the 256-byte
+// header.  Larger groups can need more and are rejected.  Every GPU that loads
+// this library holds those 28 MiB until the process exits.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr size_t kStaticScratchBytes = size_t(28) << 20;
@@ -719,10 +741,7 @@ void* g_scratch_addr[64] = {};
 
 // Device address of g_decode_scratch on the current device.  In host code the
 // symbol name is only a host-side handle, so the address is looked up once per
-// device (with that device current) and remembered.  The same one-time set-up
-// zero-fills the area (the decode keeps a few counters in its workspace that
-// must start at zero; every completed call leaves them at zero again) and waits
-// for that to finish.
+// device (with that device current) and remembered.
 pa_status static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -735,9 +754,6 @@ pa_status static_scratch(void** out) {
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess)
       return cuda_fail(e, "pa_decode_attention_static_ws (cudaGetSymbolAddress)");
-    e = cudaMemset(p, 0, kStaticScratchBytes);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention_static_ws (zero-fill)");
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -752,17 +768,31 @@ extern "C" pa_status pa_decode_attention_static_ws(
     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
     int32_t num_blocks, int32_t max_blocks, float scale, pa_dtype dtype, int32_t* dev_error,
     pa_stream stream) {
+  // Every argument is checked before the device is touched.
+  const pa_status chk = check_decode_args(dtype, batch, num_q_heads, num_kv_heads, head_dim,
+                                          block_size, num_blocks, max_blocks, scale);
+  if (chk != PA_OK) return chk;
   const size_t need = pa_decode_workspace_size(batch, num_q_heads, num_kv_heads, head_dim);
   if (need > kStaticScratchBytes)
     return fail(PA_ERR_INVALID,
                 "pa_decode_attention_static_ws: this shape needs %zu bytes of scratch, more "
                 "than the library's fixed %zu-byte area; use pa_decode_attention with a "
                 "caller-provided workspace", need, kStaticScratchBytes);
+  if (batch == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID, "pa_decode_attention: NULL pointer");
   void* scratch = nullptr;
   const pa_status st = static_scratch(&scratch);
   if (st != PA_OK) return st;
-  // The counters in the scratch were zeroed at set-up and every completed call
-  // returns them to zero; the split pieces are written before they are read.
+  // The counters this call uses (the header and one arrival word per
+  // (sequence, kv head)) are cleared on the call's stream first, so a call
+  // that an earlier one left unfinished (PA_DEVERR_TIMEOUT) starts clean; the
+  // piece slots are written before they are read.
+  const size_t counters = kArrivalsOffset + sizeof(uint32_t) * static_cast<size_t>(batch) *
+                                                num_kv_heads;
+  const cudaError_t e =
+      cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_attention_static_ws (clear counters)");
   return pa_decode_attention_ex(out, q, k_cache, v_cache, block_tables, context_lens, batch,
                                 num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                 max_blocks, scale, dtype, scratch, kStaticScratchBytes,

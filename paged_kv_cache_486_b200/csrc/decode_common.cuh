@@ -58,6 +58,8 @@ struct DecodeArgs {
   int32_t num_blocks, max_blocks;
   int32_t workers;        // workers launched (the split uses at most this many)
   float scale_log2;       // scale * log2(e)
+  int32_t test_expire;    // tests of the failure path: every worker's first tile wait
+                          // counts as run out (PA_DECODE_TEST_WAIT_EXPIRY)
 };
 
 // Ranges of the unit sequence (see the header comment).  Every range is non-empty.

@@ -432,7 +432,9 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
   for (int k = 0;; ++k) {
     const int slot = k % kStages;
     // all lanes take the same decision, so the warp never splits on a timeout
-    if (!__all_sync(kFull, mbar_wait_bounded(full0 + slot * 8, (k / kStages) & 1))) {
+    // (a test of the failure path makes the first wait count as run out)
+    if (!__all_sync(kFull, (k > 0 || !a.test_expire) &&
+                               mbar_wait_bounded(full0 + slot * 8, (k / kStages) & 1))) {
       if (lane == 0) report(a.dev_error, PA_DEVERR_TIMEOUT);
       // let stages the producer issued after this one land before exiting
       for (int i = 1; i < kStages; ++i)

@@ -64,6 +64,9 @@ def _call_decode(a):
     dict(path=pa.PA_PATH_TC, dtype=pa.PA_F32), dict(path=pa.PA_PATH_TC, Hq=32, Hkv=2),
     dict(path=pa.PA_PATH_TC, bs=8), dict(NB=1 << 24, Hkv=16, Hq=16), dict(scale=float("nan")),
     dict(flags=2), dict(B=4096, Hkv=128, Hq=128),
+    # the test-only wait-expiry flag exists on the tensor-core path only
+    dict(flags=pa.PA_DECODE_TEST_WAIT_EXPIRY, path=pa.PA_PATH_SIMT),
+    dict(flags=pa.PA_DECODE_TEST_WAIT_EXPIRY, dtype=pa.PA_F32),
 ])
 def test_decode_rejects_bad_arguments_on_host(bad):
     st = _call_decode(_decode_args(**bad))
