@@ -1,4 +1,7 @@
 """Runs a workload's op script through the oracle (test infrastructure)."""
+import concurrent.futures as cf
+import os
+
 import numpy as np
 import torch
 
@@ -55,6 +58,26 @@ def attention(wl, state, rows=None, n_threads=None):
     return oracle.paged_decode_attention(q, state["k_cache"], state["v_cache"], state["table"],
                                          state["ctx"], wl.scale, wl.dtype, rows=rows,
                                          n_threads=n_threads)
+
+
+def all_rows(wl, device="cuda", threads=None, visit=None):
+    """Oracle attention [B, Hq, D] of every batch row from the sequence's logical
+    key/value rows, which the seeded generator draws on `device` (the same bits on
+    any device; on the GPU it is plain torch arithmetic, not the library).
+    visit(b, k, v), if given, sees each row's logical keys and values first.
+    The oracle releases the GIL, so rows run in parallel on the host cores."""
+    q = raw(wl.q())
+
+    def row(b):
+        seq = int(wl.batch[b])
+        k = wl.contiguous_kv(seq, 0, device)
+        v = wl.contiguous_kv(seq, 1, device)
+        seen = visit(b, k, v) if visit else None
+        return seen, oracle.contiguous_attention(q[b], raw(k), raw(v), wl.scale, wl.dtype)
+
+    with cf.ThreadPoolExecutor(threads or os.cpu_count() or 4) as ex:
+        res = list(ex.map(row, range(wl.B)))
+    return np.stack([r[1] for r in res]), [r[0] for r in res]
 
 
 def contiguous_row(wl, b, heads=None):

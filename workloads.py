@@ -110,6 +110,13 @@ class Workload:
     batch: np.ndarray = None  # int64 seq ids in batch order
     lengths: dict = field(default_factory=dict)   # seq -> tokens after the script
     segments: dict = field(default_factory=dict)  # seq -> [(p0, p1, writer)] in order
+    # Wide-range option (powers of two only, so every value stays exact in every
+    # dtype): queries are multiplied by q_mul; the key row at position p by
+    # 2^min(p // k_ramp_tokens, k_ramp_max) when k_ramp_tokens > 0, so later keys
+    # reach larger scores and a running maximum keeps moving along the context.
+    q_mul: float = 1.0
+    k_ramp_tokens: int = 0
+    k_ramp_max: int = 0
 
     @property
     def G(self):
@@ -130,16 +137,26 @@ class Workload:
         return self.ops[self.n_prefill_ops:]
 
     # ---- values ----
+    def _ramp(self, t, p0, kind):
+        """Apply the key ramp to rows t [n, heads, D] at positions p0, p0 + 1, ..."""
+        if kind != KIND_K or self.k_ramp_tokens <= 0 or t.shape[0] == 0:
+            return t
+        p = torch.arange(p0, p0 + t.shape[0], dtype=torch.int64, device=t.device)
+        e = torch.clamp(p // self.k_ramp_tokens, max=self.k_ramp_max)
+        f = torch.pow(2.0, e.to(torch.float32)).to(t.dtype)
+        return t * f[:, None, None]
+
     def tokens(self, writer, p0, n, kind, device="cpu"):
         """[n, Hkv, D] key (kind 0) or value (kind 1) rows written by ``writer``."""
         per = self.Hkv * self.D
         t = _gen(stream_key(self.seed, kind, writer), p0 * per, n * per, device, self.dtype)
-        return t.view(n, self.Hkv, self.D)
+        return self._ramp(t.view(n, self.Hkv, self.D), p0, kind)
 
     def q(self, device="cpu"):
         n = self.B * self.Hq * self.D
-        return _gen(stream_key(self.seed, KIND_Q, 0), 0, n, device, self.dtype).view(
+        t = _gen(stream_key(self.seed, KIND_Q, 0), 0, n, device, self.dtype).view(
             self.B, self.Hq, self.D)
+        return t if self.q_mul == 1.0 else t * self.q_mul
 
     def contiguous_kv(self, seq, kind, device="cpu", heads=None):
         """Key/value rows of sequence ``seq`` in logical order: [ctx, Hkv or len(heads), D]."""
@@ -153,8 +170,8 @@ class Workload:
                 h = torch.as_tensor(heads, dtype=torch.int64, device=device)
                 d = torch.arange(self.D, dtype=torch.int64, device=device)
                 idx = (p[:, None, None] * self.Hkv + h[None, :, None]) * self.D + d[None, None, :]
-                parts.append(values(key, idx.reshape(-1)).to(TORCH_DTYPE[self.dtype]).view(
-                    p1 - p0, len(heads), self.D))
+                parts.append(self._ramp(values(key, idx.reshape(-1)).to(
+                    TORCH_DTYPE[self.dtype]).view(p1 - p0, len(heads), self.D), p0, kind))
         if not parts:
             return torch.empty(0, self.Hkv if heads is None else len(heads), self.D,
                                dtype=TORCH_DTYPE[self.dtype], device=device)
@@ -340,6 +357,14 @@ def custom(name="custom", dtype="f16", B=6, Hq=8, Hkv=2, D=128, bs=16, ctx=None,
                    shuffle=shuffle)
 
 
+def spread(wl, q_mul=2.0, ramp_tokens=256, ramp_max=3):
+    """The same workload with the wide-range option on (see Workload): scores span
+    tens of base-2 units and the largest ones come late in each context."""
+    wl.q_mul, wl.k_ramp_tokens, wl.k_ramp_max = float(q_mul), int(ramp_tokens), int(ramp_max)
+    wl.name += "_spread"
+    return wl
+
+
 # --------------------------------------------------------------- prefill
 def prefill(name, dtype, Hq, Hkv, D, bs, ctx, n_new, seed, slack=8) -> Workload:
     """Sequences of ctx[b] cached tokens whose last n_new[b] are the new chunk being
@@ -360,7 +385,8 @@ def query_start(wl) -> np.ndarray:
 def q_prefill(wl, device="cpu") -> torch.Tensor:
     T = int(wl.n_new.sum())
     n = T * wl.Hq * wl.D
-    return _gen(stream_key(wl.seed, KIND_Q, 1), 0, n, device, wl.dtype).view(T, wl.Hq, wl.D)
+    t = _gen(stream_key(wl.seed, KIND_Q, 1), 0, n, device, wl.dtype).view(T, wl.Hq, wl.D)
+    return t if wl.q_mul == 1.0 else t * wl.q_mul
 
 
 def prefill_8b(seed=4866):
