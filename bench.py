@@ -190,6 +190,18 @@ def _unique_kv_bytes(wl, table, ctx):
     return sum(rows.values()) * wl.Hkv * wl.D * 2 * wl.elem_bytes
 
 
+def workload_config(wl, world):
+    """The `config` object of the JSON line: the workload and how it is timed.  Both
+    arms print this same dict."""
+    return {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+            "head_dim": wl.D, "block_size": wl.bs, "layers_per_step": 1,
+            "context_tokens": int(wl.context_lens().sum()),
+            "kv_read_bytes_per_step": wl.kv_read_bytes(), "parallelism": f"replicas x{world}",
+            "timing": "GPU arm: CUDA-graph replay of the step, CUDA events per step; decode "
+                      "launched with PA_DECODE_OVERLAP_PROLOGUE after the cache write",
+            "l2": "GPU arm: flushed between timed steps (256 MiB read outside the events)"}
+
+
 # --------------------------------------------------------------- our arm
 def _setup(wl, extra_blocks=0):
     """Engine with the workload's pool (plus `extra_blocks` at the bottom of the free
@@ -292,18 +304,16 @@ def run_ours(args, dist, rank, world):
     del g_step, g_dec
 
     e2e = run_e2e(args, wl, eng, dist)
+    del eng, st, flush
+    torch.cuda.empty_cache()
+    bars = {} if args.no_bar_configs else {n: decode_only(n, args) for n in BAR_CONFIGS
+                                           if n != wl.name}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
         "data": "synthetic (seeded counter-based N(0,1) stand-in values, shuffled block pool)",
-        "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
-                   "head_dim": wl.D, "block_size": wl.bs, "layers_per_step": 1,
-                   "context_tokens": int(wl.context_lens().sum()),
-                   "kv_read_bytes_per_step": alg, "parallelism": f"replicas x{world}",
-                   "timing": "CUDA-graph replay of the step, CUDA events per step; decode "
-                             "launched with PA_DECODE_OVERLAP_PROLOGUE after the cache write",
-                   "l2": "flushed between timed steps (256 MiB read outside the events)"},
+        "config": workload_config(wl, world),
         "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3,
         "kv_unique_bytes": uniq, "kv_unique_read_gbs": uniq / (dec_ms / 1e3) / 1e9,
         "decode_us_min": min(decode_ms) * 1e3,
@@ -313,9 +323,56 @@ def run_ours(args, dist, rank, world):
                      "timed": "pa_decode_attention call (one kernel), graph replay"},
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
     }
+    if bars:
+        line["decode_bar"] = bars
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds, single_thread=True)
     return line
+
+
+# The decode configurations on which the >= 70% HBM bar is set (Llama-3-8B- and
+# Llama-3-70B-shaped layers); their decode-only roofline rides along the headline.
+BAR_CONFIGS = ("llama3_8b", "llama3_70b")
+
+
+def decode_only(name, args):
+    """pa_decode_attention alone on another workload: CUDA-graph replays with L2
+    flushed between them, CUDA events on the launching stream."""
+    wl = workloads.make(name)
+    eng, st = _setup(wl)
+    flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    eng.decode(st["q"], st["bt"], st["ctx"], wl.scale, out=st["out"])
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        eng.decode(st["q"], st["bt"], st["ctx"], wl.scale, out=st["out"])
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for it in range(args.warmup + args.steps):
+        _flush_l2(flush)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        e1.synchronize()
+        if it >= args.warmup:
+            ms.append(e0.elapsed_time(e1))
+    assert eng.device_errors() == 0, "device guards fired"
+    assert torch.isfinite(st["out"].float()).all()
+    del g
+    alg = wl.kv_read_bytes()
+    t = statistics.mean(ms) / 1e3
+    peak, kind = _peak_hbm()
+    res = {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
+           "dtype": wl.dtype, "kv_read_bytes": alg, "decode_us": t * 1e6,
+           "decode_us_min": min(ms) * 1e3, "tokens_per_s": wl.B / t,
+           "roofline": {"bound": "hbm", "achieved": alg / t / 1e9, "peak": peak, "unit": "GB/s",
+                        "frac": alg / t / 1e9 / peak, "peak_source": f"{kind} (hbm_gbs copy)",
+                        "traffic": _traffic(wl.name)},
+           "timed": "pa_decode_attention call alone (one kernel), graph replay"}
+    del eng, st, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_e2e(args, wl, eng, dist):
@@ -724,7 +781,10 @@ def run_prefill(args, dist, rank, world):
 
 
 # ---------------------------------------------------------- oracle timings
-def cpu_baseline(wl, target_s=10.0):
+def cpu_baseline(wl, target_s=10.0, single_thread=False, max_sample_bytes=2 << 30):
+    """The oracle on the host cores (all of them, and with single_thread one more pass
+    on one core), on the first S sequences of the workload laid out in a shuffled pool;
+    S is chosen for about target_s seconds of work and at most max_sample_bytes of K/V."""
     import oracle
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from oracle_side import raw
@@ -764,7 +824,9 @@ def cpu_baseline(wl, target_s=10.0):
     t0 = time.perf_counter()
     oracle.paged_decode_attention(q, kc, vc, table, ctx, wl.scale, wl.dtype, n_threads=threads)
     t_one = time.perf_counter() - t0
-    S = int(min(wl.B, max(1, target_s / max(t_one, 1e-3) / 4)))
+    per_seq = kc.nbytes + vc.nbytes
+    S = int(min(wl.B, max(1, target_s / max(t_one, 1e-3) / 4),
+                max(1, max_sample_bytes // max(per_seq, 1))))
     q, kc, vc, table, ctx = make(S)
     reps, elapsed = 0, 0.0
     while elapsed < target_s and reps < 50:
@@ -773,31 +835,70 @@ def cpu_baseline(wl, target_s=10.0):
                                       n_threads=threads)
         elapsed += time.perf_counter() - t0
         reps += 1
-    return {"value": S * reps / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {S} of {wl.B} sequences ({int(ctx.sum())} context tokens) of "
-                      f"{wl.name}, fp64 oracle, {reps} passes, {elapsed:.1f} s"}
+    res = {"value": S * reps / elapsed, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"first {S} of {wl.B} sequences ({int(ctx.sum())} context tokens) of "
+                     f"{wl.name}, fp64 oracle, {reps} passes, {elapsed:.1f} s",
+           "nproc": _nproc(), "hardware_concurrency": oracle.hardware_concurrency(),
+           "os_cpu_count": os.cpu_count()}
+    if single_thread:
+        # one sequence on one core, for about a third of the all-core budget
+        q1, kc1, vc1, table1, ctx1 = q[:1], kc, vc, table[:1], ctx[:1]
+        reps1, el1 = 0, 0.0
+        while el1 < target_s / 3 and reps1 < 50:
+            t0 = time.perf_counter()
+            oracle.paged_decode_attention(q1, kc1, vc1, table1, ctx1, wl.scale, wl.dtype,
+                                          n_threads=1)
+            el1 += time.perf_counter() - t0
+            reps1 += 1
+        res["single_thread"] = {"value": reps1 / el1, "unit": "tokens/s", "cores": 1,
+                                "sample": f"sequence 0 of {wl.name} ({int(ctx1[0])} context "
+                                          f"tokens), {reps1} passes, {el1:.1f} s"}
+    return res
+
+
+def _nproc():
+    try:
+        return int(subprocess.run(["nproc"], capture_output=True, text=True,
+                                  timeout=10).stdout.strip())
+    except (OSError, ValueError, subprocess.SubprocessError):
+        return None
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
     wl = workloads.make(args.config)
-    per_step = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    per_step = min(args.cpu_seconds, max(2.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(wl, target_s=min(per_step, 2.0))
-    vals = [cpu_baseline(wl, target_s=per_step) for _ in range(args.steps)]
+    vals = [cpu_baseline(wl, target_s=per_step, single_thread=(i == args.steps - 1))
+            for i in range(args.steps)]
     v = statistics.mean(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = v
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * wl.B / v, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq,
-                       "kv_heads": wl.Hkv, "head_dim": wl.D, "block_size": wl.bs},
+            "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-based N(0,1) stand-in values, shuffled block pool)",
+            "config": workload_config(wl, world),
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+def _relaunch(n):
+    """--gpus N without a launcher: run this same command as N ranks under
+    torch.distributed.run on this node (one rank per GPU)."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    sys.stdout.flush()
+    os.execv(sys.executable, cmd)
 
 
 def main():
@@ -805,7 +906,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="llama3_8b", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--config", default="long_mha", choices=sorted(workloads.CONFIGS),
+                    help="workload of the step (default long_mha: 8 x 32768 tokens, 64/64 "
+                         "heads, the largest single-GPU configuration)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="step",
                     choices=["step", "swap", "int8", "prefix", "prefill"],
@@ -816,10 +919,19 @@ def main():
                     help="--op prefill kernel: 0 automatic (tcgen05 at head_dim 128), "
                          "1 tcgen05, 2 mma.sync")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bar-configs", action="store_true",
+                    help="skip the decode-only lines of llama3_8b and llama3_70b")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        _relaunch(args.gpus)  # does not return
+    if env_world is not None and int(env_world) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={env_world}: launch one rank per GPU")
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -829,6 +941,8 @@ def main():
             print(json.dumps(line), flush=True)
         return
 
+    if not torch.cuda.is_available():
+        sys.exit("bench.py: the GPU arm needs a CUDA device (B200); none is visible")
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dist, rank, world = _dist()

@@ -97,8 +97,15 @@ def lib():
         L.orc_contiguous_attention.restype = C.c_int
         L.orc_contiguous_attention.argtypes = [P, P, P, C.c_int64, C.c_int32, C.c_int32,
                                                C.c_int32, C.c_double, C.c_int, P, P, C.c_int32]
+        L.orc_hardware_concurrency.restype = C.c_int32
+        L.orc_hardware_concurrency.argtypes = []
         _lib = L
     return _lib
+
+
+def hardware_concurrency():
+    """std::thread::hardware_concurrency() of the oracle's C++ runtime."""
+    return int(lib().orc_hardware_concurrency())
 
 
 def _ptr(a):

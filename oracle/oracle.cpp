@@ -854,4 +854,10 @@ int orc_contiguous_attention(const void* q, const void* k, const void* v, int64_
   return ORC_OK;
 }
 
+// Host threads the C++ runtime reports (std::thread::hardware_concurrency; 0 if
+// unknown): the core count printed beside the oracle's timings.
+int32_t orc_hardware_concurrency(void) {
+  return static_cast<int32_t>(std::thread::hardware_concurrency());
+}
+
 }  // extern "C"

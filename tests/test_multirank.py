@@ -50,3 +50,39 @@ def test_two_rank_aggregation_on_gloo():
         assert tokens == 1280.0                       # every replica's tokens count
         assert value == pytest.approx(1280.0 / 0.150)
     assert results[1][1] is None                      # only rank 0 runs the reference arm
+
+
+def _bench(*argv, env=None, timeout=300):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    e = dict(os.environ)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        e.pop(k, None)
+    e.update(env or {})
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py"), *argv],
+                          capture_output=True, text=True, timeout=timeout, env=e)
+
+
+def test_gpus_n_launches_n_ranks_and_rank_0_alone_prints():
+    """`bench.py --gpus 2` without a launcher relaunches itself as two ranks under
+    torch.distributed.run; on the reference arm rank 0 alone runs and prints."""
+    import json
+    r = _bench("--impl", "reference", "--gpus", "2", "--config", "tiny", "--steps", "1",
+               "--warmup", "3", "--cpu-seconds", "0.3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+    assert lines[0]["config"]["workload"] == "tiny"
+
+
+def test_gpu_arm_without_a_gpu_or_with_a_mismatched_world_fails_loudly():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("checks the CPU-only failure")
+    r = _bench("--gpus", "1", "--config", "tiny", "--steps", "1", "--warmup", "3")
+    assert r.returncode != 0 and "CUDA device" in r.stderr
+    r = _bench("--gpus", "4", "--config", "tiny", "--steps", "1", "--warmup", "3",
+               env={"WORLD_SIZE": "2"})
+    assert r.returncode != 0 and "WORLD_SIZE=2" in r.stderr
