@@ -335,10 +335,10 @@ def run_ours(args, dist, rank, world):
 BAR_CONFIGS = ("llama3_8b", "llama3_70b")
 
 
-def decode_only(name, args):
-    """pa_decode_attention alone on another workload: CUDA-graph replays with L2
-    flushed between them, CUDA events on the launching stream."""
-    wl = workloads.make(name)
+def decode_only(name, args, batch=0):
+    """pa_decode_attention alone on a workload: CUDA-graph replays with L2 flushed
+    between them, CUDA events on the launching stream."""
+    wl = workloads.make(name, batch)
     eng, st = _setup(wl)
     flush = torch.ones(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     eng.decode(st["q"], st["bt"], st["ctx"], wl.scale, out=st["out"])
@@ -510,7 +510,7 @@ def run_int8(args, dist, rank, world):
     the step's tokens, then decode attention over codes + per-token scales."""
     import paged_kv_cache_486_b200 as pa
     from paged_kv_cache_486_b200.engine import PagedKVCacheInt8
-    wl = workloads.make(args.config)
+    wl = workloads.make(args.config, args.batch)
     dt = workloads.TORCH_DTYPE[wl.dtype]
     eng = PagedKVCacheInt8(wl.num_blocks, wl.bs, wl.Hkv, wl.D, dt, wl.Hq, wl.B, "cuda")
 
@@ -614,6 +614,20 @@ def run_int8(args, dist, rank, world):
                      "timed": "pa_decode_attention_int8 call (one kernel), graph replay"},
         "gpu_launches": launches * args.steps, "clocks": clocks,
     }
+
+
+def run_decode(args, dist, rank, world):
+    """--op decode: the decode call alone on --config (and --batch), one JSON line
+    (the form the profiles' ncu captures run)."""
+    r = decode_only(args.config, args, args.batch)
+    return {"metric": METRIC + " (decode call alone)", "op": "decode",
+            "value": r["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": r["dtype"], "data": "synthetic",
+            "config": {"workload": r["workload"], "batch": r["batch"],
+                       "l2": "flushed between timed calls (256 MiB read outside the events)"},
+            "decode_us": r["decode_us"], "roofline": r["roofline"],
+            "gpu_launches": args.steps}
 
 
 def run_prefix(args, dist, rank, world):
@@ -911,10 +925,14 @@ def main():
                          "heads, the largest single-GPU configuration)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--op", default="step",
-                    choices=["step", "swap", "int8", "prefix", "prefill"],
-                    help="step: the decode step (default); swap: eviction to host and back; "
-                         "int8: the decode step over an INT8 cache; prefix: prefix caching; "
-                         "prefill: paged prefill attention (--config prefill_8b | chunked_8b)")
+                    choices=["step", "decode", "swap", "int8", "prefix", "prefill"],
+                    help="step: the decode step (default); decode: the decode call alone; "
+                         "swap: eviction to host and back; int8: the decode step over an INT8 "
+                         "cache; prefix: prefix caching; prefill: paged prefill attention "
+                         "(--config prefill_8b | chunked_8b)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="--op decode / int8: override the batch of llama3_8b, llama3_70b or "
+                         "long_mha (a reduced case for profiling)")
     ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2],
                     help="--op prefill kernel: 0 automatic (tcgen05 at head_dim 128), "
                          "1 tcgen05, 2 mma.sync")
@@ -948,7 +966,7 @@ def main():
     dist, rank, world = _dist()
     try:
         run = {"swap": run_swap, "int8": run_int8, "prefix": run_prefix,
-               "prefill": run_prefill}.get(args.op, run_ours)
+               "prefill": run_prefill, "decode": run_decode}.get(args.op, run_ours)
         line = run(args, dist, rank, world)
         if rank == 0:
             print(json.dumps(line), flush=True)

@@ -13,8 +13,15 @@
 // same order.  In O^T += V^T . P^T a lane's four value bytes are tokens
 // 4cq .. 4cq+3, which is exactly the token order that the register transpose
 // of S^T rows tau(.) gives the P^T fragment, so neither operand is shuffled.
-// Codes become 16-bit values exactly (|code| <= 127) by integer bit tricks,
-// then every product is the same mma as in the 16-bit path.
+// Every product is an fp16 mma whatever the query dtype: the codes are exact in
+// fp16, and bf16 queries (8-bit significand) become fp16 exactly after a
+// power-of-two prescale per head that puts the head's largest |q| in
+// [2^13, 2^14); the prescale is divided out of the scores.
+//  * Keys enter as 1024 + u (u = code + 128, the stored byte), exact in fp16
+//    and two byte permutes per four codes; the product then carries
+//    1152 * sum_d q_d too, which is subtracted once per segment (the
+//    accumulator starts at -1152 * sum_d q_d).
+//  * Values enter as the signed codes (exact), so O needs no correction.
 // Scales.  Key scales multiply the score rows (with scale * log2 e).  Value
 // scales are folded into P: p'_j = p_j * vs_j / sigma with sigma a lazily
 // updated running maximum of the segment's value scales (p' stays within a
@@ -32,29 +39,19 @@ namespace pa {
 namespace tc {
 
 // Four codes (bytes of w, stored offset-binary: u = c + 128) as two pairs of
-// 16-bit values: .x = bytes 0, 1, .y = bytes 2, 3.  fp16: 0x64 in the high byte
-// makes 1024 + u, and 1152 is subtracted.  bf16 (7-bit significand) goes
-// through fp32 the same way: 0x4B0000uu is 2^23 + u, minus 2^23 + 128.
-template <typename T>
-__device__ __forceinline__ uint2 codes_to(uint32_t w);
-
-template <>
-__device__ __forceinline__ uint2 codes_to<__half>(uint32_t w) {
-  uint32_t lo = __byte_perm(w, 0x64646464u, 0x5140);
-  uint32_t hi = __byte_perm(w, 0x64646464u, 0x7362);
-  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));
-  const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
-  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
-  return make_uint2(*reinterpret_cast<const uint32_t*>(&l), *reinterpret_cast<const uint32_t*>(&h));
+// fp16 values, .x = bytes 0, 1, .y = bytes 2, 3.  0x64 in the high byte makes
+// the fp16 value 1024 + u exactly.
+__device__ __forceinline__ uint2 codes_biased(uint32_t w) {
+  return make_uint2(__byte_perm(w, 0x64646464u, 0x5140), __byte_perm(w, 0x64646464u, 0x7362));
 }
 
-template <>
-__device__ __forceinline__ uint2 codes_to<__nv_bfloat16>(uint32_t w) {
-  float f[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    f[i] = __uint_as_float(__byte_perm(w, 0x4Bu, 0x4650 + i)) - 8388736.0f;
-  return make_uint2(pack2<__nv_bfloat16>(f[0], f[1]), pack2<__nv_bfloat16>(f[2], f[3]));
+// The same four codes as signed fp16 values u - 128 (1024 + u minus 1152, exact).
+__device__ __forceinline__ uint2 codes_signed(uint32_t w) {
+  const uint2 b = codes_biased(w);
+  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));
+  const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&b.x), bias);
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&b.y), bias);
+  return make_uint2(*reinterpret_cast<const uint32_t*>(&l), *reinterpret_cast<const uint32_t*>(&h));
 }
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
@@ -91,7 +88,9 @@ struct Tiles8 {
     float ks0, ks1, vs0, vs1;  // scales of the lane's tokens row_token(g), +2
   };
   struct Seg {
-    float sig, inv;
+    float sig, inv;  // value-scale normaliser sigma and 1 / sigma
+    float c0, c1;    // scale * log2 e / prescale, heads 2cq and 2cq + 1
+    float qs0, qs1;  // -1152 * sum_d q'_d, heads 2cq and 2cq + 1
     __device__ void reset() { sig = inv = 0.f; }
     __device__ float out_scale() const { return sig; }
   };
@@ -109,6 +108,56 @@ struct Tiles8 {
   }
   // lane (g, cq) holds q[g][16kc + 4cq, +1] and q[g][16kc + 4cq + 2, +3]
   __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 4 * cq + 2 * half; }
+
+  // The segment's query fragments (pairs of T) become fp16 pairs q' = q * f, f a
+  // power of two per head (1 for fp16 queries); seg gets each of the lane's two
+  // heads' score factor (scale * log2 e / f) and key-offset term.
+  __device__ static void prep_q(uint32_t (&qf)[KC][2], Seg& seg, const DecodeArgs& a, int lane) {
+    float finv = 1.f;
+    if (!std::is_same<T, __half>::value) {
+      float amax = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 x = unpack2<T>(qf[kc][h]);
+          amax = fmaxf(amax, fmaxf(fabsf(x.x), fabsf(x.y)));
+        }
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      // amax < 2^e; f = 2^(14 - e) puts it in [2^13, 2^14) (capped for tiny heads)
+      const int e = ((__float_as_int(amax) >> 23) & 0xff) - 126;
+      const int fe = min(14 - e, 126);
+      const float f = amax > 0.f ? __int_as_float((127 + fe) << 23) : 1.f;
+      finv = amax > 0.f ? __int_as_float((127 - fe) << 23) : 1.f;
+#pragma unroll
+      for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 x = unpack2<T>(qf[kc][h]);
+          qf[kc][h] = pack2<__half>(x.x * f, x.y * f);
+        }
+      }
+    }
+    float sum = 0.f;
+#pragma unroll
+    for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float2 x = unpack2<__half>(qf[kc][h]);
+        sum += x.x + x.y;
+      }
+    }
+    sum += __shfl_xor_sync(kFull, sum, 1);
+    sum += __shfl_xor_sync(kFull, sum, 2);
+    // heads 2cq and 2cq + 1 are held by lanes 8cq and 8cq + 4
+    const int cq = lane & 3;
+    seg.qs0 = -1152.f * __shfl_sync(kFull, sum, 8 * cq);
+    seg.qs1 = -1152.f * __shfl_sync(kFull, sum, 8 * cq + 4);
+    seg.c0 = a.scale_log2 * __shfl_sync(kFull, finv, 8 * cq);
+    seg.c1 = a.scale_log2 * __shfl_sync(kFull, finv, 8 * cq + 4);
+  }
 
   __device__ static void load(const DecodeArgs&, uint32_t ring0, int warp, int slot, int,
                               int lane, Frag& f) {
@@ -136,22 +185,23 @@ struct Tiles8 {
     f.vs1 = lds_f32(vt + i8::kCodeBytes + 4 * (tk + 2));
   }
 
-  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const DecodeArgs& a,
-                                int n_valid, int lane, float (&t)[4]) {
-    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const Seg& seg,
+                                const DecodeArgs&, int n_valid, int lane, float (&t)[4]) {
+    // accumulator element i is (row g or g + 8, head 2cq or 2cq + 1): start from
+    // the head's key-offset term; two accumulators halve the dependent chain
+    float s[4] = {seg.qs0, seg.qs1, seg.qs0, seg.qs1}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kc = 0; kc < KC; ++kc) {
-      const uint2 r0 = codes_to<T>(f.k[kc][0]);
-      const uint2 r1 = codes_to<T>(f.k[kc][1]);
+      const uint2 r0 = codes_biased(f.k[kc][0]);
+      const uint2 r1 = codes_biased(f.k[kc][1]);
       const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
-      if (kc & 1) mma16816<T>(s2, A, qf[kc]); else mma16816<T>(s, A, qf[kc]);
+      if (kc & 1) mma16816<__half>(s2, A, qf[kc]); else mma16816<__half>(s, A, qf[kc]);
     }
     const int tk = row_token(lane >> 2);
-    const float k0 = f.ks0 * a.scale_log2, k1 = f.ks1 * a.scale_log2;
-    t[0] = (s[0] + s2[0]) * k0;
-    t[1] = (s[1] + s2[1]) * k0;
-    t[2] = (s[2] + s2[2]) * k1;
-    t[3] = (s[3] + s2[3]) * k1;
+    t[0] = (s[0] + s2[0]) * (f.ks0 * seg.c0);
+    t[1] = (s[1] + s2[1]) * (f.ks0 * seg.c1);
+    t[2] = (s[2] + s2[2]) * (f.ks1 * seg.c0);
+    t[3] = (s[3] + s2[3]) * (f.ks1 * seg.c1);
     if (tk >= n_valid) t[0] = t[1] = -INFINITY;
     if (tk + 2 >= n_valid) t[2] = t[3] = -INFINITY;
   }
@@ -178,30 +228,15 @@ struct Tiles8 {
       seg.inv = 1.f / mx;
     }
     const float u0 = w0 * seg.inv, u1 = w1 * seg.inv;
-    // fp16 weights (11-bit significand, p' <= 2^12) in one product; bf16 as a
-    // head + tail pair, whose 8-bit significand alone would cost ~2^-9 |v|
-    constexpr bool kSplit = !std::is_same<T, __half>::value;
-    uint32_t h01, t01 = 0, h23, t23 = 0;
-    if (kSplit) {
-      split2<T>(p[0] * u0, p[1] * u0, h01, t01);
-      split2<T>(p[2] * u1, p[3] * u1, h23, t23);
-    } else {
-      h01 = pack2<T>(p[0] * u0, p[1] * u0);
-      h23 = pack2<T>(p[2] * u1, p[3] * u1);
-    }
-    const uint32_t pb[2] = {transpose8x8(h01), transpose8x8(h23)};
-    uint32_t pt[2] = {0u, 0u};
-    if (kSplit) {
-      pt[0] = transpose8x8(t01);
-      pt[1] = transpose8x8(t23);
-    }
+    // fp16 weights (11-bit significand, p' <= 2^12) in one product
+    const uint32_t pb[2] = {transpose8x8(pack2<__half>(p[0] * u0, p[1] * u0)),
+                            transpose8x8(pack2<__half>(p[2] * u1, p[3] * u1))};
 #pragma unroll
     for (int mt = 0; mt < KC; ++mt) {
-      const uint2 r0 = codes_to<T>(f.v[mt][0]);
-      const uint2 r1 = codes_to<T>(f.v[mt][1]);
+      const uint2 r0 = codes_signed(f.v[mt][0]);
+      const uint2 r1 = codes_signed(f.v[mt][1]);
       const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
-      mma16816<T>(o[mt], A, pb);
-      if (kSplit) mma16816<T>(o[mt], A, pt);
+      mma16816<__half>(o[mt], A, pb);
     }
   }
 };

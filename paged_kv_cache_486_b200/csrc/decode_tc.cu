@@ -52,6 +52,7 @@ struct Tiles16 {
   }
   // lane (g, cq) holds q[g][16kc + 2cq, +1] and q[g][16kc + 8 + 2cq, +1]
   __device__ static int q_off(int kc, int cq, int half) { return kc * 16 + 8 * half + 2 * cq; }
+  __device__ static void prep_q(uint32_t (&)[KC][2], Seg&, const DecodeArgs&, int) {}
 
   __device__ static void load(const DecodeArgs&, uint32_t ring0, int warp, int slot,
                               int n_valid, int lane, Frag& f) {
@@ -77,8 +78,8 @@ struct Tiles16 {
     }
   }
 
-  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const DecodeArgs& a,
-                                int n_valid, int lane, float (&t)[4]) {
+  __device__ static void scores(const Frag& f, const uint32_t (&qf)[KC][2], const Seg&,
+                                const DecodeArgs& a, int n_valid, int lane, float (&t)[4]) {
     // two accumulators halve the dependent chain
     float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

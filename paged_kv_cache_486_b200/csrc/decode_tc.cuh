@@ -31,8 +31,10 @@
 //   parameter), Frag (one stage in registers), Seg (per-segment state);
 //   prefetch(maps); issue(maps, a, ring0, warp, slot, tile, tok, bar) (lane 0);
 //   q_off(kc, cq, half) (head_dim offset of a query fragment register);
+//   prep_q(qf, seg, a, lane) (once per segment, after seg.reset(), on the
+//     segment's query fragments: whatever the policy's products need);
 //   load(a, ring0, warp, slot, n_valid, lane, frag);
-//   scores(frag, qf, a, n_valid, lane, t[4]);  pv(frag, p[4], o, seg, n_valid, lane).
+//   scores(frag, qf, seg, a, n_valid, lane, t[4]);  pv(frag, p[4], o, seg, n_valid, lane).
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -463,6 +465,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
       seg.reset();
+      P::prep_q(qf, seg, a, lane);
       // start fetching the next pair's queries now; they are used only then
       qn_b = -1;
       if (flags & kMoreInRange) {
@@ -492,7 +495,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
       // scores of (row g, head 2cq), (g, 2cq+1), (g+8, 2cq), (g+8, 2cq+1), base-2
       // units, -inf past the context
       float t[4];
-      P::scores(fr, qf, a, n_valid, lane, t);
+      P::scores(fr, qf, seg, a, n_valid, lane, t);
       // Lazy running maximum: weights are taken against the current reference m
       // unless some score of the stage is more than kSlack above it (then the
       // stage's maximum is reduced across the warp and the sums are rescaled).

@@ -490,5 +490,17 @@ CONFIGS = {
 }
 
 
-def make(name: str) -> Workload:
+def make(name: str, batch: int = 0) -> Workload:
+    """The named workload; batch > 0 overrides the batch of the configurations
+    that take one (llama3_8b, llama3_70b, long_mha, long_mha_bs32)."""
+    if batch > 0:
+        sized = {"llama3_8b": lambda: llama3_8b(B=batch),
+                 "llama3_70b": lambda: llama3_70b(B=batch),
+                 "long_mha": lambda: long_mha(B=batch),
+                 "long_mha_bs32": lambda: long_mha(bs=32, B=batch)}
+        if name not in sized:
+            raise ValueError(f"{name} has a fixed batch")
+        wl = sized[name]()
+        wl.name = f"{wl.name}_b{batch}"
+        return wl
     return CONFIGS[name]()
