@@ -66,7 +66,11 @@ def _peak_tensor():
 
 
 DECODE_SOURCES = ("decode_tc.cuh", "decode_tc.cu", "decode_common.cuh", "decode_simt.cu")
-PREFILL_SOURCES = ("prefill_tc5.cu", "prefill_launch.h", "decode_tc.cuh", "decode_common.cuh")
+# the tcgen05 prefill kernels: on pairs of SMs, and on one SM per item (the automatic choice)
+PREFILL_SOURCES = ("prefill_pair.cu", "tc5_ptx.cuh", "prefill_launch.h", "decode_tc.cuh",
+                   "decode_common.cuh")
+PREFILL_1SM_SOURCES = ("prefill_tc5.cu", "tc5_ptx.cuh", "prefill_launch.h", "decode_tc.cuh",
+                       "decode_common.cuh")
 INT8_SOURCES = ("decode_tc.cuh", "decode_int8.cu", "decode_common.cuh", "int8_launch.h")
 
 
@@ -785,11 +789,15 @@ def run_prefill(args, dist, rank, world):
         "prefill_us": 1e3 * statistics.mean(ms), "kv_read_bytes": kv_bytes,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "peak_source": kind,
-                     "traffic": (_traffic(wl.name, PREFILL_SOURCES)
-                                 if args.prefill_path != 2 and wl.D == 128 else None),
+                     "traffic": (None if args.prefill_path == 2 or wl.D != 128
+                                 else _traffic(wl.name + "_tc5_pair", PREFILL_SOURCES)
+                                 if args.prefill_path == 3
+                                 else _traffic(wl.name, PREFILL_1SM_SOURCES)),
                      "timed": "pa_prefill_attention (one kernel, " +
                               ("mma.sync m16n8k16" if args.prefill_path == 2 or wl.D != 128
-                               else "tcgen05 UMMA, TMEM accumulators") + ")"},
+                               else "tcgen05 UMMA on pairs of SMs (cta_group::2), TMEM "
+                                    "accumulators" if args.prefill_path == 3
+                               else "tcgen05 UMMA on one SM per item, TMEM accumulators") + ")"},
         "gpu_launches": args.steps,
     }
 
@@ -933,9 +941,10 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="--op decode / int8: override the batch of llama3_8b, llama3_70b or "
                          "long_mha (a reduced case for profiling)")
-    ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2],
-                    help="--op prefill kernel: 0 automatic (tcgen05 at head_dim 128), "
-                         "1 tcgen05, 2 mma.sync")
+    ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="--op prefill kernel: 0 automatic (tcgen05 on one SM per item at "
+                         "head_dim 128), 1 tcgen05 on one SM per item, 2 mma.sync, "
+                         "3 tcgen05 on pairs of SMs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bar-configs", action="store_true",
                     help="skip the decode-only lines of llama3_8b and llama3_70b")

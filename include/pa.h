@@ -386,7 +386,8 @@ pa_status pa_decode_plan(int32_t batch, int32_t num_q_heads, int32_t num_kv_head
  * UMMA with TMEM accumulators; items of 128 (token, head) rows of one kv head,
  * K / V tiles of 128 keys; here one item per CTA, persistent through
  * pa_prefill_attention_ex with a workspace); otherwise mma.sync (64 rows per
- * CTA, 64-key tiles).
+ * CTA, 64-key tiles).  pa_prefill_attention_ex also offers the same shapes on
+ * pairs of SMs (PA_PREFILL_TCGEN05_PAIR).
  * Alignment: k_cache, v_cache 16 bytes; q, out 4 (16 for the tcgen05
  * kernel, which the automatic choice then skips).  max_q * (num_q_heads /
  * num_kv_heads) < 2^31 - 256.  Errors: PA_ERR_INVALID for
@@ -401,10 +402,14 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
                                pa_dtype dtype, int32_t* dev_error, pa_stream stream);
 
 /* Kernels for pa_prefill_attention_ex. */
-#define PA_PREFILL_AUTO 0      /* tcgen05 where it applies, else mma.sync */
-#define PA_PREFILL_TCGEN05 1   /* head_dim 128, group dividing 128, scale > 0, q and out
-                                  16-byte aligned */
+#define PA_PREFILL_AUTO 0      /* the one-SM tcgen05 kernel where it applies, else mma.sync */
+#define PA_PREFILL_TCGEN05 1   /* one SM per item: head_dim 128, group dividing 128,
+                                  scale > 0, q and out 16-byte aligned */
 #define PA_PREFILL_MMA_SYNC 2  /* every supported shape */
+#define PA_PREFILL_TCGEN05_PAIR 3  /* the shapes of PA_PREFILL_TCGEN05, on pairs of SMs
+                                      (clusters of two CTAs, tcgen05 cta_group::2): an item is
+                                      256 rows, each SM keeps 128 of them and loads half of
+                                      every key and value tile */
 
 /* Bytes of the optional scheduling workspace of pa_prefill_attention_ex. */
 #define PA_PREFILL_WORKSPACE_BYTES 16

@@ -22,7 +22,7 @@ PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 PA_PATH_AUTO, PA_PATH_TC, PA_PATH_SIMT = 0, 1, 2
 PA_DECODE_OVERLAP_PROLOGUE = 1
 PA_DECODE_TEST_WAIT_EXPIRY = 0x100  # tests of the failure path only (see include/pa.h)
-PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA_SYNC = 0, 1, 2
+PA_PREFILL_AUTO, PA_PREFILL_TCGEN05, PA_PREFILL_MMA_SYNC, PA_PREFILL_TCGEN05_PAIR = 0, 1, 2, 3
 PA_PREFILL_WORKSPACE_BYTES = 16
 PA_DEVERR_BAD_SLOT, PA_DEVERR_BAD_BLOCK, PA_DEVERR_BAD_CTX, PA_DEVERR_TIMEOUT = 1, 2, 4, 8
 

@@ -595,7 +595,8 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
                                   int32_t max_blocks, int32_t total_q, int32_t max_q, float scale,
                                   pa_dtype dtype, int32_t* dev_error, void* workspace,
                                   int32_t path, pa_stream stream) {
-  if (path != PA_PREFILL_AUTO && path != PA_PREFILL_TCGEN05 && path != PA_PREFILL_MMA_SYNC)
+  if (path != PA_PREFILL_AUTO && path != PA_PREFILL_TCGEN05 && path != PA_PREFILL_MMA_SYNC &&
+      path != PA_PREFILL_TCGEN05_PAIR)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: unknown path %d", path);
   if (dtype != PA_F16 && dtype != PA_BF16)
     return fail(PA_ERR_INVALID, "pa_prefill_attention: dtype must be fp16 or bf16");
@@ -630,13 +631,20 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_INVALID, "pa_prefill_attention: misaligned pointer");
   const bool tc5_ok = head_dim == 128 && 128 % group == 0 && aligned(q, 16) &&
                       aligned(out, 16) && scale > 0.f;
-  if (path == PA_PREFILL_TCGEN05 && !tc5_ok)
-    return fail(PA_ERR_INVALID, "pa_prefill_attention: the tcgen05 kernel needs head_dim 128, "
+  if ((path == PA_PREFILL_TCGEN05 || path == PA_PREFILL_TCGEN05_PAIR) && !tc5_ok)
+    return fail(PA_ERR_INVALID, "pa_prefill_attention: the tcgen05 kernels need head_dim 128, "
                 "num_q_heads / num_kv_heads dividing 128, scale > 0 and q, out 16-byte aligned");
+  const bool use_pair = path == PA_PREFILL_TCGEN05_PAIR;
   const bool use_tc5 = path == PA_PREFILL_TCGEN05 || (path == PA_PREFILL_AUTO && tc5_ok);
   CUtensorMap qmap, omap, kmap, vmap;
   bool k3 = false, v3 = false;
-  if (use_tc5) {
+  if (use_pair) {
+    if (!make_q_map(&qmap, q, total_q, num_q_heads, head_dim, group, dtype) ||
+        !make_q_map(&omap, out, total_q, num_q_heads, head_dim, group, dtype) ||
+        !make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
+        !make_tile_map_2d(&vmap, v_cache, rows, head_dim, dtype))
+      return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
+  } else if (use_tc5) {
     if (!make_q_map(&qmap, q, total_q, num_q_heads, head_dim, group, dtype) ||
         !make_q_map(&omap, out, total_q, num_q_heads, head_dim, group, dtype) ||
         !make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
@@ -669,10 +677,11 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   a.v_cache = v_cache;
   a.tiles = 0;
   a.sched = static_cast<uint64_t*>(workspace);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
-      use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap, omap,
-                                       static_cast<cudaStream_t>(stream))
-              : pa::launch_prefill(a, dtype, kmap, vmap, static_cast<cudaStream_t>(stream));
+      use_pair  ? pa::launch_prefill_pair(a, dtype, qmap, kmap, vmap, omap, st)
+      : use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap, omap, st)
+                : pa::launch_prefill(a, dtype, kmap, vmap, st);
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
 }
 

@@ -22,7 +22,8 @@ struct PrefillArgs {
   int32_t num_blocks, max_blocks, max_q;
   int32_t total_q;             // rows of q and out
   int32_t three_d;             // tile maps are {64, rows, head_dim / 64}
-  int32_t tiles;               // 128-row query tiles per (sequence, kv head) (tcgen05 kernel)
+  int32_t tiles;               // query tiles (128 rows; 256 for the pair kernel) per
+                               // (sequence, kv head) (tcgen05 kernels)
   uint64_t* sched;             // NULL or {next item, CTAs done}, zero between calls (tcgen05)
   float scale_log2;
 };
@@ -45,5 +46,12 @@ cudaError_t launch_prefill(const PrefillArgs& a, pa_dtype dtype, const CUtensorM
 cudaError_t launch_prefill_tc5(PrefillArgs a, pa_dtype dtype, const CUtensorMap& qmap,
                                const CUtensorMap& kmap2d, const CUtensorMap& vmap3d,
                                const CUtensorMap& omap, cudaStream_t stream);
+
+// The same on pairs of SMs (cta_group::2, clusters of two CTAs, 256-row items):
+// the shapes of launch_prefill_tc5; kmap2d / vmap2d the {head_dim, rows} maps of
+// the key / value pools with a {64, 16} box (each CTA loads half of every tile).
+cudaError_t launch_prefill_pair(PrefillArgs a, pa_dtype dtype, const CUtensorMap& qmap,
+                                const CUtensorMap& kmap2d, const CUtensorMap& vmap2d,
+                                const CUtensorMap& omap, cudaStream_t stream);
 
 }  // namespace pa

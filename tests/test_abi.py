@@ -182,7 +182,7 @@ def _call_prefill(a):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(path=3), dict(path=-1), dict(dtype=pa.PA_F32), dict(T=-1), dict(B=-1), dict(B=70000),
+    dict(path=4), dict(path=-1), dict(dtype=pa.PA_F32), dict(T=-1), dict(B=-1), dict(B=70000),
     dict(Hkv=0), dict(Hq=7), dict(Hq=256, Hkv=2), dict(D=96), dict(bs=8), dict(bs=24),
     dict(NB=-1), dict(max_q=1 << 30), dict(scale=float("nan")), dict(kc=None),
     dict(q=C.c_void_p(2)), dict(kc=C.c_void_p(8)), dict(ws=C.c_void_p(4)),
@@ -190,6 +190,8 @@ def _call_prefill(a):
     dict(path=pa.PA_PREFILL_TCGEN05, D=64), dict(path=pa.PA_PREFILL_TCGEN05, scale=-1.0),
     dict(path=pa.PA_PREFILL_TCGEN05, q=C.c_void_p(20)),
     dict(path=pa.PA_PREFILL_TCGEN05, out=C.c_void_p(36)),
+    dict(path=pa.PA_PREFILL_TCGEN05_PAIR, D=64), dict(path=pa.PA_PREFILL_TCGEN05_PAIR, Hq=256,
+                                                       Hkv=1),
 ])
 def test_prefill_rejects_bad_arguments_on_host(bad):
     """Every limit pa.h states for pa_prefill_attention_ex is checked before anything

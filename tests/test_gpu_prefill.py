@@ -55,13 +55,21 @@ def _cases():
 CASES = _cases()
 
 
-PATHS = [pa.PA_PREFILL_AUTO, pa.PA_PREFILL_MMA_SYNC]
+# the automatic choice (the one-SM tcgen05 kernel where it applies), the tcgen05
+# kernel on pairs of SMs where it applies, and mma.sync
+PATHS = [pa.PA_PREFILL_AUTO, pa.PA_PREFILL_TCGEN05_PAIR, pa.PA_PREFILL_MMA_SYNC]
+
+
+def _path_applies(wl, path):
+    return path != pa.PA_PREFILL_TCGEN05_PAIR or (wl.D == 128 and 128 % wl.G == 0)
 
 
 @pytest.mark.parametrize("name", list(CASES))
 @pytest.mark.parametrize("path", PATHS)
 def test_prefill_small_configs_match_the_oracle(name, path):
     wl = CASES[name]()
+    if not _path_applies(wl, path):
+        pytest.skip("the tcgen05 pair kernel takes head_dim 128 only")
     eng, bt, ctx, qs, q = _build(wl)
     out = eng.prefill(q, bt, ctx, qs, int(wl.n_new.max()), wl.scale, path=path)
     torch.cuda.synchronize()
@@ -140,10 +148,12 @@ def test_prefill_guards(path):
 
 
 @pytest.mark.parametrize("name", ["f16_g4_d128", "bf16_g8_d128", "f16_g1_bs32"])
-def test_prefill_persistent_and_per_item_launches_agree(name):
-    """The tcgen05 kernel with a scheduling workspace (persistent, items handed
-    out by a counter) and without (one item per CTA) computes every item the
-    same way: identical bits, and the workspace is left zero for the next call."""
+@pytest.mark.parametrize("path", [pa.PA_PREFILL_TCGEN05, pa.PA_PREFILL_TCGEN05_PAIR])
+def test_prefill_persistent_and_per_item_launches_agree(name, path):
+    """Each tcgen05 kernel with a scheduling workspace (persistent, items handed
+    out by a counter) and without (one item per CTA or CTA pair) computes every
+    item the same way: identical bits, and the workspace is left zero for the
+    next call."""
     wl = CASES[name]()
     eng, bt, ctx, qs, q = _build(wl)
     max_q = int(wl.n_new.max())
@@ -152,7 +162,7 @@ def test_prefill_persistent_and_per_item_launches_agree(name):
     for workspace in (ws, None, ws):
         out = torch.full_like(q, float("nan"))
         pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
-                                eng.dev_error, pa.PA_PREFILL_TCGEN05, workspace)
+                                eng.dev_error, path, workspace)
         torch.cuda.synchronize()
         outs.append(out)
         assert not ws.any(), "the scheduling counter was not returned to zero"
