@@ -235,3 +235,20 @@ def test_overlapped_prologue_gives_the_same_bits():
     assert torch.equal(bits(outs[0]), bits(outs[1])) and torch.equal(bits(outs[1]), bits(outs[2]))
     assert not torch.equal(bits(outs[0]), bits(g["out"]))  # the rewritten tokens were seen
     assert eng.device_errors() == 0
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D,dtype", [(4096, 64, 64, 64, "f16"),   # B * Hkv = 262144
+                                              (4096, 32, 8, 128, "bf16")])  # the largest batch
+def test_maximum_batch_and_pair_counts(B, Hq, Hkv, D, dtype):
+    """The largest shapes the decode accepts: batch 4096 (the context scan's limit) and
+    batch x kv heads = 262144 (the workspace's arrival counts), with short contexts of
+    1..40 tokens; every row against the oracle, on both paths."""
+    rng = np.random.default_rng(90 + Hkv)
+    wl = workloads.custom("maxsz", dtype, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=16,
+                          ctx=rng.integers(1, 41, size=B), seed=91, shuffle=False)
+    ref, _ = all_rows(wl)
+    for path in (pa.PA_PATH_AUTO, pa.PA_PATH_SIMT):
+        g = build(wl, path=path)
+        ok, worst = tol_ok(g["out"].double().cpu().numpy(), ref, wl.dtype)
+        assert ok, (path, worst)
+        assert g["eng"].device_errors() == 0
