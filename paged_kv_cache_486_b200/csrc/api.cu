@@ -646,7 +646,6 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
       return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
   } else if (use_tc5) {
     if (!make_q_map(&qmap, q, total_q, num_q_heads, head_dim, group, dtype) ||
-        !make_q_map(&omap, out, total_q, num_q_heads, head_dim, group, dtype) ||
         !make_tile_map_2d(&kmap, k_cache, rows, head_dim, dtype) ||
         !make_tile_map(&vmap, &v3, v_cache, rows, head_dim, dtype) || !v3)
       return fail(PA_ERR_CUDA, "pa_prefill_attention: cuTensorMapEncodeTiled failed");
@@ -680,7 +679,7 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
       use_pair  ? pa::launch_prefill_pair(a, dtype, qmap, kmap, vmap, omap, st)
-      : use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap, omap, st)
+      : use_tc5 ? pa::launch_prefill_tc5(a, dtype, qmap, kmap, vmap, st)
                 : pa::launch_prefill(a, dtype, kmap, vmap, st);
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "pa_prefill_attention");
 }

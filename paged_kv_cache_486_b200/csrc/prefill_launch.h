@@ -22,8 +22,8 @@ struct PrefillArgs {
   int32_t num_blocks, max_blocks, max_q;
   int32_t total_q;             // rows of q and out
   int32_t three_d;             // tile maps are {64, rows, head_dim / 64}
-  int32_t tiles;               // query tiles (128 rows; 256 for the pair kernel) per
-                               // (sequence, kv head) (tcgen05 kernels)
+  int32_t tiles;               // work items of 256 query rows per (sequence, kv head)
+                               // (tcgen05 kernels)
   uint64_t* sched;             // NULL or {next item, CTAs done}, zero between calls (tcgen05)
   float scale_log2;
 };
@@ -38,17 +38,16 @@ cudaError_t launch_prefill(const PrefillArgs& a, pa_dtype dtype, const CUtensorM
                            const CUtensorMap& vmap, cudaStream_t stream);
 
 // tcgen05 kernel (persistent, one CTA per SM): head_dim 128, 128 % group == 0,
-// scale > 0, q and out 16-byte aligned; qmap / omap are the {head_dim,
-// num_q_heads, total_q} maps of q / out with a {64, group, 128 / group} box,
-// kmap2d the {head_dim, rows} map of the key pool with a {64, 16} box, vmap3d
-// the {64, rows, 2} map of the value pool with a {64, 16, 2} box, all with the
-// 128-byte swizzle.
+// scale > 0, q and out 16-byte aligned; qmap is the {head_dim, num_q_heads,
+// total_q} map of q with a {64, group, 128 / group} box, kmap2d the {head_dim,
+// rows} map of the key pool with a {64, 16} box, vmap3d the {64, rows, 2} map of
+// the value pool with a {64, 16, 2} box, all with the 128-byte swizzle.
 cudaError_t launch_prefill_tc5(PrefillArgs a, pa_dtype dtype, const CUtensorMap& qmap,
                                const CUtensorMap& kmap2d, const CUtensorMap& vmap3d,
-                               const CUtensorMap& omap, cudaStream_t stream);
+                               cudaStream_t stream);
 
 // The same on pairs of SMs (cta_group::2, clusters of two CTAs, 256-row items):
-// the shapes of launch_prefill_tc5; kmap2d / vmap2d the {head_dim, rows} maps of
+// the shapes of launch_prefill_tc5, omap the map of out like qmap; kmap2d / vmap2d the {head_dim, rows} maps of
 // the key / value pools with a {64, 16} box (each CTA loads half of every tile).
 cudaError_t launch_prefill_pair(PrefillArgs a, pa_dtype dtype, const CUtensorMap& qmap,
                                 const CUtensorMap& kmap2d, const CUtensorMap& vmap2d,
