@@ -419,8 +419,9 @@ pa_status pa_prefill_attention(void* out, const void* q, const void* k_cache,
  * workspace: NULL, or PA_PREFILL_WORKSPACE_BYTES of device memory, 8-byte
  *   aligned, owned by the caller, zero-filled once before its first use (e.g.
  *   cudaMemset); every call leaves it zero.  With it the tcgen05 kernel is
- *   persistent (one CTA per SM taking 128-row items from a counter there, by
- *   sequence and kv head with the latest query tile first), without it each
+ *   persistent (one CTA per SM taking 256-row items from a counter there: in
+ *   blocks of (sequence, kv head) pairs whose keys and values fit in part of L2,
+ *   the longest items first within a block), without it each
  *   CTA runs one item; the results are the same bits.  Calls sharing one workspace must not overlap on the GPU (order
  *   them on one stream).  The mma.sync kernel ignores it.
  * An unknown path, or PA_PREFILL_TCGEN05 for a shape it does not take, is

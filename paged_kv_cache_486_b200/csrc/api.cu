@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -676,6 +677,17 @@ pa_status pa_prefill_attention_ex(void* out, const void* q, const void* k_cache,
   a.v_cache = v_cache;
   a.tiles = 0;
   a.sched = static_cast<uint64_t*>(workspace);
+  {
+    // Pairs whose keys and values (at the table's full length) fit in about a
+    // third of L2 form one scheduling block: within it the items go longest
+    // first, so the kernel does not end on a long item, while the pairs being
+    // read at one time still fit in L2.
+    const int64_t pair_bytes =
+        std::max<int64_t>(1, static_cast<int64_t>(max_blocks) * block_size * head_dim * 2 * 2);
+    const int64_t pairs = static_cast<int64_t>(batch) * num_kv_heads;
+    a.pair_block = static_cast<int32_t>(
+        std::min<int64_t>(pairs, std::max<int64_t>(1, (int64_t(40) << 20) / pair_bytes)));
+  }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   const cudaError_t e =
       use_pair  ? pa::launch_prefill_pair(a, dtype, qmap, kmap, vmap, omap, st)

@@ -25,6 +25,8 @@ struct PrefillArgs {
   int32_t tiles;               // work items of 256 query rows per (sequence, kv head)
                                // (tcgen05 kernels)
   uint64_t* sched;             // NULL or {next item, CTAs done}, zero between calls (tcgen05)
+  int32_t pair_block;          // (one-SM tcgen05 kernel) items go longest first within
+                               // blocks of this many (sequence, kv head) pairs
   float scale_log2;
 };
 

@@ -31,9 +31,10 @@
 // contiguous bytes per row).
 //
 // Persistent when the caller gives a scheduling workspace: one CTA per SM takes
-// items from a global counter; items go by (sequence, kv head), the latest
-// (longest) rows first, so the items that read the same keys and values run on
-// neighbouring SMs at the same time and those reach each SM from L2.  The K
+// items from a global counter.  The (sequence, kv head) pairs go in blocks whose
+// keys and values fit in part of L2; within a block the longest items go first
+// (so the kernel does not end on a long one) and the items reading the same keys
+// and values run at about the same time, so those reach each SM from L2.  The K
 // producer takes the items and passes them to the other roles through a
 // four-slot ring in shared memory.  Without a workspace each CTA runs one item.
 //
@@ -149,6 +150,15 @@ __device__ __forceinline__ void mma_ts4(uint32_t d, const uint32_t (&ta)[4], con
       : "memory");
 }
 
+// One 32-byte store (the address 32-byte aligned).
+__device__ __forceinline__ void st_global8(void* p, uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
+                                           uint32_t a7) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0),
+               "r"(a1), "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+               : "memory");
+}
+
 __device__ __forceinline__ void commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                ::"r"(bar) : "memory");
@@ -175,13 +185,19 @@ struct Item {
   int r0[2], n_keys_h[2];
 };
 
-// Item w: (sequence, kv head) w / tiles, its pair of query tiles
-// tiles - 1 - w % tiles (latest first).  False when there is nothing to do (the
-// sequence has fewer rows, no new tokens, or lengths outside the launch's
-// bounds, which `rep` reports).
+// Item w.  The (sequence, kv head) pairs go in blocks of a.pair_block; within
+// a block the items go by rank, rank x being each pair's pair of query tiles
+// tiles - 1 - x (the latest, longest, first), pair by pair.  False when there
+// is nothing to do (the sequence has fewer rows, no new tokens, or lengths
+// outside the launch's bounds, which `rep` reports).
 __device__ __forceinline__ bool item_at(const PrefillArgs& a, int64_t w, Item& it, bool rep) {
-  const int64_t bg = w / a.tiles;
-  const int x = static_cast<int>(w - bg * a.tiles);
+  const int64_t n_pairs = static_cast<int64_t>(a.num_kv_heads) * a.batch;
+  const int64_t pb = a.pair_block;
+  const int64_t blk = w / (pb * a.tiles);
+  const int64_t local = w - blk * pb * a.tiles;
+  const int64_t in_blk = min(pb, n_pairs - blk * pb);  // pairs in this block
+  const int x = static_cast<int>(local / in_blk);
+  const int64_t bg = blk * pb + (local - x * in_blk);
   it.g = static_cast<int>(bg % a.num_kv_heads);
   it.b = static_cast<int>(bg / a.num_kv_heads);
   const int tile_q = a.tiles - 1 - x;
@@ -739,31 +755,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) {
         fence_after();
         const float inv = 1.f / ((l0 + l1) + (l2 + l3));
-        uint4* dst = nullptr;
+        T* dst = nullptr;
         if (grow < it.rows) {
           const int tok = grow / G, hh = grow - tok * G;
-          dst = reinterpret_cast<uint4*>(
-              static_cast<T*>(a.out) +
-              (static_cast<int64_t>(it.q0 + tok) * a.num_q_heads + it.g * G + hh) * kD);
+          dst = static_cast<T*>(a.out) +
+                (static_cast<int64_t>(it.q0 + tok) * a.num_q_heads + it.g * G + hh) * kD;
         }
+        // rows are 256 bytes: 32-byte stores when out allows them, else 16-byte
+        const bool wide = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t ou[32];
-          tmem_ld32_issue(trow + col_o + 32 * ch, ou);
-          tmem_ld_wait(ou);
+        for (int ch = 0; ch < 4; ch += 2) {
+          uint32_t ou[2][32];
+          tmem_ld32_issue(trow + col_o + 32 * ch, ou[0]);
+          tmem_ld32_issue(trow + col_o + 32 * ch + 32, ou[1]);
+          tmem_ld_wait(ou[0]);  // waits for both
+          tmem_ld_wait(ou[1]);
           if (dst) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint4 v;
-              v.x = tc::pack2<T>(__uint_as_float(ou[8 * k]) * inv,
-                                 __uint_as_float(ou[8 * k + 1]) * inv);
-              v.y = tc::pack2<T>(__uint_as_float(ou[8 * k + 2]) * inv,
-                                 __uint_as_float(ou[8 * k + 3]) * inv);
-              v.z = tc::pack2<T>(__uint_as_float(ou[8 * k + 4]) * inv,
-                                 __uint_as_float(ou[8 * k + 5]) * inv);
-              v.w = tc::pack2<T>(__uint_as_float(ou[8 * k + 6]) * inv,
-                                 __uint_as_float(ou[8 * k + 7]) * inv);
-              dst[4 * ch + k] = v;
+            for (int c2 = 0; c2 < 2; ++c2) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = tc::pack2<T>(__uint_as_float(ou[c2][2 * i]) * inv,
+                                     __uint_as_float(ou[c2][2 * i + 1]) * inv);
+              T* d = dst + 32 * (ch + c2);  // 64 bytes
+              if (wide) {
+                st_global8(d, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+                st_global8(d + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
+              } else {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  reinterpret_cast<uint4*>(d)[k] =
+                      make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+              }
             }
           }
         }
