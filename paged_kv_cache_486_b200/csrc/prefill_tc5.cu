@@ -241,9 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barriers: k_full, k_empty (one per K stage each; a stage is free after a
   // commit per half), v_full, v_empty (the same for V), per half q_full,
   // q_empty (its Q tile may be reloaded), o_free (O_h read by the epilogue),
-  // final (one per issuer: its UMMAs completed), per half and score buffer s_full (scores
-  // written), p_full (P written), pv_done (the P . V that read it completed),
-  // then the item ring
+  // final (one per issuer: its UMMAs completed), per half and score buffer
+  // s_full (scores written), p_full (P written), pv_done (the P . V that read it
+  // completed), then the item ring
   constexpr int kB = 2 * (kKStages + kVStages);
   const uint32_t b_k_full = tc::smem_u32(&bars[0]);
   const uint32_t b_k_empty = tc::smem_u32(&bars[kKStages]);
