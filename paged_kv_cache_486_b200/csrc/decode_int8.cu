@@ -21,7 +21,11 @@
 //    and two byte permutes per four codes; the product then carries
 //    1152 * sum_d q_d too, which is subtracted once per segment (the
 //    accumulator starts at -1152 * sum_d q_d).
-//  * Values enter as the signed codes (exact), so O needs no correction.
+//  * Values enter the same way, as 1024 + u: O then carries 1152 * sum_j p'_j
+//    in every row, which one more product per stage (an all-ones A operand
+//    against the same P fragment) accumulates exactly; it is subtracted at the
+//    segment's end.  (Two byte permutes per four codes instead of two byte
+//    permutes and two fp16 subtractions.)
 // Scales.  Key scales multiply the score rows (with scale * log2 e).  Value
 // scales are folded into P: p'_j = p_j * vs_j / sigma with sigma a lazily
 // updated running maximum of the segment's value scales (p' stays within a
@@ -43,15 +47,6 @@ namespace tc {
 // the fp16 value 1024 + u exactly.
 __device__ __forceinline__ uint2 codes_biased(uint32_t w) {
   return make_uint2(__byte_perm(w, 0x64646464u, 0x5140), __byte_perm(w, 0x64646464u, 0x7362));
-}
-
-// The same four codes as signed fp16 values u - 128 (1024 + u minus 1152, exact).
-__device__ __forceinline__ uint2 codes_signed(uint32_t w) {
-  const uint2 b = codes_biased(w);
-  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));
-  const __half2 l = __hsub2(*reinterpret_cast<const __half2*>(&b.x), bias);
-  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&b.y), bias);
-  return make_uint2(*reinterpret_cast<const uint32_t*>(&l), *reinterpret_cast<const uint32_t*>(&h));
 }
 
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
@@ -76,6 +71,8 @@ struct Tiles8 {
   static constexpr int D = i8::kDim;
   static constexpr int KC = D / 16;
   static constexpr int kStages = 5;
+  static constexpr int kConsumerRegs = 208;
+  static constexpr int kProducerRegs = 48;
   static constexpr int kRec = i8::kRecordBytes;
   static constexpr int kStageBytes = 2 * kRec;  // key record + value record
   static constexpr int kRingBytes = (kWarps * kStages * kStageBytes + 1023) / 1024 * 1024;
@@ -91,9 +88,28 @@ struct Tiles8 {
     float sig, inv;  // value-scale normaliser sigma and 1 / sigma
     float c0, c1;    // scale * log2 e / prescale, heads 2cq and 2cq + 1
     float qs0, qs1;  // -1152 * sum_d q'_d, heads 2cq and 2cq + 1
-    __device__ void reset() { sig = inv = 0.f; }
+    float bsum[4];   // sum_j p'_j in O's fragment layout (every row the same)
+    __device__ void reset() {
+      sig = inv = 0.f;
+      bsum[0] = bsum[1] = bsum[2] = bsum[3] = 0.f;
+    }
     __device__ float out_scale() const { return sig; }
   };
+  // the softmax reference moved: sum_j p'_j scales like O (heads 2cq, 2cq + 1)
+  __device__ static void rescale(Seg& seg, float a0, float a1) {
+    seg.bsum[0] *= a0;
+    seg.bsum[1] *= a1;
+    seg.bsum[2] *= a0;
+    seg.bsum[3] *= a1;
+  }
+  // O = O' - 1152 sum_j p'_j: the value offset carried by the biased codes
+  __device__ static void finish(float (&o)[KC][4], const Seg& seg) {
+#pragma unroll
+    for (int mt = 0; mt < KC; ++mt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[mt][e] = fmaf(-1152.f, seg.bsum[e], o[mt][e]);
+    }
+  }
 
   __device__ static void prefetch(const Maps&) {}
   __device__ static uint32_t stage(uint32_t ring0, int warp, int slot) {
@@ -224,6 +240,8 @@ struct Tiles8 {
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[mt][e] *= r;
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) seg.bsum[e] *= r;
       seg.sig = mx;
       seg.inv = 1.f / mx;
     }
@@ -233,11 +251,14 @@ struct Tiles8 {
                             transpose8x8(pack2<__half>(p[2] * u1, p[3] * u1))};
 #pragma unroll
     for (int mt = 0; mt < KC; ++mt) {
-      const uint2 r0 = codes_signed(f.v[mt][0]);
-      const uint2 r1 = codes_signed(f.v[mt][1]);
+      const uint2 r0 = codes_biased(f.v[mt][0]);
+      const uint2 r1 = codes_biased(f.v[mt][1]);
       const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
       mma16816<__half>(o[mt], A, pb);
     }
+    // sum_j p'_j of the 16 tokens for each head (fp16 1.0 pairs)
+    const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};
+    mma16816<__half>(seg.bsum, ones, pb);
   }
 };
 

@@ -21,6 +21,8 @@ template <typename T, int D>
 struct Tiles16 {
   static constexpr int KC = D / 16;
   static constexpr int kStages = 3;
+  static constexpr int kConsumerRegs = tc::kConsumerRegs;
+  static constexpr int kProducerRegs = tc::kProducerRegs;
   static constexpr int kTileBytes = kTok * D * 2;
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kWarps * kStages * kStageBytes;
@@ -35,6 +37,8 @@ struct Tiles16 {
     __device__ void reset() {}
     __device__ float out_scale() const { return 1.f; }
   };
+  __device__ static void rescale(Seg&, float, float) {}
+  __device__ static void finish(float (&)[D / 16][4], const Seg&) {}
 
   __device__ static void prefetch(const Maps& m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&m.k)) : "memory");

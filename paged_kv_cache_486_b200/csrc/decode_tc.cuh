@@ -27,14 +27,18 @@
 //   Tiles8  (decode_int8.cu): 8-bit codes with a per-token fp32 scale.
 // A policy provides:
 //   kStages, kStageBytes (bytes TMA delivers per stage), kRingBytes (shared
-//   memory of all rings, a multiple of 1024), Maps (tensor maps, a kernel
+//   memory of all rings, a multiple of 1024), kConsumerRegs / kProducerRegs
+//   (the register split, below), Maps (tensor maps, a kernel
 //   parameter), Frag (one stage in registers), Seg (per-segment state);
 //   prefetch(maps); issue(maps, a, ring0, warp, slot, tile, tok, bar) (lane 0);
 //   q_off(kc, cq, half) (head_dim offset of a query fragment register);
 //   prep_q(qf, seg, a, lane) (once per segment, after seg.reset(), on the
 //     segment's query fragments: whatever the policy's products need);
 //   load(a, ring0, warp, slot, n_valid, lane, frag);
-//   scores(frag, qf, seg, a, n_valid, lane, t[4]);  pv(frag, p[4], o, seg, n_valid, lane).
+//   scores(frag, qf, seg, a, n_valid, lane, t[4]);  pv(frag, p[4], o, seg, n_valid, lane);
+//   rescale(seg, a0, a1) (the softmax reference moved: what the policy keeps
+//     alongside O is scaled like O's heads 2cq, 2cq + 1);
+//   finish(o, seg) (at the segment's end, before O is scaled and written).
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -272,7 +276,9 @@ __device__ __forceinline__ UnitDesc shfl_desc(const UnitDesc& d, int k) {
 // warp.  Registers: the CTA is launched with kLaunchRegs per thread; producer
 // warpgroups give most of theirs up (setmaxnreg.dec to kProducerRegs), worker
 // warpgroups take them (setmaxnreg.inc to kConsumerRegs).  The two counts add
-// up to twice the launch count, the most the hand-over can provide.
+// up to twice the launch count, the most the hand-over can provide.  A policy
+// may set its own split (P::kConsumerRegs, P::kProducerRegs); the 8-bit one
+// gives its workers 208 (the codes' conversions need them) and its producers 48.
 constexpr int kLaunchRegs = 128;
 constexpr int kConsumerRegs = 216;
 constexpr int kProducerRegs = 40;
@@ -285,6 +291,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
     decode_tc_kernel(const __grid_constant__ typename P::Maps maps, DecodeArgs a) {
   constexpr int KC = D / 16;  // 16-wide chunks of head_dim
   constexpr int kStages = P::kStages;
+  static_assert(P::kConsumerRegs + P::kProducerRegs <= 2 * kLaunchRegs, "register split");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t ring0 = (raw + 1023u) & ~1023u;
@@ -322,7 +329,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
 
   if (warp >= kWarps) {
     // =============================== producer ===============================
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(P::kProducerRegs));
     if (!active) return;
     int64_t prange = w;
     int64_t pr0 = sp.start(w);
@@ -407,7 +414,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
   }
 
   // ================================ worker ==================================
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kConsumerRegs));
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(P::kConsumerRegs));
   if (!active) return;
   const int g = lane >> 2, cq = lane & 3;
   uint32_t qf[KC][2], qn[KC][2];
@@ -518,6 +525,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
           o[kc][2] *= a0;
           o[kc][3] *= a1;
         }
+        P::rescale(seg, a0, a1);
         m0 = n0;
         m1 = n1;
       }
@@ -529,6 +537,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
     }
 
     if (flags & kSegEnd) {
+      P::finish(o, seg);
       float L0 = l0, L1 = l1;
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
