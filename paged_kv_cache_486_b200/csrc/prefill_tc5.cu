@@ -150,6 +150,13 @@ __device__ __forceinline__ void mma_ts4(uint32_t d, const uint32_t (&ta)[4], con
       : "memory");
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // One 32-byte store (the address 32-byte aligned).
 __device__ __forceinline__ void st_global8(void* p, uint32_t a0, uint32_t a1, uint32_t a2,
                                            uint32_t a3, uint32_t a4, uint32_t a5, uint32_t a6,
@@ -643,7 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int grow = (h ? it.r0[1] : it.r0[0]) + r;
       const int pos = grow < it.rows ? it.past + grow / G : -1;
       float mref = -INFINITY;  // running reference, scaled (log2) domain
-      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+      // the row sum in two pairs, accumulated with packed fp32 adds
+      float2 la = make_float2(0.f, 0.f), lb = make_float2(0.f, 0.f);
       for (int u = 0; u < n_sub; ++u, ++m) {
         const uint32_t j = m & 1;
         if (ok) ok = wait_ok(bar_s + 8 * j, (m >> 1) & 1, abort_flag, a.dev_error);
@@ -675,13 +683,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            x0 = fmaxf(x0, sv[ch][i]);
-            x1 = fmaxf(x1, sv[ch][i + 1]);
-            x2 = fmaxf(x2, sv[ch][i + 2]);
-            x3 = fmaxf(x3, sv[ch][i + 3]);
+          for (int i = 0; i < 32; i += 8) {
+            x0 = fmax3(x0, sv[ch][i], sv[ch][i + 1]);
+            x1 = fmax3(x1, sv[ch][i + 2], sv[ch][i + 3]);
+            x2 = fmax3(x2, sv[ch][i + 4], sv[ch][i + 5]);
+            x3 = fmax3(x3, sv[ch][i + 6], sv[ch][i + 7]);
           }
-        const float mx_raw = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        const float mx_raw = fmax3(fmaxf(x0, x1), x2, x3);
         const float mx = mx_raw == -INFINITY ? -INFINITY : mx_raw * c;
         // a row whose maximum rose by more than 2^kSlack takes it as its new
         // reference and rescales its row of O_h once the half's previous
@@ -708,13 +716,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_st32(trow + col_o + 32 * ch, ou);
             }
           }
-          l0 *= alpha;
-          l1 *= alpha;
-          l2 *= alpha;
-          l3 *= alpha;
+          la = __fmul2_rn(la, make_float2(alpha, alpha));
+          lb = __fmul2_rn(lb, make_float2(alpha, alpha));
           mref = mnew;
         }
         const float neg = mref == -INFINITY ? 0.f : -mref;
+        // x = s c - reference, two at a time (packed fp32 FMA)
+        const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
         // P over this sub-tile's score columns: head pairs in columns 0..31,
         // tails in 32..63
 #pragma unroll
@@ -722,14 +730,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t ph[16], pt[16];
 #pragma unroll
           for (int i = 0; i < 16; i += 2) {
-            const float p0 = ex2(fmaf(sv[ch][2 * i], c, neg));
-            const float p1 = ex2(fmaf(sv[ch][2 * i + 1], c, neg));
-            const float p2 = ex2(fmaf(sv[ch][2 * i + 2], c, neg));
-            const float p3 = ex2(fmaf(sv[ch][2 * i + 3], c, neg));
-            l0 += p0;
-            l1 += p1;
-            l2 += p2;
-            l3 += p3;
+            const float2 xa = __ffma2_rn(make_float2(sv[ch][2 * i], sv[ch][2 * i + 1]), c2, n2);
+            const float2 xb =
+                __ffma2_rn(make_float2(sv[ch][2 * i + 2], sv[ch][2 * i + 3]), c2, n2);
+            const float p0 = ex2(xa.x), p1 = ex2(xa.y), p2 = ex2(xb.x), p3 = ex2(xb.y);
+            la = __fadd2_rn(la, make_float2(p0, p1));
+            lb = __fadd2_rn(lb, make_float2(p2, p3));
             if (PrefillPSplit<T>::value) {
               tc::split2<T>(p0, p1, ph[i], pt[i]);
               tc::split2<T>(p2, p3, ph[i + 1], pt[i + 1]);
@@ -754,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok) {
         fence_after();
-        const float inv = 1.f / ((l0 + l1) + (l2 + l3));
+        const float inv = 1.f / ((la.x + la.y) + (lb.x + lb.y));
         T* dst = nullptr;
         if (grow < it.rows) {
           const int tok = grow / G, hh = grow - tok * G;
