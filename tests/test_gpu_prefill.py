@@ -169,3 +169,34 @@ def test_prefill_persistent_and_per_item_launches_agree(name, path):
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
     assert eng.device_errors() == 0
+
+
+@pytest.mark.parametrize("width", [1024, 2000, 6000])
+def test_prefill_item_order_blocks_of_pairs(width):
+    """The one-SM tcgen05 kernel hands out its items longest first within blocks
+    of (sequence, kv head) pairs sized from the table's width (the pairs whose
+    keys and values fit in part of L2).  A wider table with the same contents
+    gives blocks of 5, 2 and 1 of these 48 pairs (the last block partial for 5):
+    every row still matches the oracle, persistent or one item per CTA, with the
+    same bits as the narrow table."""
+    wl = workloads.prefill("w", "f16", 32, 8, 128, 16, [40, 129, 513, 1000, 700, 260],
+                           [40, 1, 200, 513, 700, 77], 39)
+    eng, bt, ctx, qs, q = _build(wl)
+    wide, ctx_w = eng.block_tables(wl.batch, width)
+    assert torch.equal(ctx, ctx_w) and torch.equal(wide[:, :bt.shape[1]], bt)
+    max_q = int(wl.n_new.max())
+    o = run_script(wl)
+    ref = oracle.paged_prefill_attention(raw(q), o["k_cache"], o["v_cache"], o["table"],
+                                         o["ctx"], workloads.query_start(wl), wl.scale, wl.dtype)
+    narrow = torch.empty_like(q)
+    pa.pa_prefill_attention(narrow, q, eng.k_cache, eng.v_cache, bt, ctx, qs, max_q, wl.scale,
+                            eng.dev_error, pa.PA_PREFILL_TCGEN05, eng.prefill_ws)
+    for workspace in (eng.prefill_ws, None):
+        out = torch.full_like(q, float("nan"))
+        pa.pa_prefill_attention(out, q, eng.k_cache, eng.v_cache, wide, ctx, qs, max_q,
+                                wl.scale, eng.dev_error, pa.PA_PREFILL_TCGEN05, workspace)
+        torch.cuda.synchronize()
+        ok, worst = tol_ok(out.double().cpu().numpy(), ref, wl.dtype)
+        assert ok, f"worst error / bound = {worst:.3f}"
+        assert torch.equal(out.view(torch.int16), narrow.view(torch.int16))
+    assert eng.device_errors() == 0
