@@ -146,3 +146,26 @@ def int8_contiguous_row(wl, b, heads):
                                                [n], wl.scale, wl.dtype)
         out[h] = o[0, 0]
     return out
+
+
+def int8_all_rows(wl, device="cuda", threads=None):
+    """Oracle INT8 attention [B, Hq, D] of every batch row: each sequence's
+    logical rows (drawn on `device`, the same bits anywhere) quantised into a
+    fresh one-sequence oracle cache of all its kv heads, then the oracle's paged
+    INT8 decode over it.  Rows run in parallel on the host cores."""
+    q = raw(wl.q())
+
+    def row(b):
+        seq = int(wl.batch[b])
+        k = raw(wl.contiguous_kv(seq, 0, device))
+        v = raw(wl.contiguous_kv(seq, 1, device))
+        n = k.shape[0]
+        nb = max(1, -(-n // wl.bs))
+        cache = oracle.Int8Cache(nb, wl.Hkv, wl.bs, wl.D)
+        assert oracle.reshape_and_cache_int8(k, v, cache, np.arange(n), wl.dtype) == oracle.OK
+        o = oracle.paged_decode_attention_int8(q[b][None], cache, np.arange(nb)[None], [n],
+                                               wl.scale, wl.dtype, n_threads=1)
+        return o[0]
+
+    with cf.ThreadPoolExecutor(threads or os.cpu_count() or 4) as ex:
+        return np.stack(list(ex.map(row, range(wl.B))))

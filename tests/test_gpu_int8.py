@@ -114,6 +114,21 @@ def test_int8_full_size_configs(name):
     assert eng.device_errors() == 0
 
 
+@pytest.mark.parametrize("name", ["llama3_8b", "llama3_70b"])
+def test_int8_full_size_every_row(name):
+    """Every output row of the full-size INT8 decode workloads against the oracle,
+    elementwise at the fp16 / bf16 bound.  Values enter the products as biased
+    codes whose offset (1152 times the summed weights) is taken out at the end,
+    so the longest contexts are where its cancellation in fp32 would show."""
+    from oracle_side import int8_all_rows
+    wl = workloads.make(name)
+    g = build_int8(wl)
+    ref = int8_all_rows(wl)
+    ok, worst = tol_ok(g["out"].double().cpu().numpy(), ref, wl.dtype)
+    assert ok, f"worst error / bound = {worst:.3f}"
+    assert g["eng"].device_errors() == 0
+
+
 def test_int8_value_scales_of_very_different_magnitudes():
     """Token rows scaled by 2^-24 .. 2^12 (fp16 keys and values stay finite):
     the running value-scale normaliser keeps P' in [0, 1], so tiny and huge
