@@ -98,6 +98,19 @@ def _traffic(config, names=DECODE_SOURCES):
     return None
 
 
+def _spread(ms):
+    """Median and 10th / 90th percentiles (nearest rank) of per-iteration times in
+    ms, reported in microseconds."""
+    xs = sorted(ms)
+    if not xs:
+        return None
+
+    def q(p):
+        return xs[min(len(xs) - 1, max(0, int(round(p * (len(xs) - 1)))))] * 1e3
+
+    return {"p10": q(0.1), "p50": q(0.5), "p90": q(0.9), "n": len(xs), "unit": "us"}
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -320,7 +333,8 @@ def run_ours(args, dist, rank, world):
         "config": workload_config(wl, world),
         "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3,
         "kv_unique_bytes": uniq, "kv_unique_read_gbs": uniq / (dec_ms / 1e3) / 1e9,
-        "decode_us_min": min(decode_ms) * 1e3,
+        "decode_us_min": min(decode_ms) * 1e3, "decode_us_spread": _spread(decode_ms),
+        "step_us_spread": _spread(step_ms),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
                      "traffic": _traffic(wl.name),
@@ -369,7 +383,8 @@ def decode_only(name, args, batch=0):
     peak, kind = _peak_hbm()
     res = {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv,
            "dtype": wl.dtype, "kv_read_bytes": alg, "decode_us": t * 1e6,
-           "decode_us_min": min(ms) * 1e3, "tokens_per_s": wl.B / t,
+           "decode_us_min": min(ms) * 1e3, "decode_us_spread": _spread(ms),
+           "tokens_per_s": wl.B / t,
            "roofline": {"bound": "hbm", "achieved": alg / t / 1e9, "peak": peak, "unit": "GB/s",
                         "frac": alg / t / 1e9 / peak, "peak_source": f"{kind} (hbm_gbs copy)",
                         "traffic": _traffic(wl.name)},
@@ -612,6 +627,7 @@ def run_int8(args, dist, rank, world):
                              "CUDA events per step",
                    "l2": "flushed between timed steps (256 MiB read outside the events)"},
         "kv_read_gbs": achieved, "decode_us": dec_ms * 1e3, "decode_us_min": min(decode_ms) * 1e3,
+        "decode_us_spread": _spread(decode_ms), "step_us_spread": _spread(step_ms),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": f"{peak_kind} (hbm_gbs copy)",
                      "traffic": _traffic(wl.name + "_int8", INT8_SOURCES),
@@ -786,7 +802,8 @@ def run_prefill(args, dist, rank, world):
                    "head_dim": wl.D, "block_size": wl.bs, "new_tokens": tokens,
                    "context_tokens": int(c.sum()), "attended_pairs": pairs,
                    "l2": "flushed between timed calls (256 MiB read outside the events)"},
-        "prefill_us": 1e3 * statistics.mean(ms), "kv_read_bytes": kv_bytes,
+        "prefill_us": 1e3 * statistics.mean(ms), "prefill_us_spread": _spread(ms),
+        "kv_read_bytes": kv_bytes,
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "peak_source": kind,
                      "traffic": (None if args.prefill_path == 2 or wl.D != 128

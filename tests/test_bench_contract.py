@@ -32,3 +32,14 @@ def test_reduced_batch_workloads_for_profiling():
         pass
     else:
         raise AssertionError("shared_prefix has a fixed batch")
+
+
+def test_spread_is_nearest_rank_percentiles_in_microseconds():
+    """The per-iteration spread the bench lines carry (median and 10th / 90th
+    percentiles of the CUDA-event times): nearest rank over the sorted times,
+    reported in microseconds, independent of the input order."""
+    import bench
+    ms = [0.9, 0.1, 0.5, 0.3, 0.7, 0.2, 0.8, 0.4, 0.6, 1.0, 0.0]
+    s = bench._spread(ms)
+    assert s == {"p10": 100.0, "p50": 500.0, "p90": 900.0, "n": 11, "unit": "us"}
+    assert bench._spread([]) is None
