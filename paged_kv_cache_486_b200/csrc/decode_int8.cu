@@ -83,6 +83,8 @@ struct Tiles8 {
     uint32_t k[KC][2];  // [kc][row g, row g + 8]: 4 codes, d = 16kc + 4cq .. +3
     uint32_t v[KC][2];  // [mt][d = 16mt + g, +8]: 4 codes, tokens 4cq .. +3
     float ks0, ks1, vs0, vs1;  // scales of the lane's tokens row_token(g), +2
+    uint32_t va[KC][4];        // value A operands (biased fp16 pairs)
+    float u0, u1;              // value weights vs / sigma of the lane's tokens
   };
   struct Seg {
     float sig, inv;  // value-scale normaliser sigma and 1 / sigma
@@ -222,14 +224,26 @@ struct Tiles8 {
     if (tk + 2 >= n_valid) t[2] = t[3] = -INFINITY;
   }
 
-  __device__ static void pv(const Frag& f, const float (&p)[4], float (&o)[KC][4], Seg& seg,
-                            int n_valid, int lane) {
+  // Work of the value product that does not need P, done while the score
+  // products are in flight: the value codes' conversion and the normaliser.
+  __device__ static void pre_pv(Frag& f, float (&o)[KC][4], Seg& seg, int n_valid, int lane) {
+#pragma unroll
+    for (int mt = 0; mt < KC; ++mt) {
+      const uint2 r0 = codes_biased(f.v[mt][0]);
+      const uint2 r1 = codes_biased(f.v[mt][1]);
+      f.va[mt][0] = r0.x;
+      f.va[mt][1] = r1.x;
+      f.va[mt][2] = r0.y;
+      f.va[mt][3] = r1.y;
+    }
     const int tk = row_token(lane >> 2);
     const float w0 = tk < n_valid ? f.vs0 : 0.f;
     const float w1 = tk + 2 < n_valid ? f.vs1 : 0.f;
     // Lazy normaliser: sigma moves only when a value scale exceeds 16 sigma
     // (then to the stage's largest scale, the same in every lane), so
-    // vs / sigma <= 16 and p' = p vs / sigma <= 2^12, well inside fp16.
+    // vs / sigma <= 16 and p' = p vs / sigma <= 2^12, well inside fp16.  (O
+    // is rescaled here before the stage's softmax may rescale it: the two
+    // factors commute.)
     if (__any_sync(kFull, fmaxf(w0, w1) > seg.sig * 16.f)) {
       float mx = fmaxf(w0, w1);
 #pragma unroll
@@ -245,17 +259,17 @@ struct Tiles8 {
       seg.sig = mx;
       seg.inv = 1.f / mx;
     }
-    const float u0 = w0 * seg.inv, u1 = w1 * seg.inv;
+    f.u0 = w0 * seg.inv;
+    f.u1 = w1 * seg.inv;
+  }
+
+  __device__ static void pv(const Frag& f, const float (&p)[4], float (&o)[KC][4], Seg& seg,
+                            int, int) {
     // fp16 weights (11-bit significand, p' <= 2^12) in one product
-    const uint32_t pb[2] = {transpose8x8(pack2<__half>(p[0] * u0, p[1] * u0)),
-                            transpose8x8(pack2<__half>(p[2] * u1, p[3] * u1))};
+    const uint32_t pb[2] = {transpose8x8(pack2<__half>(p[0] * f.u0, p[1] * f.u0)),
+                            transpose8x8(pack2<__half>(p[2] * f.u1, p[3] * f.u1))};
 #pragma unroll
-    for (int mt = 0; mt < KC; ++mt) {
-      const uint2 r0 = codes_biased(f.v[mt][0]);
-      const uint2 r1 = codes_biased(f.v[mt][1]);
-      const uint32_t A[4] = {r0.x, r1.x, r0.y, r1.y};
-      mma16816<__half>(o[mt], A, pb);
-    }
+    for (int mt = 0; mt < KC; ++mt) mma16816<__half>(o[mt], f.va[mt], pb);
     // sum_j p'_j of the 16 tokens for each head (fp16 1.0 pairs)
     const uint32_t ones[4] = {0x3c003c00u, 0x3c003c00u, 0x3c003c00u, 0x3c003c00u};
     mma16816<__half>(seg.bsum, ones, pb);

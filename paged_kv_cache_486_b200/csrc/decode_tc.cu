@@ -38,6 +38,7 @@ struct Tiles16 {
     __device__ float out_scale() const { return 1.f; }
   };
   __device__ static void rescale(Seg&, float, float) {}
+  __device__ static void pre_pv(Frag&, float (&)[D / 16][4], Seg&, int, int) {}
   __device__ static void finish(float (&)[D / 16][4], const Seg&) {}
 
   __device__ static void prefetch(const Maps& m) {
@@ -70,6 +71,8 @@ struct Tiles16 {
         const uint32_t addr = vt + h * kBoxBytes + n_valid * 128 + r * 16;
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
       }
+      // generic writes to a slot that TMA refills later
+      fence_proxy_async_smem();
       __syncwarp();
     }
     const int mi = lane >> 3;

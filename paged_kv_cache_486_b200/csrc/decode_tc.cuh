@@ -35,7 +35,10 @@
 //   prep_q(qf, seg, a, lane) (once per segment, after seg.reset(), on the
 //     segment's query fragments: whatever the policy's products need);
 //   load(a, ring0, warp, slot, n_valid, lane, frag);
-//   scores(frag, qf, seg, a, n_valid, lane, t[4]);  pv(frag, p[4], o, seg, n_valid, lane);
+//   scores(frag, qf, seg, a, n_valid, lane, t[4]);
+//   pre_pv(frag, o, seg, n_valid, lane) (right after scores: the value
+//     product's work that does not need P, overlapping the score products);
+//   pv(frag, p[4], o, seg, n_valid, lane);
 //   rescale(seg, a0, a1) (the softmax reference moved: what the policy keeps
 //     alongside O is scaled like O's heads 2cq, 2cq + 1);
 //   finish(o, seg) (at the segment's end, before O is scaled and written).
@@ -491,10 +494,12 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
 
     const int n_valid = md.n_valid;
     const bool have = (flags & kHasData) != 0;
-    // Move the stage into registers and hand the slot straight back.
+    // Move the stage into registers and hand the slot straight back.  The
+    // arrive (release semantics) orders the warp's reads of the slot before the
+    // producer's next copy into it; a policy that writes the slot itself fences
+    // those writes against the copy (async proxy) inside load().
     typename P::Frag fr;
     if (have) P::load(a, ring0, ww, slot, n_valid, lane, fr);
-    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + slot * 8);
 
@@ -503,6 +508,7 @@ __global__ void __launch_bounds__(2 * kWarps * 32, 1)
       // units, -inf past the context
       float t[4];
       P::scores(fr, qf, seg, a, n_valid, lane, t);
+      P::pre_pv(fr, o, seg, n_valid, lane);
       // Lazy running maximum: weights are taken against the current reference m
       // unless some score of the stage is more than kSlack above it (then the
       // stage's maximum is reduced across the warp and the sums are rescaled).
