@@ -56,6 +56,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "decode_tc.cuh"
 #include "prefill_launch.h"
@@ -679,73 +680,105 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i)
               if (key0 + 32 * ch + i > pos) sv[ch][i] = -INFINITY;
         }
+        // P over this sub-tile's score columns (head pairs in columns 0..31,
+        // tails in 32..63) against the reference -neg, x = s c - reference two
+        // at a time (packed fp32 FMA); with kMax the sub-tile's raw maximum is
+        // taken in the same pass.
         float x0 = -INFINITY, x1 = -INFINITY, x2 = -INFINITY, x3 = -INFINITY;
+        auto exps = [&](float neg, auto kMax) {
+          const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t ph[16], pt[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            x0 = fmax3(x0, sv[ch][i], sv[ch][i + 1]);
-            x1 = fmax3(x1, sv[ch][i + 2], sv[ch][i + 3]);
-            x2 = fmax3(x2, sv[ch][i + 4], sv[ch][i + 5]);
-            x3 = fmax3(x3, sv[ch][i + 6], sv[ch][i + 7]);
-          }
-        const float mx_raw = fmax3(fmaxf(x0, x1), x2, x3);
-        const float mx = mx_raw == -INFINITY ? -INFINITY : mx_raw * c;
-        // a row whose maximum rose by more than 2^kSlack takes it as its new
-        // reference and rescales its row of O_h once the half's previous
-        // P . V has completed.  TMEM loads and stores are warp-collective, so
-        // the warp does this together; rows that keep their reference scale
-        // by 1.
-        const bool moves = mx > mref + kSlack;
-        if (__any_sync(kFull, moves)) {
-          const float mnew = moves ? mx : mref;
-          const float alpha = mref == -INFINITY ? 0.f : ex2(mref - mnew);
-          if (u > 0) {
-            const int mp = m - 1;
-            ok = wait_ok(bar_pv + 8 * (mp & 1), (mp >> 1) & 1, abort_flag, a.dev_error);
-            if (!ok) continue;
-            fence_after();
-#pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
-              uint32_t ou[32];
-              tmem_ld32_issue(trow + col_o + 32 * ch, ou);
-              tmem_ld_wait(ou);
-#pragma unroll
-              for (int i = 0; i < 32; ++i)
-                ou[i] = __float_as_uint(__uint_as_float(ou[i]) * alpha);
-              tmem_st32(trow + col_o + 32 * ch, ou);
+            for (int i = 0; i < 16; i += 2) {
+              if (decltype(kMax)::value && (i & 2) == 0) {
+                x0 = fmax3(x0, sv[ch][2 * i], sv[ch][2 * i + 1]);
+                x1 = fmax3(x1, sv[ch][2 * i + 2], sv[ch][2 * i + 3]);
+                x2 = fmax3(x2, sv[ch][2 * i + 4], sv[ch][2 * i + 5]);
+                x3 = fmax3(x3, sv[ch][2 * i + 6], sv[ch][2 * i + 7]);
+              }
+              const float2 xa = __ffma2_rn(make_float2(sv[ch][2 * i], sv[ch][2 * i + 1]), c2, n2);
+              const float2 xb =
+                  __ffma2_rn(make_float2(sv[ch][2 * i + 2], sv[ch][2 * i + 3]), c2, n2);
+              const float p0 = ex2(xa.x), p1 = ex2(xa.y), p2 = ex2(xb.x), p3 = ex2(xb.y);
+              la = __fadd2_rn(la, make_float2(p0, p1));
+              lb = __fadd2_rn(lb, make_float2(p2, p3));
+              if (PrefillPSplit<T>::value) {
+                tc::split2<T>(p0, p1, ph[i], pt[i]);
+                tc::split2<T>(p2, p3, ph[i + 1], pt[i + 1]);
+              } else {
+                ph[i] = tc::pack2<T>(p0, p1);
+                ph[i + 1] = tc::pack2<T>(p2, p3);
+              }
             }
+            tmem_st16(sp + 16 * ch, ph);
+            if (PrefillPSplit<T>::value) tmem_st16(sp + 32 + 16 * ch, pt);
           }
-          la = __fmul2_rn(la, make_float2(alpha, alpha));
-          lb = __fmul2_rn(lb, make_float2(alpha, alpha));
-          mref = mnew;
+        };
+        // Once every row of the warp has a reference, the exponentials are
+        // taken against it while the maximum is found; they stand unless some
+        // row's maximum rose by more than 2^kSlack (then the row sums are put
+        // back and the sub-tile is done again below, as for a first sub-tile).
+        // Either way the weights and sums are those of the plain order.
+        // (16-bit P without a tail only: the head + tail form would spill.)
+        bool done = false;
+        if (!PrefillPSplit<T>::value && __all_sync(kFull, mref != -INFINITY)) {
+          const float2 la0 = la, lb0 = lb;
+          exps(-mref, std::true_type{});
+          const float mr = fmax3(fmaxf(x0, x1), x2, x3);
+          const float m2 = mr == -INFINITY ? -INFINITY : mr * c;
+          if (!__any_sync(kFull, m2 > mref + kSlack)) {
+            done = true;
+          } else {
+            la = la0;
+            lb = lb0;
+            tmem_st_wait();  // the stores above land before the ones that replace them
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              x0 = fmax3(x0, sv[ch][i], sv[ch][i + 1]);
+              x1 = fmax3(x1, sv[ch][i + 2], sv[ch][i + 3]);
+              x2 = fmax3(x2, sv[ch][i + 4], sv[ch][i + 5]);
+              x3 = fmax3(x3, sv[ch][i + 6], sv[ch][i + 7]);
+            }
         }
-        const float neg = mref == -INFINITY ? 0.f : -mref;
-        // x = s c - reference, two at a time (packed fp32 FMA)
-        const float2 c2 = make_float2(c, c), n2 = make_float2(neg, neg);
-        // P over this sub-tile's score columns: head pairs in columns 0..31,
-        // tails in 32..63
+        if (!done) {
+          const float mx_raw = fmax3(fmaxf(x0, x1), x2, x3);
+          const float mx = mx_raw == -INFINITY ? -INFINITY : mx_raw * c;
+          // a row whose maximum rose by more than 2^kSlack takes it as its new
+          // reference and rescales its row of O_h once the half's previous
+          // P . V has completed.  TMEM loads and stores are warp-collective, so
+          // the warp does this together; rows that keep their reference scale
+          // by 1.
+          const bool moves = mx > mref + kSlack;
+          if (__any_sync(kFull, moves)) {
+            const float mnew = moves ? mx : mref;
+            const float alpha = mref == -INFINITY ? 0.f : ex2(mref - mnew);
+            if (u > 0) {
+              const int mp = m - 1;
+              ok = wait_ok(bar_pv + 8 * (mp & 1), (mp >> 1) & 1, abort_flag, a.dev_error);
+              if (!ok) continue;
+              fence_after();
+#pragma unroll 1
+              for (int ch = 0; ch < 4; ++ch) {
+                uint32_t ou[32];
+                tmem_ld32_issue(trow + col_o + 32 * ch, ou);
+                tmem_ld_wait(ou);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t ph[16], pt[16];
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            const float2 xa = __ffma2_rn(make_float2(sv[ch][2 * i], sv[ch][2 * i + 1]), c2, n2);
-            const float2 xb =
-                __ffma2_rn(make_float2(sv[ch][2 * i + 2], sv[ch][2 * i + 3]), c2, n2);
-            const float p0 = ex2(xa.x), p1 = ex2(xa.y), p2 = ex2(xb.x), p3 = ex2(xb.y);
-            la = __fadd2_rn(la, make_float2(p0, p1));
-            lb = __fadd2_rn(lb, make_float2(p2, p3));
-            if (PrefillPSplit<T>::value) {
-              tc::split2<T>(p0, p1, ph[i], pt[i]);
-              tc::split2<T>(p2, p3, ph[i + 1], pt[i + 1]);
-            } else {
-              ph[i] = tc::pack2<T>(p0, p1);
-              ph[i + 1] = tc::pack2<T>(p2, p3);
+                for (int i = 0; i < 32; ++i)
+                  ou[i] = __float_as_uint(__uint_as_float(ou[i]) * alpha);
+                tmem_st32(trow + col_o + 32 * ch, ou);
+              }
             }
+            la = __fmul2_rn(la, make_float2(alpha, alpha));
+            lb = __fmul2_rn(lb, make_float2(alpha, alpha));
+            mref = mnew;
           }
-          tmem_st16(sp + 16 * ch, ph);
-          if (PrefillPSplit<T>::value) tmem_st16(sp + 32 + 16 * ch, pt);
+          exps(mref == -INFINITY ? 0.f : -mref, std::false_type{});
         }
         tmem_st_wait();
         fence_before();
